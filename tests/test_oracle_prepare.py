@@ -1,0 +1,253 @@
+"""Pins for the oracle's preprocessing (RMSNorm, backbone, residual) and the
+fp64 reference GEMM, checked against closed forms and invariants that the
+SharQ decomposition implies (abstract, Section 1):
+
+* the backbone keeps the outliers: a backbone block's scale is the scale of
+  the whole window's amax (the group maximum is always kept);
+* |R| <= |h| (quantization never overshoots by more than the value);
+* h - deq(B) - deq(R) = R - deq(R) obeys the FP4 rounding bound;
+* inputs that are already N:M-sparse and FP4-representable give R == 0;
+* the reference GEMM equals (deq(B) + deq(R)) . deq(W)^T and tracks X . W^T.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from activation_sparsity_fp4_b200 import workloads
+
+FMTS = ["mxfp4", "nvfp4"]
+PATS = ["2:4", "4:8pair", "8:16"]
+
+
+def _rows(seed, t=24, k=512, outliers=True):
+    rng = np.random.default_rng(seed)
+    x = (0.5 * rng.standard_t(3, size=(t, k))).astype(np.float32)
+    if outliers:
+        x[:, rng.permutation(k)[:6]] *= 60.0
+    x[:, 5] = 0.0
+    return x
+
+
+# ------------------------------------------------------------------ RMSNorm
+def test_rmsnorm_against_fp64():
+    rng = np.random.default_rng(11)
+    for k in (256, 768, 4096, 5120, 14336):
+        x = (rng.standard_normal(k) * rng.uniform(0.1, 20)).astype(np.float32)
+        r = oracle.rms_rstd(x, 1e-6)
+        ref = 1.0 / math.sqrt(float(np.mean(x.astype(np.float64) ** 2)) + 1e-6)
+        assert abs(r - ref) <= 4e-7 * ref, (k, r, ref)
+
+
+def test_rmsnorm_constant_row_closed_form():
+    # x = c everywhere: mean(x^2) = c^2 exactly (power-of-two c keeps sums exact)
+    for c, k in ((1.0, 4096), (0.5, 768), (4.0, 5120)):
+        x = np.full(k, c, np.float32)
+        r = oracle.rms_rstd(x, 0.0)
+        assert r == np.float32(1.0 / c)
+
+
+def test_rmsnorm_eps_enters_once():
+    x = np.zeros(256, np.float32)
+    assert oracle.rms_rstd(x, 0.25) == 2.0
+
+
+def test_prepare_applies_norm_and_gamma():
+    rng = np.random.default_rng(12)
+    x = rng.standard_normal((4, 512)).astype(np.float32)
+    gamma = rng.uniform(0.5, 1.5, 512).astype(np.float32)
+    prep = oracle.prepare(x, "nvfp4", "4:8pair", gamma=gamma, eps=1e-6, want_float=True)
+    ref = x.astype(np.float64) / np.sqrt(np.mean(x.astype(np.float64) ** 2, axis=1, keepdims=True) + 1e-6)
+    ref *= gamma
+    np.testing.assert_allclose(prep["h"], ref, rtol=2e-6, atol=0)
+
+
+# ------------------------------------------------------------- invariants
+def _window_scale_codes(h, fmt, b, g_enc):
+    """Scale code of each 2b-logical window computed from the window's amax alone."""
+    t, k = h.shape
+    out = np.zeros((t, k // (2 * b)), np.uint8)
+    a = np.abs(h).reshape(t, k // (2 * b), 2 * b).max(axis=2)
+    for r in range(t):
+        for w in range(k // (2 * b)):
+            amax = float(a[r, w])
+            if fmt == "mxfp4":
+                e = (math.frexp(amax)[1] - 1 - 2) if amax > 0 else -127
+                out[r, w] = max(-127, min(127, e)) + 127
+            else:
+                out[r, w] = oracle.e4m3_encode([np.float32(np.float32(amax / np.float32(6.0)) * np.float32(g_enc))])[0]
+    return out
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("pat", PATS)
+def test_backbone_scale_is_window_amax_scale(fmt, pat):
+    x = _rows(20)
+    prep = oracle.prepare(x, fmt, pat, want_float=True)
+    b = oracle.block_size(fmt)
+    exp = _window_scale_codes(prep["h"], fmt, b, prep["tensor"][1])
+    np.testing.assert_array_equal(prep["bb_scales"], exp)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("pat", PATS)
+def test_residual_never_exceeds_input(fmt, pat):
+    x = _rows(21)
+    prep = oracle.prepare(x, fmt, pat, want_float=True)
+    h, bdeq = prep["h"], prep["bdeq"]
+    keep = oracle.mask(h, pat).astype(bool)
+    res = np.where(keep, h - bdeq, h).astype(np.float32)
+    slack = 1.0 if fmt == "mxfp4" else 1.0 + 2.0 ** -21
+    assert np.all(np.abs(res) <= np.abs(h) * slack)
+    # the backbone is exact only on kept positions and zero elsewhere
+    assert np.all(bdeq[~keep] == 0.0)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("pat", PATS)
+def test_decomposition_error_bound(fmt, pat):
+    """|h - deq(B) - deq(R)| = |R - deq(R)| <= max(s/4, |R|/4) per element, s = the
+    residual block's decoded scale (times g_dec for NVFP4): the E2M1 rounding bound
+    including saturation on (6, 8)."""
+    x = _rows(22)
+    prep = oracle.prepare(x, fmt, pat, want_float=True)
+    h, bdeq, rdeq = (prep[n].astype(np.float64) for n in ("h", "bdeq", "rdeq"))
+    keep = oracle.mask(prep["h"], pat).astype(bool)
+    r = np.where(keep, (prep["h"] - prep["bdeq"]).astype(np.float32), prep["h"]).astype(np.float64)
+    b = oracle.block_size(fmt)
+    sc = np.repeat(prep["res_scales"], b, axis=1)
+    if fmt == "mxfp4":
+        s = np.vectorize(lambda c: math.ldexp(1.0, int(c) - 127))(sc)
+        slack = 1.0
+    else:
+        s = oracle.e4m3_decode(sc.ravel()).reshape(sc.shape).astype(np.float64) * float(prep["tensor"][2])
+        slack = 1.0 + 1e-5
+    err = np.abs(h - bdeq - rdeq)
+    assert np.all(err <= np.maximum(s / 4, np.abs(r) / 4) * slack + 1e-30)
+    # and the two paths together are much closer to h than the backbone alone
+    assert np.linalg.norm(h - bdeq - rdeq) < 0.2 * np.linalg.norm(h - bdeq)
+
+
+def _representable_sparse_rows(fmt, pat, t=8, k=512, seed=23):
+    """Rows that are already N:M-sparse (dropped entries exactly 0, so the kept
+    nonzeros win the tie rule) and whose values in each backbone window of 2b
+    logical positions are E2M1 codes times one power of two 2^j, with one |code|
+    = 6 per window.  For NVFP4 the values carry the decode scale g_dec = 1/16
+    that a caller-given tensor amax of 2688/16 produces, so every step of the
+    quantization is exact and the residual must vanish."""
+    rng = np.random.default_rng(seed)
+    b = oracle.block_size(fmt)
+    m = {"2:4": 4, "4:8pair": 8, "8:16": 16}[pat]
+    grid = np.array([0.5, 1.0, 1.5, 2.0, 3.0, 4.0])
+    x = np.zeros((t, k), np.float32)
+    for r in range(t):
+        for g0 in range(0, k, m):
+            if pat == "4:8pair":
+                pairs = np.sort(rng.choice(4, 2, replace=False))
+                pos = np.concatenate([[2 * p, 2 * p + 1] for p in pairs])
+            else:
+                pos = np.sort(rng.choice(m, m // 2, replace=False))
+            x[r, g0 + pos] = rng.choice(grid, pos.size) * rng.choice([-1, 1], pos.size)
+        for w0 in range(0, k, 2 * b):
+            win = x[r, w0:w0 + 2 * b]
+            nz = np.flatnonzero(win)
+            win[nz[0]] = 6.0 * np.sign(win[nz[0]])
+            j = int(rng.integers(-6, 6)) if fmt == "mxfp4" else int(rng.integers(-5, 9))
+            scale = 2.0 ** j if fmt == "mxfp4" else 2.0 ** j / 16.0
+            x[r, w0:w0 + 2 * b] = win * np.float32(scale)
+    return x
+
+
+@pytest.mark.parametrize("pat", PATS)
+def test_zero_residual_on_representable_sparse_input_mxfp4(pat):
+    x = _representable_sparse_rows("mxfp4", pat)
+    prep = oracle.prepare(x, "mxfp4", pat, want_float=True)
+    np.testing.assert_array_equal(prep["bdeq"], x)
+    assert np.all(prep["res_codes"] == 0)
+    assert np.all(prep["rdeq"] == 0)
+
+
+@pytest.mark.parametrize("pat", PATS)
+def test_zero_residual_on_representable_sparse_input_nvfp4(pat):
+    x = _representable_sparse_rows("nvfp4", pat, seed=24)
+    prep = oracle.prepare(x, "nvfp4", pat, act_amax=2688.0 / 16.0, want_float=True)
+    assert prep["tensor"][1] == 16.0 and prep["tensor"][2] == 1.0 / 16.0
+    np.testing.assert_array_equal(prep["bdeq"], x)
+    assert np.all(prep["res_codes"] == 0)
+    assert np.all(prep["rdeq"] == 0)
+
+
+# --------------------------------------------------------------- weights
+@pytest.mark.parametrize("fmt", FMTS)
+def test_weight_quantization_bound_and_shared_block(fmt):
+    rng = np.random.default_rng(30)
+    w = (rng.standard_normal((64, 512)) * 0.02).astype(np.float32)
+    wq = oracle.quantize_weight(w, fmt)
+    wu = oracle.decode_weight(wq) * float(wq["tensor"][2])
+    bw = 2 * oracle.block_size(fmt)
+    assert wq["scales"].shape == (64, 512 // bw)
+    rel = np.linalg.norm(wu - w) / np.linalg.norm(w)
+    assert 0.01 < rel < 0.15
+    # one block of the weight, quantized alone, gives the same codes
+    sc, codes = oracle.quant_block(w[3, bw:2 * bw], fmt, float(wq["tensor"][1]))
+    assert sc == wq["scales"][3, 1]
+    packed = wq["codes"][3, bw // 2:bw]
+    unpacked = np.stack([packed & 15, packed >> 4], axis=1).ravel()
+    np.testing.assert_array_equal(unpacked, codes)
+
+
+# ------------------------------------------------------------ reference GEMM
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("pat", PATS)
+def test_linear_ref_matches_float_operands(fmt, pat):
+    x = _rows(40, t=16, k=256)
+    rng = np.random.default_rng(41)
+    w = (rng.standard_normal((128, 256)) * 0.02).astype(np.float32)
+    prep = oracle.prepare(x, fmt, pat, want_float=True)
+    wq = oracle.quantize_weight(w, fmt)
+    y = oracle.linear_ref(prep, wq)
+    wd = oracle.decode_weight(wq) * float(wq["tensor"][2])
+    y2 = (prep["bdeq"].astype(np.float64) + prep["rdeq"].astype(np.float64)) @ wd.T
+    assert np.linalg.norm(y - y2) <= 1e-6 * np.linalg.norm(y2)
+    # and it approximates the unquantized product: FP4 error, not a wiring error
+    y0 = prep["h"].astype(np.float64) @ w.astype(np.float64).T
+    assert np.linalg.norm(y - y0) < 0.12 * np.linalg.norm(y0)
+
+
+def test_linear_ref_exact_on_representable_input():
+    x = _representable_sparse_rows("mxfp4", "2:4", t=8, k=256)
+    rng = np.random.default_rng(42)
+    w = (rng.standard_normal((128, 256)) * 0.02).astype(np.float32)
+    prep = oracle.prepare(x, "mxfp4", "2:4")
+    wq = oracle.quantize_weight(w, "mxfp4")
+    wd = oracle.decode_weight(wq)
+    np.testing.assert_array_equal(oracle.linear_ref(prep, wq), x.astype(np.float64) @ wd.T)
+
+
+def test_sharq_beats_dense_fp4_on_outlier_rows():
+    """Informative check of the pages' qualitative claim on synthetic data: the
+    sparse backbone + residual is closer to the fp32 product than plain FP4."""
+    cfg = workloads.tiny()
+    x, w = cfg["x"], cfg["w"]
+    prep = oracle.prepare(x, "mxfp4", "2:4")
+    wq = oracle.quantize_weight(w, "mxfp4")
+    y = oracle.linear_ref(prep, wq)
+    wd = oracle.decode_weight(wq)
+    y0 = x.astype(np.float64) @ w.astype(np.float64).T
+    # dense FP4 only: the residual path with an empty backbone (blocks of 32, OCP MX)
+    xq = np.zeros_like(x, dtype=np.float64)
+    for r in range(x.shape[0]):
+        for b0 in range(0, x.shape[1], 32):
+            sc, codes = oracle.quant_block(x[r, b0:b0 + 32], "mxfp4")
+            xq[r, b0:b0 + 32] = oracle.e2m1_decode(codes) * math.ldexp(1.0, sc - 127)
+    y_dense = xq @ wd.T
+    assert np.linalg.norm(y - y0) < np.linalg.norm(y_dense - y0)
+
+
+def test_threaded_prepare_is_bit_identical():
+    cfg = workloads.q_proj(t=64)
+    a = oracle.prepare(cfg["x"], "nvfp4", "4:8pair", gamma=cfg["gamma"], threads=1)
+    b = oracle.prepare(cfg["x"], "nvfp4", "4:8pair", gamma=cfg["gamma"], threads=4)
+    for n in ("meta", "bb_codes", "bb_scales", "res_codes", "res_scales", "tensor"):
+        np.testing.assert_array_equal(a[n], b[n])
