@@ -1,0 +1,387 @@
+// gemm.cuh -- the two GEMMs of the SharQ layer in one persistent tcgen05 kernel.
+//
+// SharQ (arXiv 2606.26587), abstract and Section 1: a sparse FP4 GEMM runs over
+// the compressed backbone and its N:M metadata, a dense FP4 GEMM runs over the
+// residual and "accumulates directly into the sparse output", and "both paths
+// share one FP4 weight load with path-specific scale views".  Here both MMAs of
+// a K tile read the SAME shared-memory copy of the weight tile (one TMA load)
+// and write the SAME tensor-memory accumulator; each path brings its own
+// scale-factor view of the weight (one scale per 2b logical K for the sparse
+// MMA, the same scales repeated per b for the dense MMA).
+//
+// Structure (one CTA per SM, 6 warps):
+//   warp 0      TMA producer: weight, residual, backbone and metadata tiles by
+//               cp.async.bulk.tensor, scale factors by 1-D cp.async.bulk;
+//   warp 1      TMEM owner and MMA issuer (one thread): tcgen05.cp of scales and
+//               metadata into tensor memory, tcgen05.mma.sp over the backbone,
+//               tcgen05.mma over the residual, tcgen05.commit to free stages;
+//   warps 2-5   epilogue: tcgen05.ld of the fp32 accumulator, times the tensor
+//               scales g_dec(x) * g_dec(w), stores y (bf16 or fp32).
+// Tiles are 128 x 256 outputs; a stage is 256 logical K.  Every wait is
+// bounded in time and reports through the device error word.
+#pragma once
+#include <cuda_bf16.h>
+
+#include "prep.cuh"
+#include "ptx.cuh"
+
+namespace sharq {
+
+enum { GK_NVF4 = 0, GK_MXF4 = 1 };
+
+template <int KIND, bool SPARSE>
+struct GemmCfg {
+  static constexpr int BM = 128, BN = 256, BK = 256;
+  static constexpr int kDenseMmaK = 64;    // logical K per dense MMA
+  static constexpr int kSparseMmaK = 128;  // logical K per sparse MMA
+  static constexpr int kVecDense = (KIND == GK_NVF4) ? 16 : 32;  // logical K per scale, dense MMA
+  static constexpr int kVecSparse = 2 * kVecDense;                // logical K per scale, sparse MMA
+  static constexpr int kRowDense = BK / 2;                         // bytes per row per stage: W, R
+  static constexpr int kRowB = SPARSE ? BK / 4 : BK / 2;           // backbone (compressed or dense)
+  static constexpr int kRowE = SPARSE ? 16 : 0;                    // metadata (4:8 pair)
+  static constexpr int kWBytes = BN * kRowDense;
+  static constexpr int kRBytes = BM * kRowDense;
+  static constexpr int kBBytes = BM * kRowB;
+  static constexpr int kEBytes = BM * kRowE;
+  static constexpr int kChunksR = BK / kVecDense / 4;                  // 512-byte scale chunks per stage
+  static constexpr int kChunksB = SPARSE ? BK / kVecSparse / 4 : kChunksR;
+  static constexpr int kSfaR = kChunksR * 512;
+  static constexpr int kSfbD = 2 * kChunksR * 512;  // two 128-row blocks of the weight
+  static constexpr int kSfaB = kChunksB * 512;
+  static constexpr int kSfbS = SPARSE ? 2 * kChunksB * 512 : 0;
+  // stage layout (offsets in bytes)
+  static constexpr int oW = 0;
+  static constexpr int oR = oW + kWBytes;
+  static constexpr int oB = oR + kRBytes;
+  static constexpr int oE = oB + kBBytes;
+  static constexpr int oSfaR = oE + kEBytes;
+  static constexpr int oSfbD = oSfaR + kSfaR;
+  static constexpr int oSfaB = oSfbD + kSfbD;
+  static constexpr int oSfbS = oSfaB + kSfaB;
+  static constexpr int kStageBytes = ((oSfbS + kSfbS + 1023) / 1024) * 1024;
+  static constexpr int kStages = (SPARSE && KIND == GK_NVF4) ? 3 : 3;
+  static constexpr uint32_t kTx = kWBytes + kRBytes + kBBytes + kEBytes + kSfaR + kSfbD + kSfaB + kSfbS;
+  // tensor memory columns: accumulator, then two slots of scales + metadata
+  static constexpr int cSfaR = 0;
+  static constexpr int cSfbD = cSfaR + 4 * kChunksR;
+  static constexpr int cSfaB = cSfbD + 8 * kChunksR;
+  static constexpr int cSfbS = cSfaB + 4 * kChunksB;
+  static constexpr int cE = cSfbS + (SPARSE ? 8 * kChunksB : 0);
+  static constexpr int kSlotCols = cE + (SPARSE ? 4 : 0);
+  static constexpr int kTmemCols = 512;
+  static_assert(BN + 2 * kSlotCols <= kTmemCols, "tensor memory budget");
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+  // instruction descriptor (block-scaled kinds): E2M1 x E2M1, K-major, M=128, N=256
+  static constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                     ((KIND == GK_MXF4 ? 1u : 0u) << 23) | ((uint32_t)(BM >> 4) << 24);
+  static constexpr uint32_t kIdescSp = kIdesc | (1u << 2);
+};
+
+struct GemmParams {
+  int64_t t;          // rows of y to store (rows >= t are computed but not stored)
+  int64_t t_pad;      // rows of the prepared operands (multiple of 128)
+  int64_t n, k;
+  int32_t experts;    // 1 = plain; >1 grouped by group_offsets
+  const int32_t* group_offsets;  // device, experts + 1 (grouped only)
+  const uint8_t* sf_res;         // tiled, t_pad rows, k/b scales
+  const uint8_t* sf_bb;          // tiled, t_pad rows, k/(2b) scales (dense backbone: k/b)
+  const uint8_t* sf_w_dense;     // per expert tiled, n rows, k/b
+  const uint8_t* sf_w_sparse;    // per expert tiled, n rows, k/(2b)
+  const float* tensor_x;         // [amax, g_enc, g_dec]
+  const float* tensor_w;         // experts * 3
+  void* y;
+  int y_bf16;
+  int paths;          // bit 0 sparse backbone, bit 1 dense residual
+  uint64_t timeout_ns;
+};
+
+struct GemmMaps {
+  CUtensorMap w, r, b, e;
+};
+
+template <int KIND, bool SPARSE>
+__global__ void __launch_bounds__(192, 1) gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
+  using C = GemmCfg<KIND, SPARSE>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* acc_full = empty + C::kStages;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* drain = acc_empty + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; s++) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 4);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, C::kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch(&maps.w);
+    tma_prefetch(&maps.r);
+    tma_prefetch(&maps.b);
+    if (SPARSE) tma_prefetch(&maps.e);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  const int m_tiles = (int)(p.t_pad / C::BM);
+  const int n_tiles = (int)(p.n / C::BN);
+  const int num_tiles = m_tiles * n_tiles;
+  const int k_tiles = (int)(p.k / C::BK);
+  const int64_t sd_per_row = p.k / C::kVecDense;                    // dense-view scales per row
+  const int64_t sb_per_row = SPARSE ? p.k / C::kVecSparse : sd_per_row;
+  const int64_t wsd_bytes = tiled_sf_bytes(p.n, sd_per_row);
+  const int64_t wss_bytes = tiled_sf_bytes(p.n, p.k / C::kVecSparse);
+  const bool run_sparse = (p.paths & 1) != 0;
+  const bool run_dense = (p.paths & 2) != 0;
+
+  // expert of an m tile (grouped form); -1 = rows outside every group
+  auto tile_expert = [&](int64_t m0) -> int {
+    if (p.experts <= 1) return 0;
+    int lo = 0, hi = p.experts;  // find e with off[e] <= m0 < off[e+1]
+    if (m0 >= (int64_t)__ldg(p.group_offsets + p.experts)) return -1;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if ((int64_t)__ldg(p.group_offsets + mid) <= m0) lo = mid;
+      else hi = mid;
+    }
+    return lo;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0, issued_par = 0;  // per stage: ever issued / parity of the last batch
+      for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x) {
+        const int mt = tile % m_tiles, nt = tile / m_tiles;
+        const int64_t m0 = (int64_t)mt * C::BM;
+        const int e = tile_expert(m0);
+        if (e < 0) continue;
+        const int32_t wrow = (int32_t)(e * p.n + (int64_t)nt * C::BN);
+        for (int kt = 0; kt < k_tiles; kt++) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, p.timeout_ns, abort_flag)) { *abort_flag = 1; break; }
+          uint8_t* sb = smem + stage * C::kStageBytes;
+          mbar_arrive_expect_tx(&full[stage], C::kTx);
+          tma_load_2d(sb + C::oW, &maps.w, kt * C::kRowDense, wrow, &full[stage]);
+          tma_load_2d(sb + C::oR, &maps.r, kt * C::kRowDense, (int32_t)m0, &full[stage]);
+          tma_load_2d(sb + C::oB, &maps.b, kt * C::kRowB, (int32_t)m0, &full[stage]);
+          if constexpr (SPARSE) tma_load_2d(sb + C::oE, &maps.e, kt * C::kRowE, (int32_t)m0, &full[stage]);
+          // scale chunks: contiguous per 128-row block in the tiled layout
+          const int64_t sd_blocks = (sd_per_row + 3) / 4, sb_blocks = (sb_per_row + 3) / 4;
+          bulk_load(sb + C::oSfaR, p.sf_res + ((m0 / 128) * sd_blocks + (int64_t)kt * C::kChunksR) * 512, C::kSfaR,
+                    &full[stage]);
+          bulk_load(sb + C::oSfaB, p.sf_bb + ((m0 / 128) * sb_blocks + (int64_t)kt * C::kChunksB) * 512, C::kSfaB,
+                    &full[stage]);
+          const uint8_t* wd = p.sf_w_dense + e * wsd_bytes;
+          const int64_t nb = (int64_t)nt * 2;
+#pragma unroll
+          for (int rb = 0; rb < 2; rb++)
+            bulk_load(sb + C::oSfbD + rb * C::kChunksR * 512,
+                      wd + ((nb + rb) * sd_blocks + (int64_t)kt * C::kChunksR) * 512, C::kChunksR * 512, &full[stage]);
+          if constexpr (SPARSE) {
+            const uint8_t* ws = p.sf_w_sparse + e * wss_bytes;
+            const int64_t ss_blocks = (p.k / C::kVecSparse + 3) / 4;
+#pragma unroll
+            for (int rb = 0; rb < 2; rb++)
+              bulk_load(sb + C::oSfbS + rb * C::kChunksB * 512,
+                        ws + ((nb + rb) * ss_blocks + (int64_t)kt * C::kChunksB) * 512, C::kChunksB * 512,
+                        &full[stage]);
+          }
+          issued |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (*abort_flag) {
+        // let every load already issued land before the block can exit
+        for (int i = 0; i < C::kStages; i++)
+          if ((issued >> i) & 1u) (void)mbar_wait(&full[i], (issued_par >> i) & 1u, 1000000000ull, nullptr, true);
+      }
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------------- MMA
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      const uint32_t acc = tmem_base;
+      for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x, it++) {
+        const int mt = tile % m_tiles;
+        if (tile_expert((int64_t)mt * C::BM) < 0) { it--; continue; }
+        if (!mbar_wait(acc_empty, (it & 1) ^ 1, p.timeout_ns, abort_flag)) { *abort_flag = 1; break; }
+        tc_fence_after();
+        uint32_t accumulate = 0;
+        for (int kt = 0; kt < k_tiles; kt++) {
+          if (!mbar_wait(&full[stage], phase, p.timeout_ns, abort_flag)) { *abort_flag = 1; break; }
+          tc_fence_after();
+          const uint8_t* sb = smem + stage * C::kStageBytes;
+          const uint32_t slot = tmem_base + C::BN + (uint32_t)((kt & 1) * C::kSlotCols);
+          // scale factors and metadata -> tensor memory
+#pragma unroll
+          for (int c = 0; c < C::kChunksR; c++) {
+            tc_cp_32x128b_warpx4(slot + C::cSfaR + 4 * c, smem_desc(smem_u32(sb + C::oSfaR + 512 * c), 0, 128, 0));
+#pragma unroll
+            for (int rb = 0; rb < 2; rb++)
+              tc_cp_32x128b_warpx4(slot + C::cSfbD + 8 * c + 4 * rb,
+                                   smem_desc(smem_u32(sb + C::oSfbD + (rb * C::kChunksR + c) * 512), 0, 128, 0));
+          }
+#pragma unroll
+          for (int c = 0; c < C::kChunksB; c++) {
+            tc_cp_32x128b_warpx4(slot + C::cSfaB + 4 * c, smem_desc(smem_u32(sb + C::oSfaB + 512 * c), 0, 128, 0));
+            if constexpr (SPARSE) {
+#pragma unroll
+              for (int rb = 0; rb < 2; rb++)
+                tc_cp_32x128b_warpx4(slot + C::cSfbS + 8 * c + 4 * rb,
+                                     smem_desc(smem_u32(sb + C::oSfbS + (rb * C::kChunksB + c) * 512), 0, 128, 0));
+            }
+          }
+          if constexpr (SPARSE) tc_cp_128x128b(slot + C::cE, smem_desc(smem_u32(sb + C::oE), 0, 128, 0));
+
+          const uint32_t w_base = smem_u32(sb + C::oW);
+          if (run_sparse) {
+            if constexpr (SPARSE) {
+              // backbone: sparse MMAs, K = 128 logical each (64 stored FP4 = 32 bytes of A)
+#pragma unroll
+              for (int kb = 0; kb < C::BK / C::kSparseMmaK; kb++) {
+                const int s0 = kb * (C::kSparseMmaK / C::kVecSparse);
+                const uint32_t chunk = s0 / 4, byte = s0 % 4;
+                const uint32_t idesc = C::kIdescSp | (byte << 29) | (byte << 4);
+                const uint64_t a = smem_desc(smem_u32(sb + C::oB) + kb * 32, 16, 512, 4);   // 64B swizzle
+                const uint64_t b = smem_desc(w_base + kb * 64, 16, 1024, 2);                // 128B swizzle
+                const uint32_t sfa = (slot + C::cSfaB + 4 * chunk) | (byte << 30);
+                const uint32_t sfb = (slot + C::cSfbS + 8 * chunk) | (byte << 30);
+                if constexpr (KIND == GK_NVF4) mma_nvf4_sp(acc, a, b, slot + C::cE + 2 * kb, idesc, sfa, sfb, accumulate);
+                else mma_mxf4_sp(acc, a, b, slot + C::cE + 2 * kb, idesc, sfa, sfb, accumulate);
+                accumulate = 1;
+              }
+            } else {
+              // dense backbone (8:16): same as the residual path over the expanded backbone
+#pragma unroll
+              for (int kb = 0; kb < C::BK / C::kDenseMmaK; kb++) {
+                const int s0 = kb * (C::kDenseMmaK / C::kVecDense);
+                const uint32_t chunk = s0 / 4, byte = s0 % 4;
+                const uint32_t idesc = C::kIdesc | (byte << 29) | (byte << 4);
+                const uint64_t a = smem_desc(smem_u32(sb + C::oB) + kb * 32, 16, 1024, 2);
+                const uint64_t b = smem_desc(w_base + kb * 32, 16, 1024, 2);
+                const uint32_t sfa = (slot + C::cSfaB + 4 * chunk) | (byte << 30);
+                const uint32_t sfb = (slot + C::cSfbD + 8 * chunk) | (byte << 30);
+                if constexpr (KIND == GK_NVF4) mma_nvf4(acc, a, b, idesc, sfa, sfb, accumulate);
+                else mma_mxf4(acc, a, b, idesc, sfa, sfb, accumulate);
+                accumulate = 1;
+              }
+            }
+          }
+          if (run_dense) {
+            // residual: dense MMAs, K = 64 each (32 bytes of A and of W), same W tile
+#pragma unroll
+            for (int kb = 0; kb < C::BK / C::kDenseMmaK; kb++) {
+              const int s0 = kb * (C::kDenseMmaK / C::kVecDense);
+              const uint32_t chunk = s0 / 4, byte = s0 % 4;
+              const uint32_t idesc = C::kIdesc | (byte << 29) | (byte << 4);
+              const uint64_t a = smem_desc(smem_u32(sb + C::oR) + kb * 32, 16, 1024, 2);
+              const uint64_t b = smem_desc(w_base + kb * 32, 16, 1024, 2);
+              const uint32_t sfa = (slot + C::cSfaR + 4 * chunk) | (byte << 30);
+              const uint32_t sfb = (slot + C::cSfbD + 8 * chunk) | (byte << 30);
+              if constexpr (KIND == GK_NVF4) mma_nvf4(acc, a, b, idesc, sfa, sfb, accumulate);
+              else mma_mxf4(acc, a, b, idesc, sfa, sfb, accumulate);
+              accumulate = 1;
+            }
+          }
+          tc_commit(&empty[stage]);
+          if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+        }
+        if (*abort_flag) break;
+        tc_commit(acc_full);
+      }
+      // every tcgen05 op of this thread is complete before tensor memory is freed
+      tc_commit(drain);
+      (void)mbar_wait(drain, 0, 1000000000ull, nullptr, true);
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    int it = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, it++) {
+      const int mt = tile % m_tiles, nt = tile / m_tiles;
+      const int64_t m0 = (int64_t)mt * C::BM;
+      const int e = tile_expert(m0);
+      if (e < 0) { it--; continue; }
+      if (!mbar_wait(acc_full, it & 1, p.timeout_ns, abort_flag)) { *abort_flag = 1; break; }
+      if (*abort_flag) break;
+      tc_fence_after();
+      const float alpha = __fmul_rn(__ldg(p.tensor_x + 2), __ldg(p.tensor_w + 3 * e + 2));
+      const int64_t row = m0 + 32 * q + lane;
+      const bool st = row < p.t;
+      const int64_t n0 = (int64_t)nt * C::BN;
+#pragma unroll 1
+      for (int c = 0; c < C::BN / 32; c++) {
+        uint32_t v[32];
+        tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(32 * c), v);
+        if (st) {
+          if (p.y_bf16) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int j = 0; j < 16; j++) {
+              __nv_bfloat162 h2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[2 * j]), alpha),
+                                                        __fmul_rn(__uint_as_float(v[2 * j + 1]), alpha));
+              pk[j] = *reinterpret_cast<uint32_t*>(&h2);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.y) + row * p.n + n0 + 32 * c);
+#pragma unroll
+            for (int j = 0; j < 4; j++) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+          } else {
+            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.y) + row * p.n + n0 + 32 * c);
+#pragma unroll
+            for (int j = 0; j < 8; j++)
+              dst[j] = make_float4(__fmul_rn(__uint_as_float(v[4 * j]), alpha),
+                                   __fmul_rn(__uint_as_float(v[4 * j + 1]), alpha),
+                                   __fmul_rn(__uint_as_float(v[4 * j + 2]), alpha),
+                                   __fmul_rn(__uint_as_float(v[4 * j + 3]), alpha));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// Wait on a flag that nothing sets: exercises the bounded-wait failure path.
+__global__ void selftest_wait_kernel(uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    (void)mbar_wait(&bar, 0, timeout_ns);
+  }
+}
+
+}  // namespace sharq

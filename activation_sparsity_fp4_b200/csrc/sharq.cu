@@ -1,0 +1,409 @@
+// sharq.cu -- C ABI of the SharQ sparse-dense FP4 linear layer for sm_100a.
+// One translation unit: the kernels (prep.cuh, gemm.cuh) and the host code
+// that validates arguments, encodes TMA descriptors and launches them.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/sharq.h"
+#include "gemm.cuh"
+#include "prep.cuh"
+
+using namespace sharq;
+
+namespace {
+
+thread_local std::string g_last_error;
+thread_local uint64_t g_launches = 0;
+
+sharq_status fail(sharq_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+#define SHARQ_CUDA(call)                                                                        \
+  do {                                                                                          \
+    cudaError_t e_ = (call);                                                                    \
+    if (e_ != cudaSuccess) return fail(SHARQ_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+sharq_status launched() {
+  g_launches++;
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(SHARQ_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e));
+  return SHARQ_OK;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
+
+int fmt_block(sharq_format f) { return f == SHARQ_NVFP4 ? 16 : 32; }
+
+int64_t meta_row_bytes(int64_t k, sharq_pattern p) { return p == SHARQ_NM_4_8_PAIR ? k / 16 : k / 8; }
+
+uint64_t wait_timeout_ns() {
+  static uint64_t v = [] {
+    const char* s = getenv("SHARQ_WAIT_TIMEOUT_NS");
+    return s ? strtoull(s, nullptr, 10) : 2000000000ull;
+  }();
+  return v;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// 2-D byte tensor [rows][row_bytes] with a (box_bytes x box_rows) box.
+sharq_status make_map(CUtensorMap* map, const void* base, int64_t row_bytes, int64_t rows, int box_bytes, int box_rows,
+                      CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(SHARQ_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  cuuint32_t box[2] = {(cuuint32_t)box_bytes, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SHARQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return SHARQ_OK;
+}
+
+sharq_status check_shape(int64_t k, int64_t n_or_t, bool is_n) {
+  if (k <= 0 || k % 256 != 0) return fail(SHARQ_ERR_INVALID, "k=%lld must be a positive multiple of 256", (long long)k);
+  if (k > 16384) return fail(SHARQ_ERR_UNSUPPORTED, "k=%lld above 16384", (long long)k);
+  if (is_n && (n_or_t <= 0 || n_or_t % 256 != 0))
+    return fail(SHARQ_ERR_INVALID, "n=%lld must be a positive multiple of 256", (long long)n_or_t);
+  if (!is_n && n_or_t <= 0) return fail(SHARQ_ERR_INVALID, "t=%lld must be positive", (long long)n_or_t);
+  return SHARQ_OK;
+}
+
+// ---------------------------------------------------------------- launchers
+template <int FMT, int PAT, bool NORM, bool XBF16>
+sharq_status launch_prep(const PrepParams& pp, cudaStream_t s) {
+  const int units = (int)(pp.k / 32);
+  const int tpr = (int)round_up(units, 32);
+  const int rpb = tpr >= 512 ? 1 : 512 / tpr;
+  const int rpb_c = rpb > 16 ? 16 : rpb;
+  dim3 block(tpr, rpb_c);
+  dim3 grid((unsigned)((pp.t_pad + rpb_c - 1) / rpb_c));
+  prep_kernel<FMT, PAT, NORM, XBF16><<<grid, block, 0, s>>>(pp, rpb_c, tpr);
+  return launched();
+}
+
+template <bool NORM, bool XBF16>
+sharq_status launch_amax(const void* x, const void* gamma, float eps, int64_t t, int64_t k, float* out,
+                         cudaStream_t s) {
+  const int units = (int)(k / 32);
+  const int tpr = (int)round_up(units, 32);
+  const int rpb = tpr >= 512 ? 1 : (512 / tpr > 16 ? 16 : 512 / tpr);
+  const int64_t groups = (t + rpb - 1) / rpb;
+  const int64_t cap = (int64_t)sm_count() * 4;
+  dim3 block(tpr, rpb);
+  dim3 grid((unsigned)(groups < cap ? groups : cap));
+  amax_kernel<NORM, XBF16><<<grid, block, 0, s>>>(x, gamma, eps, t, k, out, rpb, tpr);
+  return launched();
+}
+
+template <int FMT, int PAT, bool NORM>
+sharq_status prep_dispatch_x(const PrepParams& pp, bool xbf16, cudaStream_t s) {
+  return xbf16 ? launch_prep<FMT, PAT, NORM, true>(pp, s) : launch_prep<FMT, PAT, NORM, false>(pp, s);
+}
+template <int FMT, int PAT>
+sharq_status prep_dispatch_n(const PrepParams& pp, bool norm, bool xbf16, cudaStream_t s) {
+  return norm ? prep_dispatch_x<FMT, PAT, true>(pp, xbf16, s) : prep_dispatch_x<FMT, PAT, false>(pp, xbf16, s);
+}
+template <int FMT>
+sharq_status prep_dispatch_p(const PrepParams& pp, int pat, bool norm, bool xbf16, cudaStream_t s) {
+  switch (pat) {
+    case PAT_24: return prep_dispatch_n<FMT, PAT_24>(pp, norm, xbf16, s);
+    case PAT_48P: return prep_dispatch_n<FMT, PAT_48P>(pp, norm, xbf16, s);
+    default: return prep_dispatch_n<FMT, PAT_816>(pp, norm, xbf16, s);
+  }
+}
+
+template <int KIND, bool SPARSE>
+sharq_status launch_gemm(const GemmMaps& maps, const GemmParams& gp, cudaStream_t s) {
+  using C = GemmCfg<KIND, SPARSE>;
+  static bool configured = false;
+  if (!configured) {
+    SHARQ_CUDA(cudaFuncSetAttribute(gemm_kernel<KIND, SPARSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    C::kSmemBytes));
+    configured = true;
+  }
+  const int tiles = (int)(gp.t_pad / C::BM) * (int)(gp.n / C::BN);
+  const int sms = sm_count();
+  dim3 grid(tiles < sms ? tiles : sms);
+  gemm_kernel<KIND, SPARSE><<<grid, 192, C::kSmemBytes, s>>>(maps, gp);
+  return launched();
+}
+
+sharq_status check_prepared(const sharq_prepared* a) {
+  if (!a) return fail(SHARQ_ERR_INVALID, "prepared activations: NULL");
+  sharq_status st = check_shape(a->k, a->t, false);
+  if (st != SHARQ_OK) return st;
+  if (a->fmt != SHARQ_MXFP4 && a->fmt != SHARQ_NVFP4) return fail(SHARQ_ERR_INVALID, "bad format %d", (int)a->fmt);
+  if (a->pat < SHARQ_NM_2_4 || a->pat > SHARQ_NM_8_16) return fail(SHARQ_ERR_INVALID, "bad pattern %d", (int)a->pat);
+  const void* ptrs[6] = {a->meta, a->bb_codes, a->bb_scales, a->res_codes, a->res_scales, a->tensor};
+  for (int i = 0; i < 6; i++) {
+    if (!ptrs[i]) return fail(SHARQ_ERR_INVALID, "prepared buffer %d is NULL", i);
+    if (!aligned(ptrs[i], 16)) return fail(SHARQ_ERR_INVALID, "prepared buffer %d is not 16-byte aligned", i);
+  }
+  return SHARQ_OK;
+}
+
+sharq_status check_weight(const sharq_weight* w) {
+  if (!w) return fail(SHARQ_ERR_INVALID, "weight: NULL");
+  sharq_status st = check_shape(w->k, w->n, true);
+  if (st != SHARQ_OK) return st;
+  if (w->fmt != SHARQ_MXFP4 && w->fmt != SHARQ_NVFP4) return fail(SHARQ_ERR_INVALID, "bad format %d", (int)w->fmt);
+  if (w->experts < 1) return fail(SHARQ_ERR_INVALID, "experts=%d", (int)w->experts);
+  const void* ptrs[4] = {w->codes, w->scales_dense, w->scales_sparse, w->tensor};
+  for (int i = 0; i < 4; i++) {
+    if (!ptrs[i]) return fail(SHARQ_ERR_INVALID, "weight buffer %d is NULL", i);
+    if (!aligned(ptrs[i], 16)) return fail(SHARQ_ERR_INVALID, "weight buffer %d is not 16-byte aligned", i);
+  }
+  return SHARQ_OK;
+}
+
+sharq_status run_linear(const sharq_prepared* a, const sharq_weight* w, const int32_t* offsets, void* y,
+                        sharq_dtype y_dt, int32_t paths, cudaStream_t s) {
+  sharq_status st = check_prepared(a);
+  if (st != SHARQ_OK) return st;
+  st = check_weight(w);
+  if (st != SHARQ_OK) return st;
+  if (a->k != w->k) return fail(SHARQ_ERR_INVALID, "k mismatch: activations %lld, weight %lld", (long long)a->k,
+                                (long long)w->k);
+  if (a->fmt != w->fmt) return fail(SHARQ_ERR_INVALID, "format mismatch between activations and weight");
+  if (!y || !aligned(y, 16)) return fail(SHARQ_ERR_INVALID, "y must be a 16-byte aligned device pointer");
+  if (y_dt != SHARQ_F32 && y_dt != SHARQ_BF16) return fail(SHARQ_ERR_INVALID, "bad y dtype %d", (int)y_dt);
+  if (paths < 1 || paths > 3) return fail(SHARQ_ERR_INVALID, "paths=%d", (int)paths);
+  if (offsets == nullptr && w->experts != 1)
+    return fail(SHARQ_ERR_INVALID, "a stacked weight needs sharq_linear_grouped");
+  if (a->fmt == SHARQ_NVFP4 && a->pat == SHARQ_NM_2_4)
+    return fail(SHARQ_ERR_UNSUPPORTED, "NVFP4 with element-wise 2:4 has no sparse tensor-core kind");
+  if (a->fmt == SHARQ_MXFP4 && a->pat == SHARQ_NM_2_4)
+    return fail(SHARQ_ERR_UNSUPPORTED, "MXFP4 2:4 linear is not built yet");
+
+  const int64_t t_pad = round_up(a->t, 128);
+  const bool sparse = a->pat != SHARQ_NM_8_16;
+  GemmMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  st = make_map(&maps.w, w->codes, w->k / 2, w->n * w->experts, 128, 256, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != SHARQ_OK) return st;
+  st = make_map(&maps.r, a->res_codes, a->k / 2, t_pad, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != SHARQ_OK) return st;
+  if (sparse) {
+    st = make_map(&maps.b, a->bb_codes, a->k / 4, t_pad, 64, 128, CU_TENSOR_MAP_SWIZZLE_64B);
+    if (st != SHARQ_OK) return st;
+    st = make_map(&maps.e, a->meta, meta_row_bytes(a->k, a->pat), t_pad, 16, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != SHARQ_OK) return st;
+  } else {
+    st = make_map(&maps.b, a->bb_codes, a->k / 2, t_pad, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != SHARQ_OK) return st;
+  }
+  GemmParams gp;
+  gp.t = a->t;
+  gp.t_pad = t_pad;
+  gp.n = w->n;
+  gp.k = w->k;
+  gp.experts = w->experts;
+  gp.group_offsets = offsets;
+  gp.sf_res = static_cast<const uint8_t*>(a->res_scales);
+  gp.sf_bb = static_cast<const uint8_t*>(a->bb_scales);
+  gp.sf_w_dense = static_cast<const uint8_t*>(w->scales_dense);
+  gp.sf_w_sparse = static_cast<const uint8_t*>(w->scales_sparse);
+  gp.tensor_x = a->tensor;
+  gp.tensor_w = w->tensor;
+  gp.y = y;
+  gp.y_bf16 = y_dt == SHARQ_BF16;
+  gp.paths = paths;
+  gp.timeout_ns = wait_timeout_ns();
+  if (a->fmt == SHARQ_NVFP4)
+    return sparse ? launch_gemm<GK_NVF4, true>(maps, gp, s) : launch_gemm<GK_NVF4, false>(maps, gp, s);
+  return sparse ? launch_gemm<GK_MXF4, true>(maps, gp, s) : launch_gemm<GK_MXF4, false>(maps, gp, s);
+}
+
+}  // namespace
+
+// =================================================================== C ABI
+extern "C" {
+
+sharq_status sharq_weight_sizes(int64_t n, int64_t k, sharq_format fmt, size_t* codes_bytes,
+                                size_t* scales_dense_bytes, size_t* scales_sparse_bytes) {
+  sharq_status st = check_shape(k, n, true);
+  if (st != SHARQ_OK) return st;
+  if (fmt != SHARQ_MXFP4 && fmt != SHARQ_NVFP4) return fail(SHARQ_ERR_INVALID, "bad format %d", (int)fmt);
+  const int b = fmt_block(fmt);
+  if (codes_bytes) *codes_bytes = (size_t)(n * k / 2);
+  if (scales_dense_bytes) *scales_dense_bytes = (size_t)tiled_sf_bytes(n, k / b);
+  if (scales_sparse_bytes) *scales_sparse_bytes = (size_t)tiled_sf_bytes(n, k / (2 * b));
+  return SHARQ_OK;
+}
+
+sharq_status sharq_prepared_sizes(int64_t t, int64_t k, sharq_format fmt, sharq_pattern pat, size_t* meta_bytes,
+                                  size_t* bb_codes_bytes, size_t* bb_scales_bytes, size_t* res_codes_bytes,
+                                  size_t* res_scales_bytes, size_t* workspace_bytes) {
+  sharq_status st = check_shape(k, t, false);
+  if (st != SHARQ_OK) return st;
+  if (fmt != SHARQ_MXFP4 && fmt != SHARQ_NVFP4) return fail(SHARQ_ERR_INVALID, "bad format %d", (int)fmt);
+  if (pat < SHARQ_NM_2_4 || pat > SHARQ_NM_8_16) return fail(SHARQ_ERR_INVALID, "bad pattern %d", (int)pat);
+  const int64_t tp = round_up(t, 128);
+  const int b = fmt_block(fmt);
+  if (meta_bytes) *meta_bytes = (size_t)(tp * meta_row_bytes(k, pat));
+  if (bb_codes_bytes) *bb_codes_bytes = (size_t)(pat == SHARQ_NM_8_16 ? tp * k / 2 : tp * k / 4);
+  if (bb_scales_bytes) *bb_scales_bytes = (size_t)tiled_sf_bytes(tp, pat == SHARQ_NM_8_16 ? k / b : k / (2 * b));
+  if (res_codes_bytes) *res_codes_bytes = (size_t)(tp * k / 2);
+  if (res_scales_bytes) *res_scales_bytes = (size_t)tiled_sf_bytes(tp, k / b);
+  if (workspace_bytes) *workspace_bytes = 0;
+  return SHARQ_OK;
+}
+
+sharq_status sharq_quantize_weight(const void* w, sharq_dtype w_dt, sharq_weight* out, sharq_stream stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (!w || !aligned(w, 16)) return fail(SHARQ_ERR_INVALID, "w must be a 16-byte aligned device pointer");
+  if (w_dt != SHARQ_F32 && w_dt != SHARQ_BF16) return fail(SHARQ_ERR_INVALID, "bad w dtype %d", (int)w_dt);
+  sharq_status st = check_weight(out);
+  if (st != SHARQ_OK) return st;
+  const int64_t rows = out->n * out->experts;
+  SHARQ_CUDA(cudaMemsetAsync(out->tensor, 0, sizeof(float) * 3 * out->experts, s));
+  const bool bf16 = w_dt == SHARQ_BF16;
+  if (out->fmt == SHARQ_NVFP4) {
+    const int bpe = 64;
+    dim3 grid((unsigned)(out->experts * bpe));
+    if (bf16) weight_amax_kernel<true><<<grid, 256, 0, s>>>(w, out->n, out->k, out->tensor, bpe);
+    else weight_amax_kernel<false><<<grid, 256, 0, s>>>(w, out->n, out->k, out->tensor, bpe);
+    st = launched();
+    if (st != SHARQ_OK) return st;
+  }
+  WeightParams wp;
+  wp.w = w;
+  wp.n = out->n;
+  wp.k = out->k;
+  wp.rows = rows;
+  wp.codes = static_cast<uint8_t*>(out->codes);
+  wp.sf_dense = static_cast<uint8_t*>(out->scales_dense);
+  wp.sf_sparse = static_cast<uint8_t*>(out->scales_sparse);
+  wp.tensor = out->tensor;
+  const int64_t threads = rows * (out->k / 32);
+  dim3 grid((unsigned)((threads + 255) / 256));
+  if (out->fmt == SHARQ_NVFP4) {
+    if (bf16) weight_kernel<FMT_NV, true><<<grid, 256, 0, s>>>(wp);
+    else weight_kernel<FMT_NV, false><<<grid, 256, 0, s>>>(wp);
+  } else {
+    if (bf16) weight_kernel<FMT_MX, true><<<grid, 256, 0, s>>>(wp);
+    else weight_kernel<FMT_MX, false><<<grid, 256, 0, s>>>(wp);
+  }
+  return launched();
+}
+
+sharq_status sharq_prepare(const void* x, sharq_dtype x_dt, const void* gamma, float eps, float act_amax,
+                           sharq_prepared* out, void* workspace, size_t workspace_bytes, sharq_stream stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  sharq_status st = check_prepared(out);
+  if (st != SHARQ_OK) return st;
+  if (!x || !aligned(x, 16)) return fail(SHARQ_ERR_INVALID, "x must be a 16-byte aligned device pointer");
+  if (gamma && !aligned(gamma, 16)) return fail(SHARQ_ERR_INVALID, "gamma must be 16-byte aligned");
+  if (x_dt != SHARQ_F32 && x_dt != SHARQ_BF16) return fail(SHARQ_ERR_INVALID, "bad x dtype %d", (int)x_dt);
+  if (!(eps >= 0.0f)) return fail(SHARQ_ERR_INVALID, "eps must be >= 0");
+  const bool bf16 = x_dt == SHARQ_BF16, norm = gamma != nullptr;
+  PrepParams pp;
+  pp.x = x;
+  pp.gamma = gamma;
+  pp.eps = eps;
+  pp.t = out->t;
+  pp.t_pad = round_up(out->t, 128);
+  pp.k = out->k;
+  pp.meta = static_cast<uint8_t*>(out->meta);
+  pp.bb_codes = static_cast<uint8_t*>(out->bb_codes);
+  pp.bb_scales = static_cast<uint8_t*>(out->bb_scales);
+  pp.res_codes = static_cast<uint8_t*>(out->res_codes);
+  pp.res_scales = static_cast<uint8_t*>(out->res_scales);
+  pp.tensor = out->tensor;
+  pp.act_amax = act_amax > 0.0f ? act_amax : 0.0f;
+  if (out->fmt == SHARQ_NVFP4 && !(act_amax > 0.0f)) {
+    SHARQ_CUDA(cudaMemsetAsync(out->tensor, 0, sizeof(float), s));
+    if (norm) st = bf16 ? launch_amax<true, true>(x, gamma, eps, out->t, out->k, out->tensor, s)
+                        : launch_amax<true, false>(x, gamma, eps, out->t, out->k, out->tensor, s);
+    else st = bf16 ? launch_amax<false, true>(x, gamma, eps, out->t, out->k, out->tensor, s)
+                   : launch_amax<false, false>(x, gamma, eps, out->t, out->k, out->tensor, s);
+    if (st != SHARQ_OK) return st;
+  }
+  if (out->fmt == SHARQ_NVFP4) return prep_dispatch_p<FMT_NV>(pp, out->pat, norm, bf16, s);
+  return prep_dispatch_p<FMT_MX>(pp, out->pat, norm, bf16, s);
+}
+
+sharq_status sharq_linear(const sharq_prepared* a, const sharq_weight* w, void* y, sharq_dtype y_dt,
+                          sharq_stream stream) {
+  return run_linear(a, w, nullptr, y, y_dt, 3, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sharq_status sharq_linear_paths(const sharq_prepared* a, const sharq_weight* w, void* y, sharq_dtype y_dt,
+                                int32_t paths, sharq_stream stream) {
+  return run_linear(a, w, nullptr, y, y_dt, paths, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sharq_status sharq_linear_grouped(const sharq_prepared* a, const sharq_weight* w, const int32_t* group_offsets,
+                                  void* y, sharq_dtype y_dt, sharq_stream stream) {
+  if (!group_offsets) return fail(SHARQ_ERR_INVALID, "group_offsets is NULL");
+  if (a && a->t % 128 != 0) return fail(SHARQ_ERR_INVALID, "grouped rows must be a multiple of 128");
+  return run_linear(a, w, group_offsets, y, y_dt, 3, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sharq_status sharq_sync_status(sharq_stream stream) {
+  SHARQ_CUDA(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
+  unsigned int word = 0, zero = 0;
+  SHARQ_CUDA(cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)));
+  SHARQ_CUDA(cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)));
+  if (word & kErrTimeout) return fail(SHARQ_ERR_TIMEOUT, "a device-side wait ran out of time");
+  return SHARQ_OK;
+}
+
+sharq_status sharq_selftest_wait_timeout(uint64_t timeout_ns, sharq_stream stream) {
+  selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(timeout_ns);
+  return launched();
+}
+
+const char* sharq_last_error(void) { return g_last_error.c_str(); }
+
+uint64_t sharq_launch_count(int reset) {
+  uint64_t v = g_launches;
+  if (reset) g_launches = 0;
+  return v;
+}
+
+}  // extern "C"

@@ -1,0 +1,258 @@
+"""Thin Python binding of ``include/sharq.h`` (ctypes).
+
+Every function named ``sharq_*`` here calls the C function of the same name in
+``_lib/libsharq.so``; the classes only allocate the caller-owned device
+buffers (PyTorch tensors, the library allocates nothing) and marshal pointers,
+shapes and the current CUDA stream.  All arithmetic runs in the CUDA kernels.
+There is no CPU fallback: without the built library every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build_ext
+
+MXFP4, NVFP4 = 0, 1
+NM_2_4, NM_4_8_PAIR, NM_8_16 = 0, 1, 2
+F32, BF16 = 0, 1
+FORMATS = {"mxfp4": MXFP4, "nvfp4": NVFP4}
+PATTERNS = {"2:4": NM_2_4, "4:8pair": NM_4_8_PAIR, "8:16": NM_8_16}
+STATUS = {0: "SHARQ_OK", 1: "SHARQ_ERR_INVALID", 2: "SHARQ_ERR_UNSUPPORTED", 3: "SHARQ_ERR_CUDA",
+          4: "SHARQ_ERR_TIMEOUT", 5: "SHARQ_ERR_WORKSPACE"}
+SYMBOLS = ["sharq_weight_sizes", "sharq_prepared_sizes", "sharq_quantize_weight", "sharq_prepare", "sharq_linear",
+           "sharq_linear_paths", "sharq_linear_grouped", "sharq_sync_status", "sharq_selftest_wait_timeout",
+           "sharq_last_error", "sharq_launch_count"]
+
+
+class SharqError(RuntimeError):
+    def __init__(self, status: int, where: str, msg: str):
+        super().__init__(f"{where}: {STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class sharq_weight(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales_dense", ctypes.c_void_p), ("scales_sparse", ctypes.c_void_p),
+                ("tensor", ctypes.c_void_p), ("n", ctypes.c_int64), ("k", ctypes.c_int64),
+                ("experts", ctypes.c_int32), ("fmt", ctypes.c_int)]
+
+
+class sharq_prepared(ctypes.Structure):
+    _fields_ = [("meta", ctypes.c_void_p), ("bb_codes", ctypes.c_void_p), ("bb_scales", ctypes.c_void_p),
+                ("res_codes", ctypes.c_void_p), ("res_scales", ctypes.c_void_p), ("tensor", ctypes.c_void_p),
+                ("t", ctypes.c_int64), ("k", ctypes.c_int64), ("fmt", ctypes.c_int), ("pat", ctypes.c_int)]
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return build_ext.LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded CUDA library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        path = build_ext.LIB_PATH
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with `python -m activation_sparsity_fp4_b200.build_ext` "
+                               "(there is no CPU fallback)")
+        L = ctypes.CDLL(path)
+        P, I64, I32, I, F, SZ = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int, ctypes.c_float,
+                                 ctypes.POINTER(ctypes.c_size_t))
+        sig = {
+            "sharq_weight_sizes": [I64, I64, I, SZ, SZ, SZ],
+            "sharq_prepared_sizes": [I64, I64, I, I, SZ, SZ, SZ, SZ, SZ, SZ],
+            "sharq_quantize_weight": [P, I, ctypes.POINTER(sharq_weight), P],
+            "sharq_prepare": [P, I, P, F, F, ctypes.POINTER(sharq_prepared), P, ctypes.c_size_t, P],
+            "sharq_linear": [ctypes.POINTER(sharq_prepared), ctypes.POINTER(sharq_weight), P, I, P],
+            "sharq_linear_paths": [ctypes.POINTER(sharq_prepared), ctypes.POINTER(sharq_weight), P, I, I32, P],
+            "sharq_linear_grouped": [ctypes.POINTER(sharq_prepared), ctypes.POINTER(sharq_weight), P, P, I, P],
+            "sharq_sync_status": [P],
+            "sharq_selftest_wait_timeout": [ctypes.c_uint64, P],
+        }
+        for name, args in sig.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_int
+        L.sharq_last_error.restype = ctypes.c_char_p
+        L.sharq_last_error.argtypes = []
+        L.sharq_launch_count.restype = ctypes.c_uint64
+        L.sharq_launch_count.argtypes = [ctypes.c_int]
+        _lib = L
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise SharqError(status, where, lib().sharq_last_error().decode())
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _fmt(f) -> int:
+    return FORMATS[f] if isinstance(f, str) else int(f)
+
+
+def _pat(p) -> int:
+    return PATTERNS[p] if isinstance(p, str) else int(p)
+
+
+def _dt(d) -> int:
+    if isinstance(d, torch.dtype):
+        if d == torch.bfloat16:
+            return BF16
+        if d == torch.float32:
+            return F32
+        raise ValueError(f"unsupported dtype {d}")
+    return int(d)
+
+
+# ------------------------------------------------------- same-name wrappers
+def sharq_weight_sizes(n: int, k: int, fmt) -> tuple[int, int, int]:
+    out = [ctypes.c_size_t() for _ in range(3)]
+    _check(lib().sharq_weight_sizes(n, k, _fmt(fmt), *[ctypes.byref(o) for o in out]), "sharq_weight_sizes")
+    return tuple(o.value for o in out)
+
+
+def sharq_prepared_sizes(t: int, k: int, fmt, pat) -> tuple[int, int, int, int, int, int]:
+    out = [ctypes.c_size_t() for _ in range(6)]
+    _check(lib().sharq_prepared_sizes(t, k, _fmt(fmt), _pat(pat), *[ctypes.byref(o) for o in out]),
+           "sharq_prepared_sizes")
+    return tuple(o.value for o in out)
+
+
+def sharq_quantize_weight(w_ptr: int, w_dt, out: sharq_weight, stream=None):
+    _check(lib().sharq_quantize_weight(ctypes.c_void_p(w_ptr), _dt(w_dt), ctypes.byref(out), _stream(stream)),
+           "sharq_quantize_weight")
+
+
+def sharq_prepare(x_ptr: int, x_dt, gamma_ptr, eps: float, act_amax: float, out: sharq_prepared, workspace_ptr=None,
+                  workspace_bytes: int = 0, stream=None):
+    _check(lib().sharq_prepare(ctypes.c_void_p(x_ptr), _dt(x_dt), ctypes.c_void_p(gamma_ptr) if gamma_ptr else None,
+                               float(eps), float(act_amax), ctypes.byref(out),
+                               ctypes.c_void_p(workspace_ptr) if workspace_ptr else None, workspace_bytes,
+                               _stream(stream)), "sharq_prepare")
+
+
+def sharq_linear(a: sharq_prepared, w: sharq_weight, y_ptr: int, y_dt, stream=None):
+    _check(lib().sharq_linear(ctypes.byref(a), ctypes.byref(w), ctypes.c_void_p(y_ptr), _dt(y_dt), _stream(stream)),
+           "sharq_linear")
+
+
+def sharq_linear_paths(a: sharq_prepared, w: sharq_weight, y_ptr: int, y_dt, paths: int, stream=None):
+    _check(lib().sharq_linear_paths(ctypes.byref(a), ctypes.byref(w), ctypes.c_void_p(y_ptr), _dt(y_dt), paths,
+                                    _stream(stream)), "sharq_linear_paths")
+
+
+def sharq_linear_grouped(a: sharq_prepared, w: sharq_weight, offsets_ptr: int, y_ptr: int, y_dt, stream=None):
+    _check(lib().sharq_linear_grouped(ctypes.byref(a), ctypes.byref(w), ctypes.c_void_p(offsets_ptr),
+                                      ctypes.c_void_p(y_ptr), _dt(y_dt), _stream(stream)), "sharq_linear_grouped")
+
+
+def sharq_sync_status(stream=None):
+    _check(lib().sharq_sync_status(_stream(stream)), "sharq_sync_status")
+
+
+def sharq_selftest_wait_timeout(timeout_ns: int, stream=None):
+    _check(lib().sharq_selftest_wait_timeout(int(timeout_ns), _stream(stream)), "sharq_selftest_wait_timeout")
+
+
+def sharq_last_error() -> str:
+    return lib().sharq_last_error().decode()
+
+
+def sharq_launch_count(reset: bool = False) -> int:
+    return int(lib().sharq_launch_count(1 if reset else 0))
+
+
+# ------------------------------------------------------------ buffer owners
+def _alloc(nbytes: int, device) -> torch.Tensor:
+    # 256-byte aligned (PyTorch's caching allocator aligns blocks to 512 bytes)
+    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
+class FP4Weight:
+    """Device buffers of a shared FP4 weight (one or ``experts`` stacked)."""
+
+    def __init__(self, n: int, k: int, fmt, experts: int = 1, device="cuda"):
+        self.n, self.k, self.fmt, self.experts = n, k, _fmt(fmt), experts
+        c, d, s = sharq_weight_sizes(n, k, self.fmt)
+        self.codes = _alloc(c * experts, device)
+        self.scales_dense = _alloc(d * experts, device)
+        self.scales_sparse = _alloc(s * experts, device)
+        self.tensor = torch.zeros(3 * experts, dtype=torch.float32, device=device)
+        self.struct = sharq_weight(self.codes.data_ptr(), self.scales_dense.data_ptr(),
+                                   self.scales_sparse.data_ptr(), self.tensor.data_ptr(), n, k, experts, self.fmt)
+
+    @classmethod
+    def quantize(cls, w: torch.Tensor, fmt, stream=None) -> "FP4Weight":
+        """w: (n, k) or (experts, n, k), bf16 or fp32, on the GPU."""
+        w = w.contiguous()
+        experts = w.shape[0] if w.dim() == 3 else 1
+        n, k = w.shape[-2], w.shape[-1]
+        obj = cls(n, k, fmt, experts, w.device)
+        sharq_quantize_weight(w.data_ptr(), w.dtype, obj.struct, stream)
+        obj._src = w  # keep the source alive until the stream has consumed it
+        return obj
+
+
+class Prepared:
+    """Device buffers of prepared activations for t rows."""
+
+    def __init__(self, t: int, k: int, fmt, pat, device="cuda"):
+        self.t, self.k, self.fmt, self.pat = t, k, _fmt(fmt), _pat(pat)
+        m, bc, bs, rc, rs, ws = sharq_prepared_sizes(t, k, self.fmt, self.pat)
+        self.meta = _alloc(m, device)
+        self.bb_codes = _alloc(bc, device)
+        self.bb_scales = _alloc(bs, device)
+        self.res_codes = _alloc(rc, device)
+        self.res_scales = _alloc(rs, device)
+        self.tensor = torch.zeros(3, dtype=torch.float32, device=device)
+        self.workspace = _alloc(ws, device) if ws else None
+        self.struct = sharq_prepared(self.meta.data_ptr(), self.bb_codes.data_ptr(), self.bb_scales.data_ptr(),
+                                     self.res_codes.data_ptr(), self.res_scales.data_ptr(), self.tensor.data_ptr(),
+                                     t, k, self.fmt, self.pat)
+
+
+def prepare(x: torch.Tensor, fmt, pat, gamma: torch.Tensor | None = None, eps: float = 1e-6, act_amax: float = 0.0,
+            out: Prepared | None = None, stream=None) -> Prepared:
+    """Fused preprocessing of x (t, k) on the GPU; returns (or fills) a Prepared."""
+    x = x.contiguous()
+    t, k = x.shape
+    if out is None:
+        out = Prepared(t, k, fmt, pat, x.device)
+    if gamma is not None:
+        gamma = gamma.to(x.dtype).contiguous()
+    ws = out.workspace
+    sharq_prepare(x.data_ptr(), x.dtype, gamma.data_ptr() if gamma is not None else None, eps, act_amax, out.struct,
+                  ws.data_ptr() if ws is not None else None, ws.numel() if ws is not None else 0, stream)
+    return out
+
+
+def linear(a: Prepared, w: FP4Weight, out_dtype=torch.bfloat16, out: torch.Tensor | None = None, paths: int = 3,
+           stream=None) -> torch.Tensor:
+    """y = the sparse backbone GEMM plus the dense residual GEMM, (t, n)."""
+    if out is None:
+        out = torch.empty((a.t, w.n), dtype=out_dtype, device=a.meta.device)
+    if paths == 3:
+        sharq_linear(a.struct, w.struct, out.data_ptr(), out.dtype, stream)
+    else:
+        sharq_linear_paths(a.struct, w.struct, out.data_ptr(), out.dtype, paths, stream)
+    return out
+
+
+def linear_grouped(a: Prepared, w: FP4Weight, offsets: torch.Tensor, out_dtype=torch.bfloat16,
+                   out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.zeros((a.t, w.n), dtype=out_dtype, device=a.meta.device)
+    offsets = offsets.to(torch.int32).contiguous()
+    sharq_linear_grouped(a.struct, w.struct, offsets.data_ptr(), out.data_ptr(), out.dtype, stream)
+    return out

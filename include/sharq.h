@@ -1,0 +1,181 @@
+/*
+ * sharq.h -- C ABI of the B200 (sm_100a) SharQ sparse-dense FP4 linear layer.
+ *
+ * The layer (SharQ, arXiv 2606.26587, abstract and Section 1) splits each
+ * activation row online into an outlier-dominated N:M-sparse backbone, which
+ * is quantized to FP4 and multiplied by a sparse FP4 GEMM, and a dense
+ * residual taken against the QUANTIZED backbone, quantized to FP4 and
+ * accumulated into the same output by a dense FP4 GEMM.  Both GEMMs read one
+ * shared FP4 weight through path-specific scale views, and a fused
+ * preprocessing op absorbs the layer norm, the mask and the residual.
+ *
+ * Conventions for every call:
+ *  - All tensor arguments are DEVICE pointers on the current CUDA device,
+ *    owned and allocated by the caller with the sizes the *_sizes queries
+ *    return.  The library allocates no device memory and keeps no device
+ *    state besides one error word per device.
+ *  - Calls are asynchronous on the given stream.  Argument errors are found
+ *    on the host and returned before anything is launched.  A device-side
+ *    wait that runs out of time sets the error word; sharq_sync_status()
+ *    synchronizes the stream and reports it (SHARQ_ERR_TIMEOUT).
+ *  - Shapes: k % 256 == 0; n % 256 == 0; t >= 1.  Row buffers of prepared
+ *    activations hold t_pad = roundup(t, 128) rows; rows t..t_pad-1 are
+ *    written as if their input were zero.
+ *  - Byte layouts (little endian):
+ *      codes      two E2M1 codes per byte, the lower K index in the low nibble;
+ *      scales     "tiled scale layout": a tensor with R rows and S scales per
+ *                 row is stored as ceil(R/128) x ceil(S/4) blocks of 512 bytes,
+ *                 row-block major; inside a block, row r and scale s sit at
+ *                 byte (r%32)*16 + ((r/32)%4)*4 + (s%4);
+ *      meta       row-major, 2:4 and 4:8 pair: one nibble per group of 4 (8)
+ *                 K elements, nibble = i0 | i1 << 2 with the kept element
+ *                 (pair) indices i0 < i1, group g in byte g/2, low nibble
+ *                 first; 8:16: one little-endian uint16 mask per group of 16.
+ *      tensor     3 floats: [amax, g_enc, g_dec] (NVFP4 second-level scale
+ *                 g_enc = 2688/amax, g_dec = amax/2688; MXFP4: [0, 1, 1]).
+ */
+#ifndef SHARQ_H
+#define SHARQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* sharq_stream; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  SHARQ_OK = 0,
+  SHARQ_ERR_INVALID = 1,     /* bad shape, pointer, alignment or enum value */
+  SHARQ_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. NVFP4 with 2:4 in sharq_linear) */
+  SHARQ_ERR_CUDA = 3,        /* a CUDA runtime call failed; see sharq_last_error() */
+  SHARQ_ERR_TIMEOUT = 4,     /* a device-side wait ran out of time (error word) */
+  SHARQ_ERR_WORKSPACE = 5    /* workspace missing or too small */
+} sharq_status;
+
+/* FP4 formats (SharQ abstract; Section 2.3 names OCP MX):
+ *   MXFP4 -- E2M1 elements, one E8M0 scale per 32 elements, no tensor scale;
+ *   NVFP4 -- E2M1 elements, one E4M3 scale per 16 elements, fp32 tensor scale. */
+typedef enum { SHARQ_MXFP4 = 0, SHARQ_NVFP4 = 1 } sharq_format;
+
+/* Online N:M activation masks: 2:4 (Huawei problem 137-2, "MXFP4/HiF4 with 2:4
+ * sparsity"), the NVFP4 4:8 pair pattern (SharQ Section 2.2: two of four
+ * adjacent pairs kept), and 8:16 ("From 2:4 to 8:16 sparsity patterns", abstract). */
+typedef enum { SHARQ_NM_2_4 = 0, SHARQ_NM_4_8_PAIR = 1, SHARQ_NM_8_16 = 2 } sharq_pattern;
+
+typedef enum { SHARQ_F32 = 0, SHARQ_BF16 = 1 } sharq_dtype;
+
+/* The FP4 weight shared by the sparse and the dense GEMM (SharQ abstract:
+ * "both paths share one FP4 weight load, with path-specific scale views").
+ * The sparse tensor-core MMA applies one scale per b stored (2b logical) K
+ * elements, so the weight is quantized in K blocks of 2b (b = 32 MXFP4, 16
+ * NVFP4) and carries two views of the same scales:
+ *   codes          experts * n * k/2 bytes, row-major per expert;
+ *   scales_dense   per expert, tiled scale layout, n rows, k/b scales (each 2b
+ *                  scale stored twice) -- the view of the dense residual GEMM;
+ *   scales_sparse  per expert, tiled scale layout, n rows, k/(2b) scales;
+ *   tensor         experts * 3 floats. */
+typedef struct {
+  void* codes;
+  void* scales_dense;
+  void* scales_sparse;
+  float* tensor;
+  int64_t n, k;
+  int32_t experts; /* 1 for a plain linear layer; stacked experts for sharq_linear_grouped */
+  sharq_format fmt;
+} sharq_weight;
+
+/* Prepared activations (output of sharq_prepare):
+ *   meta       t_pad * meta_row bytes (meta_row = k/8 for 2:4 and 8:16, k/16 for 4:8 pair)
+ *   bb_codes   backbone codes: 2:4 and 4:8 pair -- t_pad * k/4 bytes, the k/2 kept values
+ *              of a row in K order ("sparse input compression", SharQ Section 1);
+ *              8:16 -- t_pad * k/2 bytes, dense layout with code 0 at dropped positions
+ *   bb_scales  tiled scale layout, t_pad rows: one scale per b kept values (k/(2b) per
+ *              row); for 8:16 each is stored twice (k/b per row), the dense view
+ *   res_codes  t_pad * k/2 bytes, dense residual codes
+ *   res_scales tiled scale layout, t_pad rows, k/b scales per row
+ *   tensor     3 floats shared by backbone and residual (NVFP4) */
+typedef struct {
+  void* meta;
+  void* bb_codes;
+  void* bb_scales;
+  void* res_codes;
+  void* res_scales;
+  float* tensor;
+  int64_t t, k;
+  sharq_format fmt;
+  sharq_pattern pat;
+} sharq_prepared;
+
+/* Byte sizes of the weight buffers for one expert (multiply by experts). */
+sharq_status sharq_weight_sizes(int64_t n, int64_t k, sharq_format fmt, size_t* codes_bytes,
+                                size_t* scales_dense_bytes, size_t* scales_sparse_bytes);
+
+/* Byte sizes of the prepared-activation buffers for t rows and of the
+ * workspace sharq_prepare needs (0: it needs none). */
+sharq_status sharq_prepared_sizes(int64_t t, int64_t k, sharq_format fmt, sharq_pattern pat, size_t* meta_bytes,
+                                  size_t* bb_codes_bytes, size_t* bb_scales_bytes, size_t* res_codes_bytes,
+                                  size_t* res_scales_bytes, size_t* workspace_bytes);
+
+/* Offline weight quantization (W4 of W4A4, Huawei problem 137-2; the shared
+ * weight of the SharQ abstract).  w: experts * n * k values (row-major, nn.Linear
+ * out x in layout) of dtype w_dt.  Each expert gets its own tensor scale (NVFP4).
+ * out->codes/scales/tensor must be set by the caller; n, k, experts, fmt too. */
+sharq_status sharq_quantize_weight(const void* w, sharq_dtype w_dt, sharq_weight* out, sharq_stream stream);
+
+/* Fused preprocessing (SharQ abstract: "a fused preprocessing kernel absorbs mask
+ * generation, residual construction and layer normalization into one operator"):
+ *   h = RMSNorm(x) * gamma if gamma != NULL (fp32, eps added to the mean square), else x;
+ *   N:M mask = top-N |h| per group of M, ties to the lower index (4:8 pair: top 2 of 4
+ *   adjacent pairs by max |.|); backbone = kept values, FP4 in blocks of b kept values;
+ *   R = h - dequant(backbone) where kept, h elsewhere; R to FP4 in blocks of b.
+ * x: t * k row-major values of dtype x_dt; gamma: k values of dtype x_dt or NULL.
+ * act_amax > 0 gives the NVFP4 tensor amax; <= 0 computes max |h| on the device
+ * (one extra read of x).  out->pointers, t, k, fmt, pat must be set by the caller.
+ * workspace may be NULL when sharq_prepared_sizes reports 0. */
+sharq_status sharq_prepare(const void* x, sharq_dtype x_dt, const void* gamma, float eps, float act_amax,
+                           sharq_prepared* out, void* workspace, size_t workspace_bytes, sharq_stream stream);
+
+/* The two GEMMs of the layer (SharQ abstract, Section 1): a sparse FP4 GEMM over
+ * the compressed backbone and its metadata, and a dense FP4 GEMM over R that
+ * accumulates into the same output, one weight load per K tile feeding both:
+ *   y[t][n] = g_dec_x * g_dec_w * sum_k (B[t][k] + R[t][k]) * W[n][k]
+ * y: t * n row-major, dtype y_dt.  Supported: MXFP4 with every pattern, NVFP4 with
+ * 4:8 pair and 8:16 (NVFP4 2:4 returns SHARQ_ERR_UNSUPPORTED: no sparse tensor-core
+ * kind takes E4M3 block-16 scales with element-wise 2:4 metadata). */
+sharq_status sharq_linear(const sharq_prepared* a, const sharq_weight* w, void* y, sharq_dtype y_dt,
+                          sharq_stream stream);
+
+/* Same, with a choice of paths for diagnosis: paths bit 0 = sparse backbone GEMM,
+ * bit 1 = dense residual GEMM (3 = the layer). */
+sharq_status sharq_linear_paths(const sharq_prepared* a, const sharq_weight* w, void* y, sharq_dtype y_dt,
+                                int32_t paths, sharq_stream stream);
+
+/* Mixture-of-experts form (SharQ evaluates Qwen3-30B-A3B): a holds the routed rows of
+ * all experts, grouped by expert; group_offsets (DEVICE, experts+1 int32, non-decreasing,
+ * each a multiple of 128, last = a->t rounded up to 128) delimits expert e's rows
+ * [off[e], off[e+1]).  w holds w->experts stacked weights.  Rows of y outside every
+ * group are left unwritten. */
+sharq_status sharq_linear_grouped(const sharq_prepared* a, const sharq_weight* w, const int32_t* group_offsets,
+                                  void* y, sharq_dtype y_dt, sharq_stream stream);
+
+/* Synchronizes the stream, then reports and clears this device's error word. */
+sharq_status sharq_sync_status(sharq_stream stream);
+
+/* Test hook for the failure path: launches one block whose wait on a flag that
+ * nothing sets gives up after timeout_ns, sets the error word and returns. */
+sharq_status sharq_selftest_wait_timeout(uint64_t timeout_ns, sharq_stream stream);
+
+/* Text of the last error on this host thread ("" if none). */
+const char* sharq_last_error(void);
+
+/* Number of kernel launches the calls above have made on this host thread since the
+ * last reset (for launch accounting in benchmarks). */
+uint64_t sharq_launch_count(int reset);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SHARQ_H */

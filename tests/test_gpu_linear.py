@@ -1,0 +1,139 @@
+"""Parity of the weight quantizer (bit-exact) and of the fused sparse+dense
+FP4 GEMM (rel. Frobenius <= 1e-4 and |d| <= 1e-3 max|Y|) with the oracle's
+fp64 product of the dequantized operands."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from _layout import untile_scales
+from activation_sparsity_fp4_b200 import sharq, workloads
+from gpu_common import assert_close_gemm, gpu_prepare, readback, assert_prep_equal, to_dev
+
+pytestmark = pytest.mark.gpu
+
+LINEAR_CASES = [("nvfp4", "4:8pair"), ("nvfp4", "8:16"), ("mxfp4", "4:8pair"), ("mxfp4", "8:16")]
+
+
+def _w(seed, n, k, scale=0.02):
+    rng = np.random.default_rng(seed)
+    return workloads.to_bf16_values((rng.standard_normal((n, k)) * scale).astype(np.float32))
+
+
+def _x(seed, t, k):
+    rng = np.random.default_rng(seed)
+    x = (0.5 * rng.standard_t(3, size=(t, k))).astype(np.float32)
+    x[:, rng.permutation(k)[:6]] *= 60.0
+    return workloads.to_bf16_values(x)
+
+
+def gpu_weight(w, w_dtype, fmt):
+    wq = sharq.FP4Weight.quantize(to_dev(w, w_dtype), fmt)
+    sharq.sharq_sync_status()
+    return wq
+
+
+def weight_readback(wq):
+    n, k = wq.n, wq.k
+    b = 16 if wq.fmt == sharq.NVFP4 else 32
+    codes = wq.codes.cpu().numpy()[: n * k // 2].reshape(n, k // 2)
+    dense = untile_scales(wq.scales_dense.cpu().numpy(), n, k // b)
+    sparse = untile_scales(wq.scales_sparse.cpu().numpy(), n, k // (2 * b))
+    return codes, dense, sparse, wq.tensor.cpu().numpy()
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+@pytest.mark.parametrize("wdt", ["f32", "bf16"])
+def test_weight_quantization_bit_exact(cuda_ok, fmt, wdt):
+    w = _w(1, 512, 1024)
+    ref = oracle.quantize_weight(w, fmt)
+    codes, dense, sparse, tens = weight_readback(gpu_weight(w, wdt, fmt))
+    np.testing.assert_array_equal(codes, ref["codes"])
+    np.testing.assert_array_equal(sparse, ref["scales"])
+    np.testing.assert_array_equal(dense[:, 0::2], ref["scales"])
+    np.testing.assert_array_equal(dense[:, 1::2], ref["scales"])
+    np.testing.assert_array_equal(tens, ref["tensor"])
+
+
+def test_weight_quantization_stacked_experts(cuda_ok):
+    w = np.stack([_w(10 + e, 256, 512, scale=0.01 * (e + 1)) for e in range(3)])
+    wq = sharq.FP4Weight.quantize(to_dev(w, "bf16"), "nvfp4")
+    sharq.sharq_sync_status()
+    c, d, s = sharq.sharq_weight_sizes(256, 512, "nvfp4")
+    for e in range(3):
+        ref = oracle.quantize_weight(w[e], "nvfp4")
+        np.testing.assert_array_equal(wq.codes.cpu().numpy()[e * c:(e + 1) * c].reshape(256, 256), ref["codes"])
+        np.testing.assert_array_equal(untile_scales(wq.scales_sparse.cpu().numpy()[e * s:(e + 1) * s], 256, 16),
+                                      ref["scales"])
+        np.testing.assert_array_equal(wq.tensor.cpu().numpy()[3 * e:3 * e + 3], ref["tensor"])
+
+
+def _run_linear(x, w, fmt, pat, gamma=None, out_dtype=torch.float32, paths=3, x_dtype="bf16", w_dtype="bf16"):
+    p = gpu_prepare(x, x_dtype, fmt, pat, gamma=gamma)
+    wq = gpu_weight(w, w_dtype, fmt)
+    y = sharq.linear(p, wq, out_dtype=out_dtype, paths=paths)
+    sharq.sharq_sync_status()
+    return p, wq, y.float().cpu().numpy()
+
+
+def _ref(x, w, fmt, pat, gamma=None, rows=None, act_amax=0.0):
+    prep = oracle.prepare(x, fmt, pat, gamma=gamma, act_amax=act_amax, threads=4)
+    wq = oracle.quantize_weight(w, fmt)
+    return prep, wq
+
+
+@pytest.mark.parametrize("fmt,pat", LINEAR_CASES)
+def test_linear_matches_oracle(cuda_ok, fmt, pat):
+    t, k, n = 200, 1024, 512  # 2 row tiles (ragged), 4 K tiles, 2 column tiles
+    x, w = _x(2, t, k), _w(3, n, k)
+    _, _, y = _run_linear(x, w, fmt, pat)
+    prep, wq = _ref(x, w, fmt, pat)
+    assert_close_gemm(y, oracle.linear_ref(prep, wq), f"{fmt} {pat}")
+
+
+@pytest.mark.parametrize("fmt,pat", LINEAR_CASES)
+def test_linear_each_path_separately(cuda_ok, fmt, pat):
+    """Sparse backbone GEMM alone and dense residual GEMM alone, against the
+    oracle's two partial products (this localizes a wrong metadata or scale
+    view to one path)."""
+    t, k, n = 128, 512, 256
+    x, w = _x(4, t, k), _w(5, n, k)
+    prep, wq = _ref(x, w, fmt, pat)
+    bu, ru = oracle.decode_prepared(prep)
+    wu = oracle.decode_weight(wq)
+    alpha = float(prep["tensor"][2]) * float(wq["tensor"][2])
+    for paths, ref in ((1, alpha * bu @ wu.T), (2, alpha * ru @ wu.T)):
+        _, _, y = _run_linear(x, w, fmt, pat, paths=paths)
+        assert_close_gemm(y, ref, f"{fmt} {pat} paths={paths}")
+
+
+def test_linear_bf16_output_and_single_row(cuda_ok):
+    k, n = 512, 256
+    w = _w(6, n, k)
+    for t in (1, 129):
+        x = _x(7, t, k)
+        _, _, y = _run_linear(x, w, "nvfp4", "4:8pair", out_dtype=torch.bfloat16)
+        prep, wq = _ref(x, w, "nvfp4", "4:8pair")
+        ref = oracle.linear_ref(prep, wq)
+        # bf16 output: the rounding of the output itself dominates (2^-9 relative)
+        err = np.linalg.norm(y - ref) / np.linalg.norm(ref)
+        assert err < 4e-3
+
+
+def test_linear_tiny_config_mxfp4_4_8_pair(cuda_ok):
+    cfg = workloads.tiny()
+    _, _, y = _run_linear(cfg["x"], cfg["w"], "mxfp4", "4:8pair", x_dtype="f32", w_dtype="f32")
+    prep, wq = _ref(cfg["x"], cfg["w"], "mxfp4", "4:8pair")
+    assert_close_gemm(y, oracle.linear_ref(prep, wq), "tiny 4:8pair")
+
+
+def test_linear_q_proj_full_size_sampled_rows(cuda_ok):
+    """Llama-3.1-8B q_proj shape (2048 x 4096 -> 4096), NVFP4 4:8 pair with
+    RMSNorm, in the bench's launch configuration; 64 sampled rows against fp64."""
+    cfg = workloads.q_proj()
+    p, wq_gpu, y = _run_linear(cfg["x"], cfg["w"], "nvfp4", "4:8pair", gamma=cfg["gamma"])
+    rows = np.sort(np.random.default_rng(8).choice(2048, 64, replace=False))
+    amax = float(p.tensor[0].item())
+    prep = oracle.prepare(cfg["x"][rows], "nvfp4", "4:8pair", gamma=cfg["gamma"], act_amax=amax)
+    wq = oracle.quantize_weight(cfg["w"], "nvfp4")
+    assert_close_gemm(y[rows], oracle.linear_ref(prep, wq), "q_proj sampled rows")
