@@ -27,28 +27,48 @@
 
 namespace sharq {
 
-enum { GK_NVF4 = 0, GK_MXF4 = 1 };
+enum { GK_NVF4 = 0, GK_MXF4 = 1, GK_MXF8 = 2 };
 
+// Per-kind tile configuration.
+//   GK_NVF4  NVFP4: kind::mxf4nvf4 (dense K=64, 4 E4M3 scales of 16) and its
+//            4:8-pair sparse form (K=128 logical, 4 scales of 32 logical);
+//   GK_MXF4  MXFP4 with the 4:8 pair: kind::mxf4 (2 E8M0 scales of 32) and
+//            kind::mxf4.sp (2 scales of 64 logical);
+//   GK_MXF8  MXFP4 with element-wise 2:4: the only sparse kind that takes it is
+//            kind::mxf8f6f4.sp, with E2M1 held in 8-bit shared-memory containers
+//            (TMA unpacks 16 packed codes into 16 bytes); the dense residual runs
+//            as kind::mxf8f6f4 on the same unpacked weight tile.
+// SPARSE = false is the 8:16 form: the backbone is stored dense and runs through
+// the dense MMA like the residual.
 template <int KIND, bool SPARSE>
 struct GemmCfg {
-  static constexpr int BM = 128, BN = 256, BK = 256;
-  static constexpr int kDenseMmaK = 64;    // logical K per dense MMA
-  static constexpr int kSparseMmaK = 128;  // logical K per sparse MMA
+  static constexpr bool kUnpacked = KIND == GK_MXF8;
+  static constexpr int BM = 128, BN = kUnpacked ? 128 : 256, BK = 256;
+  static constexpr int kNRB = BN / 128;                        // 128-row blocks of the weight tile
+  static constexpr int kDenseMmaK = kUnpacked ? 32 : 64;       // logical K per dense MMA
+  static constexpr int kSparseMmaK = kUnpacked ? 64 : 128;     // logical K per sparse MMA
   static constexpr int kVecDense = (KIND == GK_NVF4) ? 16 : 32;  // logical K per scale, dense MMA
   static constexpr int kVecSparse = 2 * kVecDense;                // logical K per scale, sparse MMA
-  static constexpr int kRowDense = BK / 2;                         // bytes per row per stage: W, R
-  static constexpr int kRowB = SPARSE ? BK / 4 : BK / 2;           // backbone (compressed or dense)
-  static constexpr int kRowE = SPARSE ? 16 : 0;                    // metadata (4:8 pair)
-  static constexpr int kWBytes = BN * kRowDense;
-  static constexpr int kRBytes = BM * kRowDense;
-  static constexpr int kBBytes = BM * kRowB;
-  static constexpr int kEBytes = BM * kRowE;
+  static constexpr int kBoxElems = kUnpacked ? 128 : 256;      // K elements per 128-byte smem row of a box
+  static constexpr int kBoxesDense = BK / kBoxElems;           // boxes per stage of W and R
+  static constexpr int kBoxR = BM * 128, kBoxW = BN * 128;     // bytes of one box
+  static constexpr int kWBytes = kBoxesDense * kBoxW;
+  static constexpr int kRBytes = kBoxesDense * kBoxR;
+  static constexpr int kRowB = SPARSE ? (kUnpacked ? 128 : 64) : 128;  // smem bytes per backbone row per box
+  static constexpr int kBoxesB = SPARSE ? 1 : kBoxesDense;
+  static constexpr int kBBytes = kBoxesB * BM * kRowB;
+  static constexpr int kMetaStage = SPARSE ? (kUnpacked ? BK / 8 : BK / 16) : 0;  // metadata bytes per row
+  static constexpr int kEBoxes = kMetaStage / 16;              // 16-byte metadata boxes per stage
+  static constexpr int kEBytes = kEBoxes * BM * 16;
+  // TMA inner coordinate per stage (packed maps count bytes, unpacked maps elements)
+  static constexpr int kXStage = kUnpacked ? BK : BK / 2;
+  static constexpr int kXStageB = SPARSE ? (kUnpacked ? BK / 2 : BK / 4) : kXStage;
   static constexpr int kChunksR = BK / kVecDense / 4;                  // 512-byte scale chunks per stage
   static constexpr int kChunksB = SPARSE ? BK / kVecSparse / 4 : kChunksR;
   static constexpr int kSfaR = kChunksR * 512;
-  static constexpr int kSfbD = 2 * kChunksR * 512;  // two 128-row blocks of the weight
+  static constexpr int kSfbD = kNRB * kChunksR * 512;
   static constexpr int kSfaB = kChunksB * 512;
-  static constexpr int kSfbS = SPARSE ? 2 * kChunksB * 512 : 0;
+  static constexpr int kSfbS = SPARSE ? kNRB * kChunksB * 512 : 0;
   // stage layout (offsets in bytes)
   static constexpr int oW = 0;
   static constexpr int oR = oW + kWBytes;
@@ -59,22 +79,30 @@ struct GemmCfg {
   static constexpr int oSfaB = oSfbD + kSfbD;
   static constexpr int oSfbS = oSfaB + kSfaB;
   static constexpr int kStageBytes = ((oSfbS + kSfbS + 1023) / 1024) * 1024;
-  static constexpr int kStages = (SPARSE && KIND == GK_NVF4) ? 3 : 3;
-  static constexpr uint32_t kTx = kWBytes + kRBytes + kBBytes + kEBytes + kSfaR + kSfbD + kSfaB + kSfbS;
+  static constexpr int kStages = kUnpacked ? 2 : 3;
+  // transaction bytes: unpacking loads count the packed (global) size, half their smem footprint
+  static constexpr uint32_t kTx = (kWBytes + kRBytes + kBBytes) / (kUnpacked ? 2 : 1) + kEBytes + kSfaR + kSfbD + kSfaB +
+                                  kSfbS;
   // tensor memory columns: accumulator, then two slots of scales + metadata
   static constexpr int cSfaR = 0;
   static constexpr int cSfbD = cSfaR + 4 * kChunksR;
-  static constexpr int cSfaB = cSfbD + 8 * kChunksR;
+  static constexpr int cSfaB = cSfbD + 4 * kNRB * kChunksR;
   static constexpr int cSfbS = cSfaB + 4 * kChunksB;
-  static constexpr int cE = cSfbS + (SPARSE ? 8 * kChunksB : 0);
-  static constexpr int kSlotCols = cE + (SPARSE ? 4 : 0);
-  static constexpr int kTmemCols = 512;
+  static constexpr int cE = cSfbS + (SPARSE ? 4 * kNRB * kChunksB : 0);
+  static constexpr int kSlotCols = cE + 4 * kEBoxes;
+  static constexpr int kTmemCols = BN + 2 * kSlotCols <= 256 ? 256 : 512;
   static_assert(BN + 2 * kSlotCols <= kTmemCols, "tensor memory budget");
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
-  // instruction descriptor (block-scaled kinds): E2M1 x E2M1, K-major, M=128, N=256
-  static constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                                     ((KIND == GK_MXF4 ? 1u : 0u) << 23) | ((uint32_t)(BM >> 4) << 24);
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  // instruction descriptor (block-scaled kinds): E2M1 x E2M1, K-major, M=128, N=BN
+  static constexpr uint32_t kFmt = kUnpacked ? 5u : 1u;
+  static constexpr uint32_t kIdesc = (kFmt << 7) | (kFmt << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                     ((KIND == GK_NVF4 ? 0u : 1u) << 23) | ((uint32_t)(BM >> 4) << 24);
   static constexpr uint32_t kIdescSp = kIdesc | (1u << 2);
+  // 16-byte-unit offset inside a stage of the dense operand slice for logical K index kk
+  __host__ __device__ static constexpr uint32_t dense_off(int box_bytes, int kk) {
+    return (uint32_t)((kk / kBoxElems) * (box_bytes / 16) + (kUnpacked ? (kk % kBoxElems) / 16 : (kk % kBoxElems) / 32));
+  }
 };
 
 struct GemmParams {
@@ -134,7 +162,7 @@ __global__ void __launch_bounds__(192, 1) gemm_kernel(const __grid_constant__ Ge
     tma_prefetch(&maps.w);
     tma_prefetch(&maps.r);
     tma_prefetch(&maps.b);
-    if (SPARSE) tma_prefetch(&maps.e);
+    if (C::kEBoxes > 0) tma_prefetch(&maps.e);
   }
   tc_fence_before();
   __syncthreads();
@@ -171,41 +199,57 @@ __global__ void __launch_bounds__(192, 1) gemm_kernel(const __grid_constant__ Ge
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued = 0, issued_par = 0;  // per stage: ever issued / parity of the last batch
+      const uint32_t smem0 = smem_u32(smem), full0 = smem_u32(full);
+      const int64_t sd_blocks = (sd_per_row + 3) / 4, sb_blocks = (sb_per_row + 3) / 4;
+      const int64_t ss_blocks = (p.k / C::kVecSparse + 3) / 4;
       for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x) {
         const int mt = tile % m_tiles, nt = tile / m_tiles;
         const int64_t m0 = (int64_t)mt * C::BM;
         const int e = tile_expert(m0);
         if (e < 0) continue;
         const int32_t wrow = (int32_t)(e * p.n + (int64_t)nt * C::BN);
+        const int64_t nb = (int64_t)nt * C::kNRB;
+        // scale chunks of this tile: contiguous per 128-row block, advanced per K tile
+        const uint8_t* g_sfa_r = p.sf_res + (m0 / 128) * sd_blocks * 512;
+        const uint8_t* g_sfa_b = p.sf_bb + (m0 / 128) * sb_blocks * 512;
+        const uint8_t* g_sfb_d = p.sf_w_dense + e * wsd_bytes + nb * sd_blocks * 512;
+        const uint8_t* g_sfb_s = p.sf_w_sparse + e * wss_bytes + nb * ss_blocks * 512;
+        int32_t kx = 0, kx_b = 0, kx_e = 0;
         for (int kt = 0; kt < k_tiles; kt++) {
           if (!mbar_wait(&empty[stage], phase ^ 1, p.timeout_ns, abort_flag)) { *abort_flag = 1; break; }
-          uint8_t* sb = smem + stage * C::kStageBytes;
-          mbar_arrive_expect_tx(&full[stage], C::kTx);
-          tma_load_2d(sb + C::oW, &maps.w, kt * C::kRowDense, wrow, &full[stage]);
-          tma_load_2d(sb + C::oR, &maps.r, kt * C::kRowDense, (int32_t)m0, &full[stage]);
-          tma_load_2d(sb + C::oB, &maps.b, kt * C::kRowB, (int32_t)m0, &full[stage]);
-          if constexpr (SPARSE) tma_load_2d(sb + C::oE, &maps.e, kt * C::kRowE, (int32_t)m0, &full[stage]);
-          // scale chunks: contiguous per 128-row block in the tiled layout
-          const int64_t sd_blocks = (sd_per_row + 3) / 4, sb_blocks = (sb_per_row + 3) / 4;
-          bulk_load(sb + C::oSfaR, p.sf_res + ((m0 / 128) * sd_blocks + (int64_t)kt * C::kChunksR) * 512, C::kSfaR,
-                    &full[stage]);
-          bulk_load(sb + C::oSfaB, p.sf_bb + ((m0 / 128) * sb_blocks + (int64_t)kt * C::kChunksB) * 512, C::kSfaB,
-                    &full[stage]);
-          const uint8_t* wd = p.sf_w_dense + e * wsd_bytes;
-          const int64_t nb = (int64_t)nt * 2;
+          const uint32_t sb = smem0 + (uint32_t)(stage * C::kStageBytes);
+          const uint32_t fb = full0 + (uint32_t)(stage * 8);
+          mbar_arrive_expect_tx_u32(fb, C::kTx);
 #pragma unroll
-          for (int rb = 0; rb < 2; rb++)
-            bulk_load(sb + C::oSfbD + rb * C::kChunksR * 512,
-                      wd + ((nb + rb) * sd_blocks + (int64_t)kt * C::kChunksR) * 512, C::kChunksR * 512, &full[stage]);
-          if constexpr (SPARSE) {
-            const uint8_t* ws = p.sf_w_sparse + e * wss_bytes;
-            const int64_t ss_blocks = (p.k / C::kVecSparse + 3) / 4;
-#pragma unroll
-            for (int rb = 0; rb < 2; rb++)
-              bulk_load(sb + C::oSfbS + rb * C::kChunksB * 512,
-                        ws + ((nb + rb) * ss_blocks + (int64_t)kt * C::kChunksB) * 512, C::kChunksB * 512,
-                        &full[stage]);
+          for (int bx = 0; bx < C::kBoxesDense; bx++) {
+            tma_load_2d_u32(sb + C::oW + bx * C::kBoxW, &maps.w, kx + 128 * bx, wrow, fb);
+            tma_load_2d_u32(sb + C::oR + bx * C::kBoxR, &maps.r, kx + 128 * bx, (int32_t)m0, fb);
           }
+#pragma unroll
+          for (int bx = 0; bx < C::kBoxesB; bx++)
+            tma_load_2d_u32(sb + C::oB + bx * C::BM * C::kRowB, &maps.b, kx_b + 128 * bx, (int32_t)m0, fb);
+#pragma unroll
+          for (int bx = 0; bx < C::kEBoxes; bx++)
+            tma_load_2d_u32(sb + C::oE + bx * C::BM * 16, &maps.e, kx_e + 16 * bx, (int32_t)m0, fb);
+          bulk_load_u32(sb + C::oSfaR, g_sfa_r, C::kSfaR, fb);
+          bulk_load_u32(sb + C::oSfaB, g_sfa_b, C::kSfaB, fb);
+#pragma unroll
+          for (int rb = 0; rb < C::kNRB; rb++)
+            bulk_load_u32(sb + C::oSfbD + rb * C::kChunksR * 512, g_sfb_d + rb * sd_blocks * 512, C::kChunksR * 512,
+                          fb);
+          if constexpr (SPARSE) {
+#pragma unroll
+            for (int rb = 0; rb < C::kNRB; rb++)
+              bulk_load_u32(sb + C::oSfbS + rb * C::kChunksB * 512, g_sfb_s + rb * ss_blocks * 512,
+                            C::kChunksB * 512, fb);
+          }
+          kx += C::kXStage;
+          kx_b += C::kXStageB;
+          kx_e += C::kMetaStage;
+          g_sfa_r += C::kSfaR;
+          g_sfa_b += C::kSfaB;
+          g_sfb_d += C::kChunksR * 512;
+          g_sfb_s += C::kChunksB * 512;
           issued |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
@@ -224,6 +268,12 @@ __global__ void __launch_bounds__(192, 1) gemm_kernel(const __grid_constant__ Ge
       uint32_t phase = 0;
       int it = 0;
       const uint32_t acc = tmem_base;
+      // descriptor halves: start addresses in 16-byte units (stage 0), constant high words
+      constexpr uint32_t kHi128 = desc_hi(1024, 2), kHi64 = desc_hi(512, 4), kHiCp = desc_hi(128, 0);
+      constexpr uint32_t kHiB = (SPARSE && !C::kUnpacked) ? kHi64 : kHi128;  // backbone rows of 64 or 128 bytes
+      constexpr uint32_t kLbo = 1u << 16;  // 16-byte leading offset (ignored by swizzled K-major layouts)
+      const uint32_t lo0 = smem_u32(smem) >> 4;
+      const uint32_t empty0 = smem_u32(empty);
       for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x, it++) {
         const int mt = tile % m_tiles;
         if (tile_expert((int64_t)mt * C::BM) < 0) { it--; continue; }
@@ -233,80 +283,90 @@ __global__ void __launch_bounds__(192, 1) gemm_kernel(const __grid_constant__ Ge
         for (int kt = 0; kt < k_tiles; kt++) {
           if (!mbar_wait(&full[stage], phase, p.timeout_ns, abort_flag)) { *abort_flag = 1; break; }
           tc_fence_after();
-          const uint8_t* sb = smem + stage * C::kStageBytes;
+          const uint32_t ls = lo0 + (uint32_t)(stage * (C::kStageBytes >> 4));  // stage base, 16-byte units
           const uint32_t slot = tmem_base + C::BN + (uint32_t)((kt & 1) * C::kSlotCols);
           // scale factors and metadata -> tensor memory
 #pragma unroll
           for (int c = 0; c < C::kChunksR; c++) {
-            tc_cp_32x128b_warpx4(slot + C::cSfaR + 4 * c, smem_desc(smem_u32(sb + C::oSfaR + 512 * c), 0, 128, 0));
+            tc_cp_32x128b_warpx4(slot + C::cSfaR + 4 * c, desc_lohi(ls + (C::oSfaR >> 4) + 32 * c, kHiCp));
 #pragma unroll
-            for (int rb = 0; rb < 2; rb++)
-              tc_cp_32x128b_warpx4(slot + C::cSfbD + 8 * c + 4 * rb,
-                                   smem_desc(smem_u32(sb + C::oSfbD + (rb * C::kChunksR + c) * 512), 0, 128, 0));
+            for (int rb = 0; rb < C::kNRB; rb++)
+              tc_cp_32x128b_warpx4(slot + C::cSfbD + 4 * C::kNRB * c + 4 * rb,
+                                   desc_lohi(ls + ((C::oSfbD + rb * C::kChunksR * 512) >> 4) + 32 * c, kHiCp));
           }
 #pragma unroll
           for (int c = 0; c < C::kChunksB; c++) {
-            tc_cp_32x128b_warpx4(slot + C::cSfaB + 4 * c, smem_desc(smem_u32(sb + C::oSfaB + 512 * c), 0, 128, 0));
+            tc_cp_32x128b_warpx4(slot + C::cSfaB + 4 * c, desc_lohi(ls + (C::oSfaB >> 4) + 32 * c, kHiCp));
             if constexpr (SPARSE) {
 #pragma unroll
-              for (int rb = 0; rb < 2; rb++)
-                tc_cp_32x128b_warpx4(slot + C::cSfbS + 8 * c + 4 * rb,
-                                     smem_desc(smem_u32(sb + C::oSfbS + (rb * C::kChunksB + c) * 512), 0, 128, 0));
+              for (int rb = 0; rb < C::kNRB; rb++)
+                tc_cp_32x128b_warpx4(slot + C::cSfbS + 4 * C::kNRB * c + 4 * rb,
+                                     desc_lohi(ls + ((C::oSfbS + rb * C::kChunksB * 512) >> 4) + 32 * c, kHiCp));
             }
           }
-          if constexpr (SPARSE) tc_cp_128x128b(slot + C::cE, smem_desc(smem_u32(sb + C::oE), 0, 128, 0));
+#pragma unroll
+          for (int bx = 0; bx < C::kEBoxes; bx++)
+            tc_cp_128x128b(slot + C::cE + 4 * bx, desc_lohi(ls + ((C::oE + bx * C::BM * 16) >> 4), kHiCp));
 
-          const uint32_t w_base = smem_u32(sb + C::oW);
           if (run_sparse) {
             if constexpr (SPARSE) {
-              // backbone: sparse MMAs, K = 128 logical each (64 stored FP4 = 32 bytes of A)
+              // backbone: sparse MMAs (32 bytes of compressed A, 64 bytes of W per MMA)
 #pragma unroll
               for (int kb = 0; kb < C::BK / C::kSparseMmaK; kb++) {
-                const int s0 = kb * (C::kSparseMmaK / C::kVecSparse);
-                const uint32_t chunk = s0 / 4, byte = s0 % 4;
+                constexpr int kScales = C::kSparseMmaK / C::kVecSparse;
+                const uint32_t chunk = (kb * kScales) / 4, byte = (kb * kScales) % 4;
                 const uint32_t idesc = C::kIdescSp | (byte << 29) | (byte << 4);
-                const uint64_t a = smem_desc(smem_u32(sb + C::oB) + kb * 32, 16, 512, 4);   // 64B swizzle
-                const uint64_t b = smem_desc(w_base + kb * 64, 16, 1024, 2);                // 128B swizzle
+                const uint64_t a = desc_lohi((ls + (C::oB >> 4) + 2 * kb) | kLbo, kHiB);
+                const uint32_t wo = (uint32_t)((kb * 64) / 128 * (C::kBoxW / 16) + ((kb * 64) % 128) / 16);
+                const uint64_t b = desc_lohi((ls + (C::oW >> 4) + wo) | kLbo, kHi128);
                 const uint32_t sfa = (slot + C::cSfaB + 4 * chunk) | (byte << 30);
-                const uint32_t sfb = (slot + C::cSfbS + 8 * chunk) | (byte << 30);
-                if constexpr (KIND == GK_NVF4) mma_nvf4_sp(acc, a, b, slot + C::cE + 2 * kb, idesc, sfa, sfb, accumulate);
-                else mma_mxf4_sp(acc, a, b, slot + C::cE + 2 * kb, idesc, sfa, sfb, accumulate);
+                const uint32_t sfb = (slot + C::cSfbS + 4 * C::kNRB * chunk) | (byte << 30);
+                const uint32_t e = slot + C::cE + 2 * kb;
+                if constexpr (KIND == GK_NVF4) mma_nvf4_sp(acc, a, b, e, idesc, sfa, sfb, accumulate);
+                else if constexpr (KIND == GK_MXF4) mma_mxf4_sp(acc, a, b, e, idesc, sfa, sfb, accumulate);
+                else mma_mxf8f6f4_sp(acc, a, b, e, idesc, sfa, sfb, accumulate);
                 accumulate = 1;
               }
             } else {
               // dense backbone (8:16): same as the residual path over the expanded backbone
 #pragma unroll
               for (int kb = 0; kb < C::BK / C::kDenseMmaK; kb++) {
-                const int s0 = kb * (C::kDenseMmaK / C::kVecDense);
-                const uint32_t chunk = s0 / 4, byte = s0 % 4;
+                constexpr int kScales = C::kDenseMmaK / C::kVecDense;
+                const uint32_t chunk = (kb * kScales) / 4, byte = (kb * kScales) % 4;
                 const uint32_t idesc = C::kIdesc | (byte << 29) | (byte << 4);
-                const uint64_t a = smem_desc(smem_u32(sb + C::oB) + kb * 32, 16, 1024, 2);
-                const uint64_t b = smem_desc(w_base + kb * 32, 16, 1024, 2);
+                const uint64_t a = desc_lohi((ls + (C::oB >> 4) + C::dense_off(C::BM * 128, kb * C::kDenseMmaK)) | kLbo,
+                                             kHi128);
+                const uint64_t b = desc_lohi((ls + (C::oW >> 4) + C::dense_off(C::kBoxW, kb * C::kDenseMmaK)) | kLbo,
+                                             kHi128);
                 const uint32_t sfa = (slot + C::cSfaB + 4 * chunk) | (byte << 30);
-                const uint32_t sfb = (slot + C::cSfbD + 8 * chunk) | (byte << 30);
+                const uint32_t sfb = (slot + C::cSfbD + 4 * C::kNRB * chunk) | (byte << 30);
                 if constexpr (KIND == GK_NVF4) mma_nvf4(acc, a, b, idesc, sfa, sfb, accumulate);
-                else mma_mxf4(acc, a, b, idesc, sfa, sfb, accumulate);
+                else if constexpr (KIND == GK_MXF4) mma_mxf4(acc, a, b, idesc, sfa, sfb, accumulate);
+                else mma_mxf8f6f4(acc, a, b, idesc, sfa, sfb, accumulate);
                 accumulate = 1;
               }
             }
           }
           if (run_dense) {
-            // residual: dense MMAs, K = 64 each (32 bytes of A and of W), same W tile
+            // residual: dense MMAs over the same W tile
 #pragma unroll
             for (int kb = 0; kb < C::BK / C::kDenseMmaK; kb++) {
-              const int s0 = kb * (C::kDenseMmaK / C::kVecDense);
-              const uint32_t chunk = s0 / 4, byte = s0 % 4;
+              constexpr int kScales = C::kDenseMmaK / C::kVecDense;
+              const uint32_t chunk = (kb * kScales) / 4, byte = (kb * kScales) % 4;
               const uint32_t idesc = C::kIdesc | (byte << 29) | (byte << 4);
-              const uint64_t a = smem_desc(smem_u32(sb + C::oR) + kb * 32, 16, 1024, 2);
-              const uint64_t b = smem_desc(w_base + kb * 32, 16, 1024, 2);
+              const uint64_t a = desc_lohi((ls + (C::oR >> 4) + C::dense_off(C::kBoxR, kb * C::kDenseMmaK)) | kLbo,
+                                           kHi128);
+              const uint64_t b = desc_lohi((ls + (C::oW >> 4) + C::dense_off(C::kBoxW, kb * C::kDenseMmaK)) | kLbo,
+                                           kHi128);
               const uint32_t sfa = (slot + C::cSfaR + 4 * chunk) | (byte << 30);
-              const uint32_t sfb = (slot + C::cSfbD + 8 * chunk) | (byte << 30);
+              const uint32_t sfb = (slot + C::cSfbD + 4 * C::kNRB * chunk) | (byte << 30);
               if constexpr (KIND == GK_NVF4) mma_nvf4(acc, a, b, idesc, sfa, sfb, accumulate);
-              else mma_mxf4(acc, a, b, idesc, sfa, sfb, accumulate);
+              else if constexpr (KIND == GK_MXF4) mma_mxf4(acc, a, b, idesc, sfa, sfb, accumulate);
+              else mma_mxf8f6f4(acc, a, b, idesc, sfa, sfb, accumulate);
               accumulate = 1;
             }
           }
-          tc_commit(&empty[stage]);
+          tc_commit_u32(empty0 + (uint32_t)(stage * 8));
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
         }
         if (*abort_flag) break;

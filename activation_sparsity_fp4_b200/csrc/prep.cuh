@@ -6,14 +6,13 @@
 // to FP4 as well; "a fused preprocessing kernel absorbs mask generation,
 // residual construction and layer normalization into one operator".
 //
-// Work split: one thread owns 32 consecutive K elements of one row (one
-// "unit"): 4 x 16-byte loads of bf16 (8 for fp32).  For NVFP4 a unit is exactly
-// one backbone block (16 kept values) and two residual blocks; for MXFP4 a
-// backbone block spans the two units of a lane pair (shuffle for its amax) and
-// a residual block is one unit.  A row is handled by ceil(K/32) threads rounded
-// up to whole warps; small K packs several rows into one block.  Every floating
-// point step is an explicitly rounded fp32 op in a fixed order, so codes and
-// scales are reproducible bit for bit.
+// Work split: a thread owns 32 consecutive K elements (one "unit": 4 x
+// 16-byte loads of bf16, 8 of fp32); a power-of-two number of threads (8..128)
+// shares a row, several rows share a block of 128 threads when rows are short.
+// For NVFP4 a unit is exactly one backbone block (16 kept values) and two
+// residual blocks; for MXFP4 a backbone block spans the units of a lane pair
+// (shuffle for its amax) and a residual block is one unit.  Every floating point step is an explicitly rounded fp32 op
+// in a fixed order, so codes and scales are reproducible bit for bit.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -76,43 +75,46 @@ __device__ __forceinline__ void load_unit(const void* base, int64_t off, float (
   }
 }
 
-// Sum of squares of one row in the fixed order: 16-element chunk sums by
-// sequential FMA, then a pairwise tree of adjacent chunks (levels 1..5 inside
-// the warp by xor shuffles, the rest over the row's warps, zero padded).
-// All threads of the block must call it.  red: per-block scratch [rows][32].
-template <bool XBF16>
-__device__ __forceinline__ float row_rstd(const float (&x)[32], bool active, float eps, int64_t k, float* red,
-                                          int row_in_block, int warps_per_row) {
-  float c0 = 0.0f, c1 = 0.0f;
-  if (active) {
+// Two E2M1 codes (low nibble = first element) -> exact fp32 values.
+__device__ __forceinline__ void e2m1x2_values(uint32_t c, float& lo, float& hi) {
+  uint32_t h2;
+  const uint16_t byte = (uint16_t)(c & 0xFF);
+  asm("{\n\t.reg .b8 t;\n\tcvt.u8.u16 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(h2) : "h"(byte));
+  lo = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFF)));
+  hi = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+}
+
+// Eight E2M1 codes (nibbles of c, element i in nibble i) -> exact fp32 values.
+__device__ __forceinline__ void e2m1x8_values(uint32_t c, float* out) {
 #pragma unroll
-    for (int i = 0; i < 16; i++) c0 = __fmaf_rn(x[i], x[i], c0);
-#pragma unroll
-    for (int i = 16; i < 32; i++) c1 = __fmaf_rn(x[i], x[i], c1);
+  for (int b = 0; b < 4; b++) {
+    uint32_t h2;
+    const uint16_t byte = (uint16_t)((c >> (8 * b)) & 0xFF);
+    asm("{\n\t.reg .b8 t;\n\tcvt.u8.u16 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(h2) : "h"(byte));
+    out[2 * b] = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFF)));
+    out[2 * b + 1] = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
   }
-  float s = __fadd_rn(c0, c1);
-#pragma unroll
-  for (int m = 1; m < 32; m <<= 1) s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, m));
-  const int warp_in_row = threadIdx.x >> 5;
-  if ((threadIdx.x & 31) == 0) red[row_in_block * 32 + warp_in_row] = s;
-  __syncthreads();
-  // adjacent-pair tree over the row's warp sums, zero padded to 16 leaves (a
-  // larger zero padding than the minimal power of two adds only x + 0 = x)
-  float a[16];
-#pragma unroll
-  for (int i = 0; i < 16; i++) a[i] = (i < warps_per_row) ? red[row_in_block * 32 + i] : 0.0f;
-#pragma unroll
-  for (int w = 16; w > 1; w >>= 1)
-#pragma unroll
-    for (int i = 0; i < w / 2; i++) a[i] = __fadd_rn(a[2 * i], a[2 * i + 1]);
-  const float mean = __fdiv_rn(a[0], (float)k);
-  return __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(mean, eps)));
 }
 
 // ------------------------------------------------------------------- mask
 // keep bits (bit i = element i of the unit kept) and metadata for 32 values.
-// Ranks: element i is kept iff fewer than N elements of its group beat it,
-// where j beats i if |h_j| > |h_i|, or equal and j < i.
+// Element (pair) i is kept iff fewer than N of its group beat it, where j
+// beats i if |h_j| > |h_i|, or they are equal and j < i.
+__device__ __forceinline__ uint32_t top2of4(float a0, float a1, float a2, float a3) {
+  const int b01 = a0 >= a1, b02 = a0 >= a2, b03 = a0 >= a3, b12 = a1 >= a2, b13 = a1 >= a3, b23 = a2 >= a3;
+  const int n0 = 3 - b01 - b02 - b03;
+  const int n1 = b01 + 2 - b12 - b13;
+  const int n2 = b02 + b12 + 1 - b23;
+  const int n3 = b03 + b13 + b23;
+  return (uint32_t)(n0 < 2) | ((uint32_t)(n1 < 2) << 1) | ((uint32_t)(n2 < 2) << 2) | ((uint32_t)(n3 < 2) << 3);
+}
+// metadata nibble (i0 | i1 << 2) of a 4-bit mask with exactly two bits set
+__device__ __forceinline__ uint32_t pair_nibble(uint32_t kp) {
+  // kp: 0b0011 -> 4, 0b0101 -> 8, 0b0110 -> 9, 0b1001 -> 12, 0b1010 -> 13, 0b1100 -> 14
+  constexpr uint64_t LUT = (4ull << 12) | (8ull << 20) | (9ull << 24) | (12ull << 36) | (13ull << 40) | (14ull << 48);
+  return (uint32_t)(LUT >> (4 * kp)) & 15u;
+}
+
 template <int PAT>
 __device__ __forceinline__ uint32_t unit_mask(const float (&h)[32], uint32_t& meta) {
   uint32_t keep = 0;
@@ -120,46 +122,20 @@ __device__ __forceinline__ uint32_t unit_mask(const float (&h)[32], uint32_t& me
   if constexpr (PAT == PAT_48P) {
 #pragma unroll
     for (int g = 0; g < 4; g++) {
-      float sc[4];
-#pragma unroll
-      for (int p = 0; p < 4; p++) sc[p] = fmaxf(fabsf(h[8 * g + 2 * p]), fabsf(h[8 * g + 2 * p + 1]));
-      uint32_t kp = 0;
-#pragma unroll
-      for (int p = 0; p < 4; p++) {
-        int beat = 0;
-#pragma unroll
-        for (int q = 0; q < 4; q++) {
-          if (q < p) beat += (sc[q] >= sc[p]) ? 1 : 0;
-          if (q > p) beat += (sc[q] > sc[p]) ? 1 : 0;
-        }
-        kp |= (beat < 2 ? 1u : 0u) << p;
-      }
-      // kept pair indices p0 < p1
-      const int p0 = __ffs(kp) - 1;
-      const int p1 = 31 - __clz(kp);
-      meta |= (uint32_t)(p0 | (p1 << 2)) << (4 * g);
-      keep |= (3u << (8 * g + 2 * p0)) | (3u << (8 * g + 2 * p1));
+      const float* hg = h + 8 * g;
+      const uint32_t kp = top2of4(fmaxf(fabsf(hg[0]), fabsf(hg[1])), fmaxf(fabsf(hg[2]), fabsf(hg[3])),
+                                  fmaxf(fabsf(hg[4]), fabsf(hg[5])), fmaxf(fabsf(hg[6]), fabsf(hg[7])));
+      meta |= pair_nibble(kp) << (4 * g);
+      // spread pair bits to element bits: pair p -> elements 2p, 2p+1
+      uint32_t e = (kp & 1u) | ((kp & 2u) << 1) | ((kp & 4u) << 2) | ((kp & 8u) << 3);
+      keep |= (e | (e << 1)) << (8 * g);
     }
   } else if constexpr (PAT == PAT_24) {
 #pragma unroll
     for (int g = 0; g < 8; g++) {
-      float a[4];
-#pragma unroll
-      for (int i = 0; i < 4; i++) a[i] = fabsf(h[4 * g + i]);
-      uint32_t kg = 0;
-#pragma unroll
-      for (int i = 0; i < 4; i++) {
-        int beat = 0;
-#pragma unroll
-        for (int j = 0; j < 4; j++) {
-          if (j < i) beat += (a[j] >= a[i]) ? 1 : 0;
-          if (j > i) beat += (a[j] > a[i]) ? 1 : 0;
-        }
-        kg |= (beat < 2 ? 1u : 0u) << i;
-      }
-      const int i0 = __ffs(kg) - 1;
-      const int i1 = 31 - __clz(kg);
-      meta |= (uint32_t)(i0 | (i1 << 2)) << (4 * g);
+      const float* hg = h + 4 * g;
+      const uint32_t kg = top2of4(fabsf(hg[0]), fabsf(hg[1]), fabsf(hg[2]), fabsf(hg[3]));
+      meta |= pair_nibble(kg) << (4 * g);
       keep |= kg << (4 * g);
     }
   } else {
@@ -199,45 +175,32 @@ __device__ __forceinline__ float pow2f(int e) {  // exact 2^e for e in [-127, 12
   return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(0x00400000u);
 }
 
-// Quantize n (multiple of 8) values with one scale: writes packed codes
-// (n/8 words) and the dequantized values (with g_dec); returns the scale code.
-template <int FMT, int N>
-__device__ __forceinline__ uint32_t quant_block(const float* v, float amax, float g_enc, float g_dec,
-                                                uint32_t* codes, float* deq) {
-  float q[N];
-  uint32_t sc;
+// Block scale: returns the scale code, the multiplier that maps values onto the
+// E2M1 grid (0 means "all codes +0") and the decoded scale (times g_dec for
+// the dequantized value: deq = (e2m1 * sv) * g_dec for NVFP4, e2m1 * sv for MX).
+// NVFP4: s = (amax / 6) * g_enc, S = E4M3(s), mul = g_enc / S (exact table).
+template <int FMT>
+__device__ __forceinline__ uint32_t block_scale(float amax, float g_enc, const float* inv_tab, float& mul, float& sv) {
   if constexpr (FMT == FMT_MX) {
     const int e = mx_exponent(amax);
-    sc = (uint32_t)(e + 127);
-    const float mul = pow2f(-e);
-    const float dsc = pow2f(e);
-#pragma unroll
-    for (int i = 0; i < N; i++) q[i] = __fmul_rn(v[i], mul);
-#pragma unroll
-    for (int w = 0; w < N / 8; w++) codes[w] = cvt_e2m1x8(q + 8 * w);
-#pragma unroll
-    for (int i = 0; i < N; i++) deq[i] = __fmul_rn(e2m1_value((codes[i / 8] >> (4 * (i % 8))) & 15), dsc);
+    mul = pow2f(-e);
+    sv = pow2f(e);
+    return (uint32_t)(e + 127);
   } else {
-    const float s32 = __fmul_rn(__fdiv_rn(amax, 6.0f), g_enc);
-    sc = cvt_e4m3(s32);
-    const float sv = e4m3_value(sc);
-    if (sv == 0.0f) {
-#pragma unroll
-      for (int w = 0; w < N / 8; w++) codes[w] = 0;
-#pragma unroll
-      for (int i = 0; i < N; i++) deq[i] = 0.0f;
-    } else {
-      const float inv = __fdiv_rn(g_enc, sv);
-#pragma unroll
-      for (int i = 0; i < N; i++) q[i] = __fmul_rn(v[i], inv);
-#pragma unroll
-      for (int w = 0; w < N / 8; w++) codes[w] = cvt_e2m1x8(q + 8 * w);
-#pragma unroll
-      for (int i = 0; i < N; i++)
-        deq[i] = __fmul_rn(__fmul_rn(e2m1_value((codes[i / 8] >> (4 * (i % 8))) & 15), sv), g_dec);
-    }
+    const uint32_t sc = cvt_e4m3(__fmul_rn(__fdiv_rn(amax, 6.0f), g_enc));
+    sv = e4m3_value(sc);
+    mul = inv_tab[sc];  // 0 for code 0
+    return sc;
   }
-  return sc;
+}
+
+// Quantize 8 values: returns 8 codes (nibbles); mul = 0 gives +0 codes.
+__device__ __forceinline__ uint32_t quant8(const float* v, float mul) {
+  float q[8];
+#pragma unroll
+  for (int i = 0; i < 8; i++) q[i] = __fmul_rn(v[i], mul);
+  const uint32_t c = cvt_e2m1x8(q);
+  return mul == 0.0f ? 0u : c;
 }
 
 // tensor scale from the amax (same rule as the weights'): g_enc = 2688 / A,
@@ -253,249 +216,353 @@ __device__ __forceinline__ void tensor_scales(float amax, float& g_enc, float& g
   g_dec = __fdiv_rn(amax, 2688.0f);
 }
 
+// Exact table of g_enc / value(code) for the E4M3 codes 1..126 (code 0 -> 0).
+// Needs >= 128 threads in the block and a __syncthreads() after.
+__device__ __forceinline__ void fill_inv_table(float* tab, float g_enc) {
+  const int c = threadIdx.x;
+  if (c < 128) tab[c] = (c >= 1 && c <= 126) ? __fdiv_rn(g_enc, e4m3_value((uint32_t)c)) : 0.0f;
+}
+
+// ------------------------------------------------------------ row mapping
+// A block of 128 threads handles kRpb = 128 / tpr rows at a time; tpr threads
+// per row (a power of two, 8..128); thread t of a row owns the units t + tpr*j.
+// Blocks stride over row groups.
+struct RowMap {
+  int tpr;   // threads per row
+  int lg;    // log2(tpr)
+  int units; // units (32 elements) per row
+  int nj;    // units per thread, <= 4
+};
+
+__device__ __forceinline__ RowMap row_map(int64_t k) {
+  RowMap m;
+  m.units = (int)(k / 32);
+  int tpr = 8;
+  while (tpr < m.units && tpr < 128) tpr <<= 1;
+  m.tpr = tpr;
+  m.lg = 31 - __clz(tpr);
+  m.nj = (m.units + tpr - 1) / tpr;
+  return m;
+}
+
+// Sum of squares of the thread's row in the fixed order of the oracle:
+// 16-element chunk sums by sequential FMA; then a pairwise tree of adjacent
+// entries: the two chunks of a unit inside the thread, units across the row's
+// threads by xor butterflies (inside a warp, then across the row's warps via
+// shared memory), then the per-j slab sums pairwise, zero padded to 4.  This
+// equals the tree over all chunks zero padded to a power of two.
+// All threads of the block must call it (it contains __syncthreads()).
+template <bool XBF16>
+__device__ __forceinline__ float row_sumsq(const void* x, int64_t row_off, bool real, const RowMap& m, int t,
+                                           int row_in_block, float* red /* [32 rows][4 warps][4 j] */) {
+  float s[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  const int wlanes = m.tpr < 32 ? m.tpr : 32;
+#pragma unroll
+  for (int j = 0; j < 4; j++) {
+    if (j < m.nj) {
+      const int u = t + m.tpr * j;
+      float c0 = 0.0f, c1 = 0.0f;
+      if (real && u < m.units) {
+        float v[32];
+        load_unit<XBF16>(x, row_off + (int64_t)u * 32, v);
+#pragma unroll
+        for (int i = 0; i < 16; i++) c0 = __fmaf_rn(v[i], v[i], c0);
+#pragma unroll
+        for (int i = 16; i < 32; i++) c1 = __fmaf_rn(v[i], v[i], c1);
+      }
+      float a = __fadd_rn(c0, c1);
+      for (int msk = 1; msk < wlanes; msk <<= 1) a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, msk));
+      s[j] = a;
+    }
+  }
+  if (m.tpr > 32) {
+    const int w = t >> 5, nw = m.tpr >> 5;
+    if ((t & 31) == 0) {
+#pragma unroll
+      for (int j = 0; j < 4; j++) red[(row_in_block * 4 + w) * 4 + j] = s[j];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+      const float w0 = red[(row_in_block * 4 + 0) * 4 + j], w1 = red[(row_in_block * 4 + 1) * 4 + j];
+      if (nw == 2) {
+        s[j] = __fadd_rn(w0, w1);
+      } else {
+        const float w2 = red[(row_in_block * 4 + 2) * 4 + j], w3 = red[(row_in_block * 4 + 3) * 4 + j];
+        s[j] = __fadd_rn(__fadd_rn(w0, w1), __fadd_rn(w2, w3));
+      }
+    }
+    __syncthreads();
+  }
+  return __fadd_rn(__fadd_rn(s[0], s[1]), __fadd_rn(s[2], s[3]));
+}
+
+__device__ __forceinline__ float rstd_from_sumsq(float sumsq, int64_t k, float eps) {
+  const float mean = __fdiv_rn(sumsq, (float)k);
+  return __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(mean, eps)));
+}
+
 // ------------------------------------------------------------ amax kernel
-// max |h| over all rows, atomically folded into tensor[0] (zeroed beforehand).
-// Grid-stride over row groups so that only one atomic per block is issued.
+// max |h| over all rows, folded into out[0] (zeroed beforehand) with one
+// atomic per block.
 template <bool NORM, bool XBF16>
-__global__ void __launch_bounds__(512) amax_kernel(const void* x, const void* gamma, float eps, int64_t t, int64_t k,
-                                                   float* out, int rows_per_block, int threads_per_row) {
-  __shared__ float red[16 * 32];
-  __shared__ float bmax[16];
-  const int row_in_block = threadIdx.y;
-  const int u = threadIdx.x;
-  const int units = (int)(k / 32);
-  const bool in_row = u < units;
-  const int warps_per_row = threads_per_row / 32;
+__global__ void __launch_bounds__(128) amax_kernel(const void* x, const void* gamma, float eps, int64_t t, int64_t k,
+                                                   float* out) {
+  __shared__ float red[32 * 16];
+  __shared__ float wmax[4];
+  const RowMap m = row_map(k);
+  const int rpb = 128 / m.tpr;
+  const int row_in_block = threadIdx.x >> m.lg, tt = threadIdx.x & (m.tpr - 1);
   float my = 0.0f;
-  for (int64_t r0 = (int64_t)blockIdx.x * rows_per_block; r0 < t; r0 += (int64_t)gridDim.x * rows_per_block) {
+  for (int64_t r0 = (int64_t)blockIdx.x * rpb; r0 < t; r0 += (int64_t)gridDim.x * rpb) {
     const int64_t r = r0 + row_in_block;
-    const bool active = in_row && r < t;
-    float v[32];
-    if (active) load_unit<XBF16>(x, r * k + (int64_t)u * 32, v);
-    else {
+    const bool real = r < t;
+    const int64_t off = r * k;
+    float rs = 1.0f;
+    if constexpr (NORM) rs = rstd_from_sumsq(row_sumsq<XBF16>(x, off, real, m, tt, row_in_block, red), k, eps);
+    for (int j = 0; j < m.nj; j++) {
+      const int u = tt + m.tpr * j;
+      if (!real || u >= m.units) continue;
+      float v[32];
+      load_unit<XBF16>(x, off + (int64_t)u * 32, v);
+      if constexpr (NORM) {
+        float g[32];
+        load_unit<XBF16>(gamma, (int64_t)u * 32, g);
 #pragma unroll
-      for (int i = 0; i < 32; i++) v[i] = 0.0f;
+        for (int i = 0; i < 32; i++) my = fmaxf(my, fabsf(__fmul_rn(__fmul_rn(v[i], rs), g[i])));
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; i++) my = fmaxf(my, fabsf(v[i]));
+      }
     }
-    if constexpr (NORM) {
-      const float rs = row_rstd<XBF16>(v, active, eps, k, red, row_in_block, warps_per_row);
-      float g[32];
-      if (active) load_unit<XBF16>(gamma, (int64_t)u * 32, g);
-#pragma unroll
-      for (int i = 0; i < 32; i++) v[i] = active ? __fmul_rn(__fmul_rn(v[i], rs), g[i]) : 0.0f;
-      __syncthreads();  // red[] is reused by the next row group
-    }
-#pragma unroll
-    for (int i = 0; i < 32; i++) my = fmaxf(my, fabsf(v[i]));
   }
 #pragma unroll
-  for (int m = 16; m >= 1; m >>= 1) my = fmaxf(my, __shfl_xor_sync(0xffffffffu, my, m));
-  const int tid = threadIdx.y * blockDim.x + threadIdx.x;
-  if ((tid & 31) == 0) bmax[tid >> 5] = my;
+  for (int msk = 16; msk >= 1; msk >>= 1) my = fmaxf(my, __shfl_xor_sync(0xffffffffu, my, msk));
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = my;
   __syncthreads();
-  if (tid == 0) {
-    float m = 0.0f;
-    const int nw = (blockDim.x * blockDim.y) / 32;
-    for (int i = 0; i < nw; i++) m = fmaxf(m, bmax[i]);
-    atomicMax(reinterpret_cast<unsigned int*>(out), __float_as_uint(m));
+  if (threadIdx.x == 0) {
+    const float mm = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
+    atomicMax(reinterpret_cast<unsigned int*>(out), __float_as_uint(mm));
   }
 }
 
 // ------------------------------------------------------------ prep kernel
-template <int FMT, int PAT, bool NORM, bool XBF16>
-__global__ void __launch_bounds__(512) prep_kernel(PrepParams p, int rows_per_block, int threads_per_row) {
-  __shared__ float red[16 * 32];
-  const int row_in_block = threadIdx.y;
-  const int u = threadIdx.x;  // unit index in the row
-  const int64_t k = p.k;
-  const int units = (int)(k / 32);
-  const int64_t r = (int64_t)blockIdx.x * rows_per_block + row_in_block;
-  const bool in_row = u < units;
-  const bool real = in_row && r < p.t;        // a row of the input
-  const bool store = in_row && r < p.t_pad;   // padding rows are written as zero input
-
-  float h[32];
-  if (real) load_unit<XBF16>(p.x, r * k + (int64_t)u * 32, h);
-  else {
+// One unit of 32 values: mask, backbone quantization, residual (in place in
+// h) and residual quantization.  Outputs: meta bits, backbone codes (k/2
+// kept codes: 2 words; 8:16 dense layout: 4 words) and scale, residual codes
+// (4 words) and scales.
+template <int FMT, int PAT>
+__device__ __forceinline__ void quantize_unit(float (&h)[32], float g_enc, float g_dec, const float* inv_tab,
+                                              uint32_t& meta, uint32_t (&bc)[4], uint32_t& bsc, uint32_t (&rc)[4],
+                                              uint32_t& rsc0, uint32_t& rsc1) {
+  // the group maximum is always kept, so the backbone block amax is the window amax
+  float bamax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 32; i++) h[i] = 0.0f;
-  }
-  if constexpr (NORM) {
-    const float rs = row_rstd<XBF16>(h, real, p.eps, k, red, row_in_block, threads_per_row / 32);
-    float g[32];
-    if (real) load_unit<XBF16>(p.gamma, (int64_t)u * 32, g);
-#pragma unroll
-    for (int i = 0; i < 32; i++) h[i] = real ? __fmul_rn(__fmul_rn(h[i], rs), g[i]) : 0.0f;
-  }
+  for (int i = 0; i < 32; i++) bamax = fmaxf(bamax, fabsf(h[i]));
+  if constexpr (FMT == FMT_MX) bamax = fmaxf(bamax, __shfl_xor_sync(0xffffffffu, bamax, 1));
+  float bmul, bsv;
+  bsc = block_scale<FMT>(bamax, g_enc, inv_tab, bmul, bsv);
+  const float dsc = FMT == FMT_NV ? g_dec : 1.0f;
+  meta = 0;
+  bc[0] = bc[1] = bc[2] = bc[3] = 0;
 
-  float g_enc = 1.0f, g_dec = 1.0f;
-  if constexpr (FMT == FMT_NV) {
-    const float amax = p.act_amax > 0.0f ? p.act_amax : *reinterpret_cast<volatile const float*>(p.tensor);
-    tensor_scales(amax, g_enc, g_dec);
-    if (blockIdx.x == 0 && threadIdx.x == 0 && threadIdx.y == 0) {
-      p.tensor[0] = amax;
-      p.tensor[1] = g_enc;
-      p.tensor[2] = g_dec;
+  if constexpr (PAT == PAT_48P) {
+#pragma unroll
+    for (int g = 0; g < 4; g++) {
+      float* hg = h + 8 * g;
+      const uint32_t kp = top2of4(fmaxf(fabsf(hg[0]), fabsf(hg[1])), fmaxf(fabsf(hg[2]), fabsf(hg[3])),
+                                  fmaxf(fabsf(hg[4]), fabsf(hg[5])), fmaxf(fabsf(hg[6]), fabsf(hg[7])));
+      const uint32_t nib = pair_nibble(kp);
+      meta |= nib << (4 * g);
+      const int p0 = nib & 3, p1 = nib >> 2;
+      float k4[4];
+      k4[0] = (p0 == 0) ? hg[0] : (p0 == 1) ? hg[2] : hg[4];
+      k4[1] = (p0 == 0) ? hg[1] : (p0 == 1) ? hg[3] : hg[5];
+      k4[2] = (p1 == 1) ? hg[2] : (p1 == 2) ? hg[4] : hg[6];
+      k4[3] = (p1 == 1) ? hg[3] : (p1 == 2) ? hg[5] : hg[7];
+      const uint32_t c01 = cvt_e2m1x2(__fmul_rn(k4[0], bmul), __fmul_rn(k4[1], bmul));
+      const uint32_t c23 = cvt_e2m1x2(__fmul_rn(k4[2], bmul), __fmul_rn(k4[3], bmul));
+      const uint32_t c4 = bmul == 0.0f ? 0u : (c01 | (c23 << 8));
+      bc[g >> 1] |= c4 << (16 * (g & 1));
+      float d[4];
+      e2m1x2_values(c4 & 0xFF, d[0], d[1]);
+      e2m1x2_values(c4 >> 8, d[2], d[3]);
+#pragma unroll
+      for (int i = 0; i < 4; i++) d[i] = __fmul_rn(__fmul_rn(d[i], bsv), dsc);
+#pragma unroll
+      for (int pp = 0; pp < 4; pp++)
+#pragma unroll
+        for (int jj = 0; jj < 2; jj++) {
+          float& hv = hg[2 * pp + jj];
+          hv = (pp == p0) ? __fsub_rn(hv, d[jj]) : (pp == p1) ? __fsub_rn(hv, d[2 + jj]) : hv;
+        }
+    }
+  } else if constexpr (PAT == PAT_24) {
+#pragma unroll
+    for (int q = 0; q < 8; q++) {
+      float* hq = h + 4 * q;
+      const uint32_t kg = top2of4(fabsf(hq[0]), fabsf(hq[1]), fabsf(hq[2]), fabsf(hq[3]));
+      const uint32_t nib = pair_nibble(kg);
+      meta |= nib << (4 * q);
+      const int i0 = nib & 3, i1 = nib >> 2;
+      const float k0 = (i0 == 0) ? hq[0] : (i0 == 1) ? hq[1] : hq[2];
+      const float k1 = (i1 == 1) ? hq[1] : (i1 == 2) ? hq[2] : hq[3];
+      const uint32_t c2 = bmul == 0.0f ? 0u : cvt_e2m1x2(__fmul_rn(k0, bmul), __fmul_rn(k1, bmul));
+      bc[q >> 2] |= c2 << (8 * (q & 3));
+      float d0, d1;
+      e2m1x2_values(c2, d0, d1);
+      d0 = __fmul_rn(__fmul_rn(d0, bsv), dsc);
+      d1 = __fmul_rn(__fmul_rn(d1, bsv), dsc);
+#pragma unroll
+      for (int jj = 0; jj < 4; jj++) {
+        float& hv = hq[jj];
+        hv = (jj == i0) ? __fsub_rn(hv, d0) : (jj == i1) ? __fsub_rn(hv, d1) : hv;
+      }
     }
   } else {
-    if (blockIdx.x == 0 && threadIdx.x == 0 && threadIdx.y == 0) {
-      p.tensor[0] = 0.0f;
-      p.tensor[1] = 1.0f;
-      p.tensor[2] = 1.0f;
-    }
-  }
-
-  // ---- mask
-  uint32_t meta;
-  const uint32_t keep = unit_mask<PAT>(h, meta);
-
-  // ---- backbone: the 16 kept values in K order
-  float kv[16];
-  if constexpr (PAT == PAT_816) {
-    int n = 0;
+    uint32_t keep = unit_mask<PAT_816>(h, meta);
+    // kept values in K order -> codes; dense layout keeps dropped positions at code 0
+    float kv[16];
 #pragma unroll
     for (int i = 0; i < 32; i++) {
-      // compaction by running count: kept element i goes to slot (popc of keep below i)
       const bool kp = (keep >> i) & 1u;
       const int slot = __popc(keep & ((1u << i) - 1u));
 #pragma unroll
-      for (int s = 0; s < 16; s++)
-        if (kp && slot == s) kv[s] = h[i];
-      n += kp;
+      for (int s2 = 0; s2 < 16; s2++)
+        if (kp && slot == s2) kv[s2] = h[i];
     }
-    (void)n;
-  } else if constexpr (PAT == PAT_48P) {
-    // group g keeps pairs p0 < p1 (from the metadata nibble)
+    const uint32_t cw0 = quant8(kv, bmul), cw1 = quant8(kv + 8, bmul);
+    float bdeq[16];
+    e2m1x8_values(cw0, bdeq);
+    e2m1x8_values(cw1, bdeq + 8);
 #pragma unroll
-    for (int g = 0; g < 4; g++) {
-      const int p0 = (meta >> (4 * g)) & 3, p1 = (meta >> (4 * g + 2)) & 3;
-      const float* hg = h + 8 * g;
-      kv[4 * g + 0] = (p0 == 0) ? hg[0] : (p0 == 1) ? hg[2] : hg[4];
-      kv[4 * g + 1] = (p0 == 0) ? hg[1] : (p0 == 1) ? hg[3] : hg[5];
-      kv[4 * g + 2] = (p1 == 1) ? hg[2] : (p1 == 2) ? hg[4] : hg[6];
-      kv[4 * g + 3] = (p1 == 1) ? hg[3] : (p1 == 2) ? hg[5] : hg[7];
-    }
-  } else {
-    // 2:4 keeps elements i0 < i1 of every quad
-#pragma unroll
-    for (int q = 0; q < 8; q++) {
-      const int i0 = (meta >> (4 * q)) & 3, i1 = (meta >> (4 * q + 2)) & 3;
-      const float* hq = h + 4 * q;
-      kv[2 * q] = (i0 == 0) ? hq[0] : (i0 == 1) ? hq[1] : hq[2];
-      kv[2 * q + 1] = (i1 == 1) ? hq[1] : (i1 == 2) ? hq[2] : hq[3];
-    }
-  }
-  float bamax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 16; i++) bamax = fmaxf(bamax, fabsf(kv[i]));
-  if constexpr (FMT == FMT_MX) bamax = fmaxf(bamax, __shfl_xor_sync(0xffffffffu, bamax, 1));
-  uint32_t bcodes[2];
-  float bdeq[16];
-  const uint32_t bsc = quant_block<FMT, 16>(kv, bamax, g_enc, g_dec, bcodes, bdeq);
-
-  // ---- residual against the quantized backbone
-  float res[32];
-  if constexpr (PAT == PAT_816) {
+    for (int i = 0; i < 16; i++) bdeq[i] = __fmul_rn(__fmul_rn(bdeq[i], bsv), dsc);
+    const uint32_t cw[2] = {cw0, cw1};
 #pragma unroll
     for (int i = 0; i < 32; i++) {
       const bool kp = (keep >> i) & 1u;
       const int slot = __popc(keep & ((1u << i) - 1u));
       float d = 0.0f;
 #pragma unroll
-      for (int s = 0; s < 16; s++)
-        if (slot == s) d = bdeq[s];
-      res[i] = kp ? __fsub_rn(h[i], d) : h[i];
-    }
-  } else if constexpr (PAT == PAT_48P) {
-#pragma unroll
-    for (int g = 0; g < 4; g++) {
-      const int p0 = (meta >> (4 * g)) & 3, p1 = (meta >> (4 * g + 2)) & 3;
-#pragma unroll
-      for (int p = 0; p < 4; p++)
-#pragma unroll
-        for (int j = 0; j < 2; j++) {
-          const float hv = h[8 * g + 2 * p + j];
-          res[8 * g + 2 * p + j] = (p == p0)   ? __fsub_rn(hv, bdeq[4 * g + j])
-                                   : (p == p1) ? __fsub_rn(hv, bdeq[4 * g + 2 + j])
-                                               : hv;
-        }
-    }
-  } else {
-#pragma unroll
-    for (int q = 0; q < 8; q++) {
-      const int i0 = (meta >> (4 * q)) & 3, i1 = (meta >> (4 * q + 2)) & 3;
-#pragma unroll
-      for (int j = 0; j < 4; j++) {
-        const float hv = h[4 * q + j];
-        res[4 * q + j] = (j == i0) ? __fsub_rn(hv, bdeq[2 * q]) : (j == i1) ? __fsub_rn(hv, bdeq[2 * q + 1]) : hv;
-      }
+      for (int s2 = 0; s2 < 16; s2++)
+        if (slot == s2) d = bdeq[s2];
+      h[i] = kp ? __fsub_rn(h[i], d) : h[i];
+      const uint32_t c = (cw[slot >> 3] >> (4 * (slot & 7))) & 15u;
+      bc[i >> 3] |= (kp ? c : 0u) << (4 * (i & 7));
     }
   }
-  uint32_t rcodes[4];
-  float rdeq[32];
-  uint32_t rsc0, rsc1 = 0;
+
+  // residual quantization
   if constexpr (FMT == FMT_NV) {
     float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 16; i++) a0 = fmaxf(a0, fabsf(res[i]));
+    for (int i = 0; i < 16; i++) a0 = fmaxf(a0, fabsf(h[i]));
 #pragma unroll
-    for (int i = 16; i < 32; i++) a1 = fmaxf(a1, fabsf(res[i]));
-    rsc0 = quant_block<FMT, 16>(res, a0, g_enc, g_dec, rcodes, rdeq);
-    rsc1 = quant_block<FMT, 16>(res + 16, a1, g_enc, g_dec, rcodes + 2, rdeq + 16);
+    for (int i = 16; i < 32; i++) a1 = fmaxf(a1, fabsf(h[i]));
+    float m0, m1, sv0, sv1;
+    rsc0 = block_scale<FMT>(a0, g_enc, inv_tab, m0, sv0);
+    rsc1 = block_scale<FMT>(a1, g_enc, inv_tab, m1, sv1);
+    rc[0] = quant8(h, m0);
+    rc[1] = quant8(h + 8, m0);
+    rc[2] = quant8(h + 16, m1);
+    rc[3] = quant8(h + 24, m1);
   } else {
     float a0 = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 32; i++) a0 = fmaxf(a0, fabsf(res[i]));
-    rsc0 = quant_block<FMT, 32>(res, a0, g_enc, g_dec, rcodes, rdeq);
-  }
-
-  if (!store) return;
-  // ---- stores
-  const int64_t K = k;
-  if constexpr (PAT == PAT_48P) {
-    *reinterpret_cast<uint16_t*>(p.meta + r * (K / 16) + 2 * u) = (uint16_t)meta;
-  } else {
-    *reinterpret_cast<uint32_t*>(p.meta + r * (K / 8) + 4 * u) = meta;
-  }
-  if constexpr (PAT == PAT_816) {
-    // dense layout: code of kept element i at position i, 0 elsewhere
-    uint32_t dense[4] = {0, 0, 0, 0};
+    for (int i = 0; i < 32; i++) a0 = fmaxf(a0, fabsf(h[i]));
+    float m0, sv0;
+    rsc0 = block_scale<FMT>(a0, g_enc, inv_tab, m0, sv0);
+    rsc1 = 0;
 #pragma unroll
-    for (int i = 0; i < 32; i++) {
-      const bool kp = (keep >> i) & 1u;
-      const int slot = __popc(keep & ((1u << i) - 1u));
-      const uint32_t c = (bcodes[slot >> 3] >> (4 * (slot & 7))) & 15u;
-      dense[i >> 3] |= (kp ? c : 0u) << (4 * (i & 7));
-    }
-    *reinterpret_cast<uint4*>(p.bb_codes + r * (K / 2) + 16 * u) = make_uint4(dense[0], dense[1], dense[2], dense[3]);
-  } else {
-    *reinterpret_cast<uint2*>(p.bb_codes + r * (K / 4) + 8 * u) = make_uint2(bcodes[0], bcodes[1]);
-  }
-  *reinterpret_cast<uint4*>(p.res_codes + r * (K / 2) + 16 * u) = make_uint4(rcodes[0], rcodes[1], rcodes[2], rcodes[3]);
-
-  if constexpr (FMT == FMT_NV) {
-    // backbone: one scale per 16 kept values (32 logical); 8:16 stores the dense view twice
-    if constexpr (PAT == PAT_816) {
-      const int64_t S = K / 16;
-      *reinterpret_cast<uint16_t*>(p.bb_scales + tiled_sf_offset(r, 2 * u, S)) = (uint16_t)(bsc | (bsc << 8));
-    } else {
-      p.bb_scales[tiled_sf_offset(r, u, K / 32)] = (uint8_t)bsc;
-    }
-    *reinterpret_cast<uint16_t*>(p.res_scales + tiled_sf_offset(r, 2 * u, K / 16)) = (uint16_t)(rsc0 | (rsc1 << 8));
-  } else {
-    if constexpr (PAT == PAT_816) {
-      p.bb_scales[tiled_sf_offset(r, u, K / 32)] = (uint8_t)bsc;
-    } else {
-      if ((u & 1) == 0) p.bb_scales[tiled_sf_offset(r, u >> 1, K / 64)] = (uint8_t)bsc;
-    }
-    p.res_scales[tiled_sf_offset(r, u, K / 32)] = (uint8_t)rsc0;
+    for (int w = 0; w < 4; w++) rc[w] = quant8(h + 8 * w, m0);
   }
 }
 
-// Zero the tiled-scale padding that no thread writes (rows >= t_pad in the last
-// 128-row block and scale columns beyond S in the last 4-column block).
-__global__ void zero_bytes_kernel(uint8_t* p, int64_t n) {
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
-    p[i] = 0;
+template <int FMT, int PAT, bool NORM, bool XBF16>
+__global__ void __launch_bounds__(128, 6) prep_kernel(PrepParams p) {
+  __shared__ float inv_tab[128];
+  __shared__ float red[32 * 16];
+  const int64_t k = p.k;
+  const RowMap m = row_map(k);
+  const int rpb = 128 / m.tpr;
+  const int row_in_block = threadIdx.x >> m.lg, tt = threadIdx.x & (m.tpr - 1);
+
+  float g_enc = 1.0f, g_dec = 1.0f;
+  if constexpr (FMT == FMT_NV) {
+    const float amax = p.act_amax > 0.0f ? p.act_amax : *reinterpret_cast<volatile const float*>(p.tensor);
+    tensor_scales(amax, g_enc, g_dec);
+    fill_inv_table(inv_tab, g_enc);
+    __syncthreads();
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      p.tensor[0] = amax;
+      p.tensor[1] = g_enc;
+      p.tensor[2] = g_dec;
+    }
+  } else if (blockIdx.x == 0 && threadIdx.x == 0) {
+    p.tensor[0] = 0.0f;
+    p.tensor[1] = 1.0f;
+    p.tensor[2] = 1.0f;
+  }
+  const int b = FMT == FMT_NV ? 16 : 32;
+  const int64_t s_res = k / b;
+  const int64_t s_bb = PAT == PAT_816 ? k / b : k / (2 * b);
+
+  for (int64_t r0 = (int64_t)blockIdx.x * rpb; r0 < p.t_pad; r0 += (int64_t)gridDim.x * rpb) {
+    const int64_t r = r0 + row_in_block;
+    const bool in_pad = r < p.t_pad;
+    const bool real = r < p.t;
+    const int64_t off = r * k;
+    float rs = 1.0f;
+    if constexpr (NORM) rs = rstd_from_sumsq(row_sumsq<XBF16>(p.x, off, real, m, tt, row_in_block, red), k, p.eps);
+
+    for (int j = 0; j < m.nj; j++) {
+      const int u = tt + m.tpr * j;
+      const bool active = u < m.units;
+      float h[32];
+      if (real && active) {
+        load_unit<XBF16>(p.x, off + (int64_t)u * 32, h);
+        if constexpr (NORM) {
+          float g[32];
+          load_unit<XBF16>(p.gamma, (int64_t)u * 32, g);
+#pragma unroll
+          for (int i = 0; i < 32; i++) h[i] = __fmul_rn(__fmul_rn(h[i], rs), g[i]);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; i++) h[i] = 0.0f;
+      }
+      uint32_t meta, bc[4], bsc, rc[4], rsc0, rsc1;
+      quantize_unit<FMT, PAT>(h, g_enc, g_dec, inv_tab, meta, bc, bsc, rc, rsc0, rsc1);
+      if (!active || !in_pad) continue;
+
+      if constexpr (PAT == PAT_48P) {
+        *reinterpret_cast<uint16_t*>(p.meta + r * (k / 16) + 2 * u) = (uint16_t)meta;
+      } else {
+        *reinterpret_cast<uint32_t*>(p.meta + r * (k / 8) + 4 * u) = meta;
+      }
+      if constexpr (PAT == PAT_816) {
+        *reinterpret_cast<uint4*>(p.bb_codes + r * (k / 2) + 16 * u) = make_uint4(bc[0], bc[1], bc[2], bc[3]);
+      } else {
+        *reinterpret_cast<uint2*>(p.bb_codes + r * (k / 4) + 8 * u) = make_uint2(bc[0], bc[1]);
+      }
+      *reinterpret_cast<uint4*>(p.res_codes + r * (k / 2) + 16 * u) = make_uint4(rc[0], rc[1], rc[2], rc[3]);
+      if constexpr (FMT == FMT_NV) {
+        if constexpr (PAT == PAT_816) {
+          *reinterpret_cast<uint16_t*>(p.bb_scales + tiled_sf_offset(r, 2 * u, s_bb)) = (uint16_t)(bsc | (bsc << 8));
+        } else {
+          p.bb_scales[tiled_sf_offset(r, u, s_bb)] = (uint8_t)bsc;
+        }
+        *reinterpret_cast<uint16_t*>(p.res_scales + tiled_sf_offset(r, 2 * u, s_res)) = (uint16_t)(rsc0 | (rsc1 << 8));
+      } else {
+        if constexpr (PAT == PAT_816) {
+          p.bb_scales[tiled_sf_offset(r, u, s_bb)] = (uint8_t)bsc;
+        } else {
+          if ((u & 1) == 0) p.bb_scales[tiled_sf_offset(r, u >> 1, s_bb)] = (uint8_t)bsc;
+        }
+        p.res_scales[tiled_sf_offset(r, u, s_res)] = (uint8_t)rsc0;
+      }
+    }
+  }
 }
 
 // --------------------------------------------------------- weight kernel
@@ -532,8 +599,19 @@ __global__ void __launch_bounds__(256) weight_kernel(WeightParams p) {
   for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(v[i]));
   if constexpr (FMT == FMT_MX) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
   uint32_t codes[4];
-  float deq[32];
-  const uint32_t sc = quant_block<FMT, 32>(v, amax, g_enc, g_dec, codes, deq);
+  uint32_t sc;
+  float mul;
+  if constexpr (FMT == FMT_MX) {
+    const int e = mx_exponent(amax);
+    sc = (uint32_t)(e + 127);
+    mul = pow2f(-e);
+  } else {
+    sc = cvt_e4m3(__fmul_rn(__fdiv_rn(amax, 6.0f), g_enc));
+    const float sv = e4m3_value(sc);
+    mul = sv == 0.0f ? 0.0f : __fdiv_rn(g_enc, sv);
+  }
+#pragma unroll
+  for (int w = 0; w < 4; w++) codes[w] = quant8(v + 8 * w, mul);
   if (!active) return;
   if (u == 0 && rl == 0) {
     p.tensor[3 * e + 1] = g_enc;

@@ -101,6 +101,24 @@ sharq_status make_map(CUtensorMap* map, const void* base, int64_t row_bytes, int
   return SHARQ_OK;
 }
 
+// 2-D tensor of packed E2M1 codes [rows][elems] (two per byte) that TMA expands
+// into 8-bit shared-memory containers (16 codes -> 16 bytes); box of 128 codes.
+sharq_status make_map_u4(CUtensorMap* map, const void* base, int64_t elems, int64_t rows, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(SHARQ_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  if (!aligned(base, 32) || (elems / 2) % 32 != 0 || elems % 128 != 0)
+    return fail(SHARQ_ERR_INVALID, "unpacked FP4 operand needs 32-byte aligned rows of a multiple of 128 codes");
+  cuuint64_t dims[2] = {(cuuint64_t)elems, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(elems / 2)};
+  cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SHARQ_ERR_CUDA, "cuTensorMapEncodeTiled (16U4) failed (%d)", (int)r);
+  return SHARQ_OK;
+}
+
 sharq_status check_shape(int64_t k, int64_t n_or_t, bool is_n) {
   if (k <= 0 || k % 256 != 0) return fail(SHARQ_ERR_INVALID, "k=%lld must be a positive multiple of 256", (long long)k);
   if (k > 16384) return fail(SHARQ_ERR_UNSUPPORTED, "k=%lld above 16384", (long long)k);
@@ -111,29 +129,34 @@ sharq_status check_shape(int64_t k, int64_t n_or_t, bool is_n) {
 }
 
 // ---------------------------------------------------------------- launchers
+// Blocks of 128 threads handle 128 / tpr rows at a time (tpr threads per row,
+// see RowMap); as many resident blocks as the SMs hold, striding over rows.
+template <typename Kern>
+unsigned row_grid(Kern kern, int64_t rows, int64_t k) {
+  static int per_sm = 0;
+  if (per_sm == 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 128, 0) != cudaSuccess || per_sm < 1) per_sm = 1;
+  }
+  int tpr = 8;
+  while (tpr < k / 32 && tpr < 128) tpr <<= 1;
+  const int64_t rpb = 128 / tpr;
+  const int64_t groups = (rows + rpb - 1) / rpb;
+  const int64_t cap = (int64_t)sm_count() * per_sm;
+  return (unsigned)(groups < cap ? groups : cap);
+}
+
 template <int FMT, int PAT, bool NORM, bool XBF16>
 sharq_status launch_prep(const PrepParams& pp, cudaStream_t s) {
-  const int units = (int)(pp.k / 32);
-  const int tpr = (int)round_up(units, 32);
-  const int rpb = tpr >= 512 ? 1 : 512 / tpr;
-  const int rpb_c = rpb > 16 ? 16 : rpb;
-  dim3 block(tpr, rpb_c);
-  dim3 grid((unsigned)((pp.t_pad + rpb_c - 1) / rpb_c));
-  prep_kernel<FMT, PAT, NORM, XBF16><<<grid, block, 0, s>>>(pp, rpb_c, tpr);
+  auto kern = prep_kernel<FMT, PAT, NORM, XBF16>;
+  kern<<<row_grid(kern, pp.t_pad, pp.k), 128, 0, s>>>(pp);
   return launched();
 }
 
 template <bool NORM, bool XBF16>
 sharq_status launch_amax(const void* x, const void* gamma, float eps, int64_t t, int64_t k, float* out,
                          cudaStream_t s) {
-  const int units = (int)(k / 32);
-  const int tpr = (int)round_up(units, 32);
-  const int rpb = tpr >= 512 ? 1 : (512 / tpr > 16 ? 16 : 512 / tpr);
-  const int64_t groups = (t + rpb - 1) / rpb;
-  const int64_t cap = (int64_t)sm_count() * 4;
-  dim3 block(tpr, rpb);
-  dim3 grid((unsigned)(groups < cap ? groups : cap));
-  amax_kernel<NORM, XBF16><<<grid, block, 0, s>>>(x, gamma, eps, t, k, out, rpb, tpr);
+  auto kern = amax_kernel<NORM, XBF16>;
+  kern<<<row_grid(kern, t, k), 128, 0, s>>>(x, gamma, eps, t, k, out);
   return launched();
 }
 
@@ -214,25 +237,35 @@ sharq_status run_linear(const sharq_prepared* a, const sharq_weight* w, const in
     return fail(SHARQ_ERR_INVALID, "a stacked weight needs sharq_linear_grouped");
   if (a->fmt == SHARQ_NVFP4 && a->pat == SHARQ_NM_2_4)
     return fail(SHARQ_ERR_UNSUPPORTED, "NVFP4 with element-wise 2:4 has no sparse tensor-core kind");
-  if (a->fmt == SHARQ_MXFP4 && a->pat == SHARQ_NM_2_4)
-    return fail(SHARQ_ERR_UNSUPPORTED, "MXFP4 2:4 linear is not built yet");
 
   const int64_t t_pad = round_up(a->t, 128);
   const bool sparse = a->pat != SHARQ_NM_8_16;
+  const bool unpacked = a->fmt == SHARQ_MXFP4 && a->pat == SHARQ_NM_2_4;  // kind::mxf8f6f4
   GemmMaps maps;
   memset(&maps, 0, sizeof(maps));
-  st = make_map(&maps.w, w->codes, w->k / 2, w->n * w->experts, 128, 256, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (st != SHARQ_OK) return st;
-  st = make_map(&maps.r, a->res_codes, a->k / 2, t_pad, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (st != SHARQ_OK) return st;
-  if (sparse) {
-    st = make_map(&maps.b, a->bb_codes, a->k / 4, t_pad, 64, 128, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (unpacked) {
+    st = make_map_u4(&maps.w, w->codes, w->k, w->n * w->experts, GemmCfg<GK_MXF8, true>::BN);
+    if (st != SHARQ_OK) return st;
+    st = make_map_u4(&maps.r, a->res_codes, a->k, t_pad, 128);
+    if (st != SHARQ_OK) return st;
+    st = make_map_u4(&maps.b, a->bb_codes, a->k / 2, t_pad, 128);
     if (st != SHARQ_OK) return st;
     st = make_map(&maps.e, a->meta, meta_row_bytes(a->k, a->pat), t_pad, 16, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (st != SHARQ_OK) return st;
   } else {
-    st = make_map(&maps.b, a->bb_codes, a->k / 2, t_pad, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    st = make_map(&maps.w, w->codes, w->k / 2, w->n * w->experts, 128, 256, CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != SHARQ_OK) return st;
+    st = make_map(&maps.r, a->res_codes, a->k / 2, t_pad, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != SHARQ_OK) return st;
+    if (sparse) {
+      st = make_map(&maps.b, a->bb_codes, a->k / 4, t_pad, 64, 128, CU_TENSOR_MAP_SWIZZLE_64B);
+      if (st != SHARQ_OK) return st;
+      st = make_map(&maps.e, a->meta, meta_row_bytes(a->k, a->pat), t_pad, 16, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+      if (st != SHARQ_OK) return st;
+    } else {
+      st = make_map(&maps.b, a->bb_codes, a->k / 2, t_pad, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+      if (st != SHARQ_OK) return st;
+    }
   }
   GemmParams gp;
   gp.t = a->t;
@@ -253,6 +286,7 @@ sharq_status run_linear(const sharq_prepared* a, const sharq_weight* w, const in
   gp.timeout_ns = wait_timeout_ns();
   if (a->fmt == SHARQ_NVFP4)
     return sparse ? launch_gemm<GK_NVF4, true>(maps, gp, s) : launch_gemm<GK_NVF4, false>(maps, gp, s);
+  if (unpacked) return launch_gemm<GK_MXF8, true>(maps, gp, s);
   return sparse ? launch_gemm<GK_MXF4, true>(maps, gp, s) : launch_gemm<GK_MXF4, false>(maps, gp, s);
 }
 

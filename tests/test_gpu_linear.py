@@ -12,7 +12,7 @@ from gpu_common import assert_close_gemm, gpu_prepare, readback, assert_prep_equ
 
 pytestmark = pytest.mark.gpu
 
-LINEAR_CASES = [("nvfp4", "4:8pair"), ("nvfp4", "8:16"), ("mxfp4", "4:8pair"), ("mxfp4", "8:16")]
+LINEAR_CASES = [("nvfp4", "4:8pair"), ("nvfp4", "8:16"), ("mxfp4", "4:8pair"), ("mxfp4", "8:16"), ("mxfp4", "2:4")]
 
 
 def _w(seed, n, k, scale=0.02):
@@ -120,11 +120,80 @@ def test_linear_bf16_output_and_single_row(cuda_ok):
         assert err < 4e-3
 
 
-def test_linear_tiny_config_mxfp4_4_8_pair(cuda_ok):
+@pytest.mark.parametrize("pat", ["2:4", "4:8pair"])
+def test_linear_tiny_config(cuda_ok, pat):
+    """The Tiny case (16 x 256 fp32, channels 3 and 77 x40, MXFP4); 2:4 is the
+    configuration as specified, 4:8 pair exercises the other sparse kind."""
     cfg = workloads.tiny()
-    _, _, y = _run_linear(cfg["x"], cfg["w"], "mxfp4", "4:8pair", x_dtype="f32", w_dtype="f32")
-    prep, wq = _ref(cfg["x"], cfg["w"], "mxfp4", "4:8pair")
-    assert_close_gemm(y, oracle.linear_ref(prep, wq), "tiny 4:8pair")
+    _, _, y = _run_linear(cfg["x"], cfg["w"], "mxfp4", pat, x_dtype="f32", w_dtype="f32")
+    prep, wq = _ref(cfg["x"], cfg["w"], "mxfp4", pat)
+    assert_close_gemm(y, oracle.linear_ref(prep, wq), f"tiny {pat}")
+
+
+def test_nvfp4_2_4_linear_is_unsupported(cuda_ok):
+    p = gpu_prepare(_x(9, 16, 256), "bf16", "nvfp4", "2:4")
+    wq = gpu_weight(_w(9, 256, 256), "bf16", "nvfp4")
+    with pytest.raises(sharq.SharqError) as ei:
+        sharq.linear(p, wq)
+    assert ei.value.status == 2
+
+
+@pytest.mark.parametrize("t", [1, 16, 64, 256])
+def test_linear_down_proj_token_sweep(cuda_ok, t):
+    """Llama-3.1-8B down_proj (14336 -> 4096), MXFP4 2:4, decode-size token counts."""
+    cfg = workloads.down_proj(t=t)
+    _, _, y = _run_linear(cfg["x"], cfg["w"], "mxfp4", "2:4")
+    prep, wq = _ref(cfg["x"], cfg["w"], "mxfp4", "2:4")
+    assert_close_gemm(y, oracle.linear_ref(prep, wq), f"down_proj t={t}")
+
+
+def test_linear_down_proj_2048_sampled_rows(cuda_ok):
+    cfg = workloads.down_proj()
+    _, _, y = _run_linear(cfg["x"], cfg["w"], "mxfp4", "2:4", out_dtype=torch.float32)
+    rows = np.sort(np.random.default_rng(11).choice(2048, 48, replace=False))
+    prep = oracle.prepare(cfg["x"][rows], "mxfp4", "2:4")
+    wq = oracle.quantize_weight(cfg["w"], "mxfp4")
+    assert_close_gemm(y[rows], oracle.linear_ref(prep, wq), "down_proj sampled rows")
+
+
+@pytest.mark.parametrize("pat", ["4:8pair", "8:16"])
+def test_linear_wan_full_size_sampled_rows(cuda_ok, pat):
+    """Wan2.2 DiT linear (32768 x 5120 -> 5120), NVFP4 with RMSNorm, 4:8 pair and 8:16."""
+    cfg = workloads.wan(pat=pat)
+    p, _, y = _run_linear(cfg["x"], cfg["w"], "nvfp4", pat, gamma=cfg["gamma"], out_dtype=torch.float32)
+    rows = np.sort(np.random.default_rng(12).choice(32768, 24, replace=False))
+    amax = float(p.tensor[0].item())
+    prep = oracle.prepare(cfg["x"][rows], "nvfp4", pat, gamma=cfg["gamma"], act_amax=amax)
+    wq = oracle.quantize_weight(cfg["w"], "nvfp4")
+    assert_close_gemm(y[rows], oracle.linear_ref(prep, wq), f"wan {pat} sampled rows")
+
+
+@pytest.mark.parametrize("which", ["gate_up", "down"])
+def test_linear_grouped_qwen_moe(cuda_ok, which):
+    """Qwen3-30B-A3B experts: 128 stacked NVFP4 weights, routed rows grouped by
+    expert (segments padded to 128 rows), one grouped launch; rows sampled from
+    several experts against the oracle with each row's own expert weight."""
+    cfg = workloads.qwen_moe()
+    x = cfg["x"] if which == "gate_up" else cfg["x_down"]
+    w = cfg["w_gu"] if which == "gate_up" else cfg["w_d"]
+    offsets = cfg["offsets"]
+    p = gpu_prepare(x, "bf16", "nvfp4", "4:8pair")
+    wq = sharq.FP4Weight.quantize(to_dev(w, "bf16"), "nvfp4")
+    off_dev = torch.from_numpy(offsets.astype(np.int32)).cuda()
+    y = sharq.linear_grouped(p, wq, off_dev, out_dtype=torch.float32)
+    sharq.sharq_sync_status()
+    y = y.cpu().numpy()
+    amax = float(p.tensor[0].item())
+    rng = np.random.default_rng(13)
+    experts = [0, 5, 64, 127] + list(rng.choice(128, 4, replace=False))
+    for e in experts:
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        if hi == lo:
+            continue
+        rows = np.unique(np.concatenate([[lo, hi - 1], rng.integers(lo, hi, 6)]))
+        prep = oracle.prepare(x[rows], "nvfp4", "4:8pair", act_amax=amax)
+        wqe = oracle.quantize_weight(w[e], "nvfp4")
+        assert_close_gemm(y[rows], oracle.linear_ref(prep, wqe), f"moe {which} expert {e}")
 
 
 def test_linear_q_proj_full_size_sampled_rows(cuda_ok):
