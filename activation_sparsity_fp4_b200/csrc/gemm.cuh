@@ -2,8 +2,8 @@
 //
 // SharQ (arXiv 2606.26587), abstract and Section 1: a sparse FP4 GEMM runs over
 // the compressed backbone and its N:M metadata, a dense FP4 GEMM runs over the
-// residual and "accumulates directly into the sparse output", and "both paths
-// share one FP4 weight load with path-specific scale views".  Here both MMAs of
+// residual and adds its result into the same output, and the two paths load
+// the FP4 weight once, each reading it through its own scale view.  Here both MMAs of
 // a K tile read the SAME shared-memory copy of the weight tile (one TMA load)
 // and write the SAME tensor-memory accumulator; each path brings its own
 // scale-factor view of the weight (one scale per 2b logical K for the sparse

@@ -3,8 +3,8 @@
 // SharQ (arXiv 2606.26587) abstract / Section 1: per activation row, an online
 // N:M mask extracts an outlier-dominated sparse backbone that is quantized to
 // FP4; the dense residual is taken against the QUANTIZED backbone and quantized
-// to FP4 as well; "a fused preprocessing kernel absorbs mask generation,
-// residual construction and layer normalization into one operator".
+// to FP4 as well; mask selection, residual construction and the layer norm
+// are done by one fused preprocessing operator.
 //
 // Work split: a thread owns 32 consecutive K elements (one "unit": 4 x
 // 16-byte loads of bf16, 8 of fp32); a power-of-two number of threads (8..128)

@@ -60,15 +60,16 @@ typedef enum {
  *   NVFP4 -- E2M1 elements, one E4M3 scale per 16 elements, fp32 tensor scale. */
 typedef enum { SHARQ_MXFP4 = 0, SHARQ_NVFP4 = 1 } sharq_format;
 
-/* Online N:M activation masks: 2:4 (Huawei problem 137-2, "MXFP4/HiF4 with 2:4
- * sparsity"), the NVFP4 4:8 pair pattern (SharQ Section 2.2: two of four
- * adjacent pairs kept), and 8:16 ("From 2:4 to 8:16 sparsity patterns", abstract). */
+/* Online N:M activation masks: 2:4 (Huawei problem 137-2 asks for MXFP4/HiF4
+ * combined with 2:4), the NVFP4 4:8 pair pattern (SharQ Section 2.2: two of four
+ * adjacent pairs kept), and 8:16 (paper on 2:4-to-8:16 sparsity patterns, abstract). */
 typedef enum { SHARQ_NM_2_4 = 0, SHARQ_NM_4_8_PAIR = 1, SHARQ_NM_8_16 = 2 } sharq_pattern;
 
 typedef enum { SHARQ_F32 = 0, SHARQ_BF16 = 1 } sharq_dtype;
 
 /* The FP4 weight shared by the sparse and the dense GEMM (SharQ abstract:
- * "both paths share one FP4 weight load, with path-specific scale views").
+ * the two GEMM paths load the FP4 weight once and each reads it through its
+ * own view of the scales).
  * The sparse tensor-core MMA applies one scale per b stored (2b logical) K
  * elements, so the weight is quantized in K blocks of 2b (b = 32 MXFP4, 16
  * NVFP4) and carries two views of the same scales:
@@ -90,7 +91,7 @@ typedef struct {
 /* Prepared activations (output of sharq_prepare):
  *   meta       t_pad * meta_row bytes (meta_row = k/8 for 2:4 and 8:16, k/16 for 4:8 pair)
  *   bb_codes   backbone codes: 2:4 and 4:8 pair -- t_pad * k/4 bytes, the k/2 kept values
- *              of a row in K order ("sparse input compression", SharQ Section 1);
+ *              of a row in K order (the compressed sparse input of SharQ Section 1);
  *              8:16 -- t_pad * k/2 bytes, dense layout with code 0 at dropped positions
  *   bb_scales  tiled scale layout, t_pad rows: one scale per b kept values (k/(2b) per
  *              row); for 8:16 each is stored twice (k/b per row), the dense view
@@ -125,8 +126,8 @@ sharq_status sharq_prepared_sizes(int64_t t, int64_t k, sharq_format fmt, sharq_
  * out->codes/scales/tensor must be set by the caller; n, k, experts, fmt too. */
 sharq_status sharq_quantize_weight(const void* w, sharq_dtype w_dt, sharq_weight* out, sharq_stream stream);
 
-/* Fused preprocessing (SharQ abstract: "a fused preprocessing kernel absorbs mask
- * generation, residual construction and layer normalization into one operator"):
+/* Fused preprocessing (SharQ abstract: one fused operator does the mask, the
+ * residual and the layer norm):
  *   h = RMSNorm(x) * gamma if gamma != NULL (fp32, eps added to the mean square), else x;
  *   N:M mask = top-N |h| per group of M, ties to the lower index (4:8 pair: top 2 of 4
  *   adjacent pairs by max |.|); backbone = kept values, FP4 in blocks of b kept values;

@@ -5,8 +5,8 @@
  * this file; only tests/, the smoke check and the CPU-baseline leg of bench.py
  * use it.  It shares no code, header, table or helper with the CUDA library.
  *
- * Method: "SharQ: Bridging Activation Sparsity and FP4 Quantization for LLM
- * Inference" (Meng, Luo, Zhao et al.), abstract and Section 1:
+ * Method: SharQ, sparse-dense decomposition for FP4 inference (arXiv 2606.26587,
+ * Meng, Luo, Zhao et al.), abstract and Section 1:
  *   - an input-adaptive N:M mask is built online from the current activation;
  *   - the masked, outlier-dominated sparse backbone is quantized to FP4;
  *   - the dense residual is defined against the QUANTIZED backbone;
@@ -15,9 +15,9 @@
  *     scale views; the layer norm is absorbed into the preprocessing op.
  * The 4:8 "pair" pattern of NVFP4 is named in its Section 2.2; the OCP MX
  * (MXFP4) format in Section 2.3.  The 8:16 pattern and its metadata cost come
- * from "From 2:4 to 8:16 sparsity patterns in LLMs for Outliers and Weights with
- * Variance Correction" (abstract).  Top-k selection per group comes from the
- * Huawei problem statement (page "华为黄大年茶思屋第137期·难题2", section 4).
+ * from the 2:4-to-8:16 sparsity-pattern paper (arXiv 2507.03052, abstract).
+ * Top-k selection per group comes from the Huawei problem statement (Tea House
+ * issue 137, problem 2, section 4).
  *
  * The pages give no equations.  Every step below is the plainest reading, with
  * fixed fp32 round-to-nearest-even operations so that a GPU implementation can
