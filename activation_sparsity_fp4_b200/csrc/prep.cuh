@@ -45,6 +45,7 @@ struct PrepParams {
   uint8_t* res_scales;
   float* tensor;     // [amax, g_enc, g_dec]
   float act_amax;    // > 0: given by the caller
+  const float* rstd; // per-row RMSNorm factors from the amax pass, or null
 };
 
 // ------------------------------------------------------------- loading
@@ -178,16 +179,16 @@ __device__ __forceinline__ float pow2f(int e) {  // exact 2^e for e in [-127, 12
 // Block scale: returns the scale code, the multiplier that maps values onto the
 // E2M1 grid (0 means "all codes +0") and the decoded scale (times g_dec for
 // the dequantized value: deq = (e2m1 * sv) * g_dec for NVFP4, e2m1 * sv for MX).
-// NVFP4: s = (amax / 6) * g_enc, S = E4M3(s), mul = g_enc / S (exact table).
+// NVFP4: s = amax * c6 with c6 = g_enc / 6, S = E4M3(s), mul = g_enc / S (exact table).
 template <int FMT>
-__device__ __forceinline__ uint32_t block_scale(float amax, float g_enc, const float* inv_tab, float& mul, float& sv) {
+__device__ __forceinline__ uint32_t block_scale(float amax, float c6, const float* inv_tab, float& mul, float& sv) {
   if constexpr (FMT == FMT_MX) {
     const int e = mx_exponent(amax);
     mul = pow2f(-e);
     sv = pow2f(e);
     return (uint32_t)(e + 127);
   } else {
-    const uint32_t sc = cvt_e4m3(__fmul_rn(__fdiv_rn(amax, 6.0f), g_enc));
+    const uint32_t sc = cvt_e4m3(__fmul_rn(amax, c6));
     sv = e4m3_value(sc);
     mul = inv_tab[sc];  // 0 for code 0
     return sc;
@@ -224,14 +225,14 @@ __device__ __forceinline__ void fill_inv_table(float* tab, float g_enc) {
 }
 
 // ------------------------------------------------------------ row mapping
-// A block of 128 threads handles kRpb = 128 / tpr rows at a time; tpr threads
-// per row (a power of two, 8..128); thread t of a row owns the units t + tpr*j.
+// A block of 128 threads handles 128 / tpr rows at a time; tpr threads per row
+// (a power of two, 8..128); thread t of a row owns the units t + tpr*j.
 // Blocks stride over row groups.
 struct RowMap {
-  int tpr;   // threads per row
-  int lg;    // log2(tpr)
-  int units; // units (32 elements) per row
-  int nj;    // units per thread, <= 4
+  int tpr;    // threads per row
+  int lg;     // log2(tpr)
+  int units;  // units (32 elements) per row
+  int nj;     // units per thread, <= 4
 };
 
 __device__ __forceinline__ RowMap row_map(int64_t k) {
@@ -302,12 +303,30 @@ __device__ __forceinline__ float rstd_from_sumsq(float sumsq, int64_t k, float e
   return __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(mean, eps)));
 }
 
-// ------------------------------------------------------------ amax kernel
-// max |h| over all rows, folded into out[0] (zeroed beforehand) with one
-// atomic per block.
+// ---------------------------------------------------------- packed fp32
+// Elementwise IEEE round-to-nearest on two fp32 lanes at once (sm_100 f32x2).
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+  return (uint64_t)__float_as_uint(lo) | ((uint64_t)__float_as_uint(hi) << 32);
+}
+__device__ __forceinline__ void mul2(float& a, float& b, float c, float d) {  // (a, b) *= (c, d)
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pk2(a, b)), "l"(pk2(c, d)));
+  a = __uint_as_float((uint32_t)r);
+  b = __uint_as_float((uint32_t)(r >> 32));
+}
+__device__ __forceinline__ void sub2(float& a, float& b, float c, float d) {  // (a, b) -= (c, d)
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pk2(a, b)), "l"(pk2(c, d)));
+  a = __uint_as_float((uint32_t)r);
+  b = __uint_as_float((uint32_t)(r >> 32));
+}
+
+// ------------------------------------------------------------ stats kernel
+// Per row: rstd (RMSNorm) into rstd_out (if non-null) and max |h| folded into
+// amax_out[0] (zeroed beforehand) with one atomic per block.
 template <bool NORM, bool XBF16>
 __global__ void __launch_bounds__(128) amax_kernel(const void* x, const void* gamma, float eps, int64_t t, int64_t k,
-                                                   float* out) {
+                                                   float* amax_out, float* rstd_out) {
   __shared__ float red[32 * 16];
   __shared__ float wmax[4];
   const RowMap m = row_map(k);
@@ -319,7 +338,10 @@ __global__ void __launch_bounds__(128) amax_kernel(const void* x, const void* ga
     const bool real = r < t;
     const int64_t off = r * k;
     float rs = 1.0f;
-    if constexpr (NORM) rs = rstd_from_sumsq(row_sumsq<XBF16>(x, off, real, m, tt, row_in_block, red), k, eps);
+    if constexpr (NORM) {
+      rs = rstd_from_sumsq(row_sumsq<XBF16>(x, off, real, m, tt, row_in_block, red), k, eps);
+      if (rstd_out && real && tt == 0) rstd_out[r] = rs;
+    }
     for (int j = 0; j < m.nj; j++) {
       const int u = tt + m.tpr * j;
       if (!real || u >= m.units) continue;
@@ -329,11 +351,13 @@ __global__ void __launch_bounds__(128) amax_kernel(const void* x, const void* ga
         float g[32];
         load_unit<XBF16>(gamma, (int64_t)u * 32, g);
 #pragma unroll
-        for (int i = 0; i < 32; i++) my = fmaxf(my, fabsf(__fmul_rn(__fmul_rn(v[i], rs), g[i])));
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; i++) my = fmaxf(my, fabsf(v[i]));
+        for (int i = 0; i < 32; i += 2) {
+          mul2(v[i], v[i + 1], rs, rs);
+          mul2(v[i], v[i + 1], g[i], g[i + 1]);
+        }
       }
+#pragma unroll
+      for (int i = 0; i < 32; i++) my = fmaxf(my, fabsf(v[i]));
     }
   }
 #pragma unroll
@@ -342,114 +366,143 @@ __global__ void __launch_bounds__(128) amax_kernel(const void* x, const void* ga
   __syncthreads();
   if (threadIdx.x == 0) {
     const float mm = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
-    atomicMax(reinterpret_cast<unsigned int*>(out), __float_as_uint(mm));
+    atomicMax(reinterpret_cast<unsigned int*>(amax_out), __float_as_uint(mm));
   }
 }
 
 // ------------------------------------------------------------ prep kernel
+// Byte mask of the kept pairs of a 4:8 group: byte p = 0xFF if pair p kept.
+__device__ __forceinline__ uint32_t pair_byte_mask(uint32_t kp) {
+  return ((kp & 1u) ? 0x000000FFu : 0u) | ((kp & 2u) ? 0x0000FF00u : 0u) | ((kp & 4u) ? 0x00FF0000u : 0u) |
+         ((kp & 8u) ? 0xFF000000u : 0u);
+}
+// Nibble mask of kept elements of a 2:4 quad pair (8 elements, two quads).
+__device__ __forceinline__ uint32_t nibble_mask8(uint32_t keep8) {
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < 8; i++) m |= ((keep8 >> i) & 1u) ? (0xFu << (4 * i)) : 0u;
+  return m;
+}
+// Compact the codes of the two kept bytes (pairs p0 < p1) of a 4-byte word.
+__device__ __forceinline__ uint32_t compact_pairs(uint32_t w, uint32_t p0, uint32_t p1) {
+  return __byte_perm(w, 0u, p0 | (p1 << 4) | 0x4400u);  // bytes p0, p1 -> positions 0, 1; zeros above
+}
+
+// Residual of 8 values against their backbone codes: h -= (e2m1(c_i) * sv) * g
+// (g = 1 for MX).  e2m1 * sv is exact (2-bit times 4-bit significands), so
+// the packed multiply is safe; the NVFP4 product with g rounds, and the
+// compiler contracts a packed multiply followed by a packed subtract into one
+// fused multiply-add even with explicit rounding, which skips that rounding:
+// that step stays on scalar __fmul_rn / __fsub_rn, which are never contracted.
+template <int FMT>
+__device__ __forceinline__ void sub_deq8(float* h, uint32_t c, float sv, float g) {
+  float d[8];
+  e2m1x8_values(c, d);
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    mul2(d[i], d[i + 1], sv, sv);
+    if constexpr (FMT == FMT_NV) {
+      h[i] = __fsub_rn(h[i], __fmul_rn(d[i], g));
+      h[i + 1] = __fsub_rn(h[i + 1], __fmul_rn(d[i + 1], g));
+    } else {
+      sub2(h[i], h[i + 1], d[i], d[i + 1]);
+    }
+  }
+}
+
 // One unit of 32 values: mask, backbone quantization, residual (in place in
-// h) and residual quantization.  Outputs: meta bits, backbone codes (k/2
-// kept codes: 2 words; 8:16 dense layout: 4 words) and scale, residual codes
-// (4 words) and scales.
+// h) and residual quantization.  Outputs: meta bits, backbone codes (k/2 kept
+// codes: 2 words; 8:16 dense layout: 4 words) and scale, residual codes (4
+// words) and scales.  The backbone is quantized in its expanded form (codes
+// of dropped positions masked to +0), so R = h - deq needs no selects.
 template <int FMT, int PAT>
-__device__ __forceinline__ void quantize_unit(float (&h)[32], float g_enc, float g_dec, const float* inv_tab,
+__device__ __forceinline__ void quantize_unit(float (&h)[32], float c6, float g_dec, const float* inv_tab,
                                               uint32_t& meta, uint32_t (&bc)[4], uint32_t& bsc, uint32_t (&rc)[4],
                                               uint32_t& rsc0, uint32_t& rsc1) {
-  // the group maximum is always kept, so the backbone block amax is the window amax
-  float bamax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 32; i++) bamax = fmaxf(bamax, fabsf(h[i]));
-  if constexpr (FMT == FMT_MX) bamax = fmaxf(bamax, __shfl_xor_sync(0xffffffffu, bamax, 1));
-  float bmul, bsv;
-  bsc = block_scale<FMT>(bamax, g_enc, inv_tab, bmul, bsv);
-  const float dsc = FMT == FMT_NV ? g_dec : 1.0f;
+  uint32_t keepw[4];  // nibble mask of kept elements, per 8 elements
   meta = 0;
-  bc[0] = bc[1] = bc[2] = bc[3] = 0;
-
+  float bamax = 0.0f;
   if constexpr (PAT == PAT_48P) {
 #pragma unroll
     for (int g = 0; g < 4; g++) {
-      float* hg = h + 8 * g;
-      const uint32_t kp = top2of4(fmaxf(fabsf(hg[0]), fabsf(hg[1])), fmaxf(fabsf(hg[2]), fabsf(hg[3])),
-                                  fmaxf(fabsf(hg[4]), fabsf(hg[5])), fmaxf(fabsf(hg[6]), fabsf(hg[7])));
-      const uint32_t nib = pair_nibble(kp);
-      meta |= nib << (4 * g);
-      const int p0 = nib & 3, p1 = nib >> 2;
-      float k4[4];
-      k4[0] = (p0 == 0) ? hg[0] : (p0 == 1) ? hg[2] : hg[4];
-      k4[1] = (p0 == 0) ? hg[1] : (p0 == 1) ? hg[3] : hg[5];
-      k4[2] = (p1 == 1) ? hg[2] : (p1 == 2) ? hg[4] : hg[6];
-      k4[3] = (p1 == 1) ? hg[3] : (p1 == 2) ? hg[5] : hg[7];
-      const uint32_t c01 = cvt_e2m1x2(__fmul_rn(k4[0], bmul), __fmul_rn(k4[1], bmul));
-      const uint32_t c23 = cvt_e2m1x2(__fmul_rn(k4[2], bmul), __fmul_rn(k4[3], bmul));
-      const uint32_t c4 = bmul == 0.0f ? 0u : (c01 | (c23 << 8));
-      bc[g >> 1] |= c4 << (16 * (g & 1));
-      float d[4];
-      e2m1x2_values(c4 & 0xFF, d[0], d[1]);
-      e2m1x2_values(c4 >> 8, d[2], d[3]);
-#pragma unroll
-      for (int i = 0; i < 4; i++) d[i] = __fmul_rn(__fmul_rn(d[i], bsv), dsc);
-#pragma unroll
-      for (int pp = 0; pp < 4; pp++)
-#pragma unroll
-        for (int jj = 0; jj < 2; jj++) {
-          float& hv = hg[2 * pp + jj];
-          hv = (pp == p0) ? __fsub_rn(hv, d[jj]) : (pp == p1) ? __fsub_rn(hv, d[2 + jj]) : hv;
-        }
+      const float* hg = h + 8 * g;
+      const float s0 = fmaxf(fabsf(hg[0]), fabsf(hg[1])), s1 = fmaxf(fabsf(hg[2]), fabsf(hg[3]));
+      const float s2 = fmaxf(fabsf(hg[4]), fabsf(hg[5])), s3 = fmaxf(fabsf(hg[6]), fabsf(hg[7]));
+      bamax = fmaxf(bamax, fmaxf(fmaxf(s0, s1), fmaxf(s2, s3)));
+      const uint32_t kp = top2of4(s0, s1, s2, s3);
+      meta |= pair_nibble(kp) << (4 * g);
+      keepw[g] = pair_byte_mask(kp);
     }
   } else if constexpr (PAT == PAT_24) {
 #pragma unroll
-    for (int q = 0; q < 8; q++) {
-      float* hq = h + 4 * q;
-      const uint32_t kg = top2of4(fabsf(hq[0]), fabsf(hq[1]), fabsf(hq[2]), fabsf(hq[3]));
-      const uint32_t nib = pair_nibble(kg);
-      meta |= nib << (4 * q);
-      const int i0 = nib & 3, i1 = nib >> 2;
-      const float k0 = (i0 == 0) ? hq[0] : (i0 == 1) ? hq[1] : hq[2];
-      const float k1 = (i1 == 1) ? hq[1] : (i1 == 2) ? hq[2] : hq[3];
-      const uint32_t c2 = bmul == 0.0f ? 0u : cvt_e2m1x2(__fmul_rn(k0, bmul), __fmul_rn(k1, bmul));
-      bc[q >> 2] |= c2 << (8 * (q & 3));
-      float d0, d1;
-      e2m1x2_values(c2, d0, d1);
-      d0 = __fmul_rn(__fmul_rn(d0, bsv), dsc);
-      d1 = __fmul_rn(__fmul_rn(d1, bsv), dsc);
+    for (int g = 0; g < 4; g++) {
+      uint32_t k8 = 0;
 #pragma unroll
-      for (int jj = 0; jj < 4; jj++) {
-        float& hv = hq[jj];
-        hv = (jj == i0) ? __fsub_rn(hv, d0) : (jj == i1) ? __fsub_rn(hv, d1) : hv;
+      for (int q = 0; q < 2; q++) {
+        const float* hq = h + 8 * g + 4 * q;
+        const float a0 = fabsf(hq[0]), a1 = fabsf(hq[1]), a2 = fabsf(hq[2]), a3 = fabsf(hq[3]);
+        bamax = fmaxf(bamax, fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)));
+        const uint32_t kg = top2of4(a0, a1, a2, a3);
+        meta |= pair_nibble(kg) << (4 * (2 * g + q));
+        k8 |= kg << (4 * q);
       }
+      keepw[g] = nibble_mask8(k8);
     }
   } else {
-    uint32_t keep = unit_mask<PAT_816>(h, meta);
-    // kept values in K order -> codes; dense layout keeps dropped positions at code 0
-    float kv[16];
+    const uint32_t keep = unit_mask<PAT_816>(h, meta);
 #pragma unroll
-    for (int i = 0; i < 32; i++) {
-      const bool kp = (keep >> i) & 1u;
-      const int slot = __popc(keep & ((1u << i) - 1u));
+    for (int i = 0; i < 32; i++) bamax = fmaxf(bamax, fabsf(h[i]));
 #pragma unroll
-      for (int s2 = 0; s2 < 16; s2++)
-        if (kp && slot == s2) kv[s2] = h[i];
+    for (int g = 0; g < 4; g++) keepw[g] = nibble_mask8((keep >> (8 * g)) & 0xFFu);
+  }
+  // the group maximum is always kept, so the backbone block amax is the window amax
+  if constexpr (FMT == FMT_MX) bamax = fmaxf(bamax, __shfl_xor_sync(0xffffffffu, bamax, 1));
+  float bmul, bsv;
+  bsc = block_scale<FMT>(bamax, c6, inv_tab, bmul, bsv);
+
+  // backbone codes in expanded form; dropped positions -> +0
+  uint32_t cw[4];
+#pragma unroll
+  for (int g = 0; g < 4; g++) {
+    float q[8];
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      q[i] = h[8 * g + i];
+      q[i + 1] = h[8 * g + i + 1];
+      mul2(q[i], q[i + 1], bmul, bmul);
     }
-    const uint32_t cw0 = quant8(kv, bmul), cw1 = quant8(kv + 8, bmul);
-    float bdeq[16];
-    e2m1x8_values(cw0, bdeq);
-    e2m1x8_values(cw1, bdeq + 8);
+    cw[g] = (bmul == 0.0f ? 0u : cvt_e2m1x8(q)) & keepw[g];
+  }
+  // residual R = h - deq(backbone) (deq = +0 where dropped: R = h exactly)
 #pragma unroll
-    for (int i = 0; i < 16; i++) bdeq[i] = __fmul_rn(__fmul_rn(bdeq[i], bsv), dsc);
-    const uint32_t cw[2] = {cw0, cw1};
+  for (int g = 0; g < 4; g++) sub_deq8<FMT>(h + 8 * g, cw[g], bsv, g_dec);
+  // compaction of the kept codes (K order) for storage
+  if constexpr (PAT == PAT_48P) {
+    uint32_t half[4];
 #pragma unroll
-    for (int i = 0; i < 32; i++) {
-      const bool kp = (keep >> i) & 1u;
-      const int slot = __popc(keep & ((1u << i) - 1u));
-      float d = 0.0f;
-#pragma unroll
-      for (int s2 = 0; s2 < 16; s2++)
-        if (slot == s2) d = bdeq[s2];
-      h[i] = kp ? __fsub_rn(h[i], d) : h[i];
-      const uint32_t c = (cw[slot >> 3] >> (4 * (slot & 7))) & 15u;
-      bc[i >> 3] |= (kp ? c : 0u) << (4 * (i & 7));
+    for (int g = 0; g < 4; g++) {
+      const uint32_t nib = (meta >> (4 * g)) & 15u;
+      half[g] = compact_pairs(cw[g], nib & 3u, nib >> 2);
     }
+    bc[0] = half[0] | (half[1] << 16);
+    bc[1] = half[2] | (half[3] << 16);
+    bc[2] = bc[3] = 0;
+  } else if constexpr (PAT == PAT_24) {
+    // per quad: two kept nibbles i0 < i1 -> one byte
+    uint32_t byte8[8];
+#pragma unroll
+    for (int q = 0; q < 8; q++) {
+      const uint32_t nib = (meta >> (4 * q)) & 15u;
+      const uint32_t quad = (cw[q >> 1] >> (16 * (q & 1))) & 0xFFFFu;
+      const uint32_t c0 = (quad >> (4 * (nib & 3u))) & 15u, c1 = (quad >> (4 * (nib >> 2))) & 15u;
+      byte8[q] = c0 | (c1 << 4);
+    }
+    bc[0] = byte8[0] | (byte8[1] << 8) | (byte8[2] << 16) | (byte8[3] << 24);
+    bc[1] = byte8[4] | (byte8[5] << 8) | (byte8[6] << 16) | (byte8[7] << 24);
+    bc[2] = bc[3] = 0;
+  } else {
+#pragma unroll
+    for (int g = 0; g < 4; g++) bc[g] = cw[g];
   }
 
   // residual quantization
@@ -460,21 +513,38 @@ __device__ __forceinline__ void quantize_unit(float (&h)[32], float g_enc, float
 #pragma unroll
     for (int i = 16; i < 32; i++) a1 = fmaxf(a1, fabsf(h[i]));
     float m0, m1, sv0, sv1;
-    rsc0 = block_scale<FMT>(a0, g_enc, inv_tab, m0, sv0);
-    rsc1 = block_scale<FMT>(a1, g_enc, inv_tab, m1, sv1);
-    rc[0] = quant8(h, m0);
-    rc[1] = quant8(h + 8, m0);
-    rc[2] = quant8(h + 16, m1);
-    rc[3] = quant8(h + 24, m1);
+    rsc0 = block_scale<FMT>(a0, c6, inv_tab, m0, sv0);
+    rsc1 = block_scale<FMT>(a1, c6, inv_tab, m1, sv1);
+#pragma unroll
+    for (int w = 0; w < 4; w++) {
+      const float mm = w < 2 ? m0 : m1;
+      float q[8];
+#pragma unroll
+      for (int i = 0; i < 8; i += 2) {
+        q[i] = h[8 * w + i];
+        q[i + 1] = h[8 * w + i + 1];
+        mul2(q[i], q[i + 1], mm, mm);
+      }
+      rc[w] = mm == 0.0f ? 0u : cvt_e2m1x8(q);
+    }
   } else {
     float a0 = 0.0f;
 #pragma unroll
     for (int i = 0; i < 32; i++) a0 = fmaxf(a0, fabsf(h[i]));
     float m0, sv0;
-    rsc0 = block_scale<FMT>(a0, g_enc, inv_tab, m0, sv0);
+    rsc0 = block_scale<FMT>(a0, c6, inv_tab, m0, sv0);
     rsc1 = 0;
 #pragma unroll
-    for (int w = 0; w < 4; w++) rc[w] = quant8(h + 8 * w, m0);
+    for (int w = 0; w < 4; w++) {
+      float q[8];
+#pragma unroll
+      for (int i = 0; i < 8; i += 2) {
+        q[i] = h[8 * w + i];
+        q[i + 1] = h[8 * w + i + 1];
+        mul2(q[i], q[i + 1], m0, m0);
+      }
+      rc[w] = cvt_e2m1x8(q);
+    }
   }
 }
 
@@ -487,10 +557,11 @@ __global__ void __launch_bounds__(128, 6) prep_kernel(PrepParams p) {
   const int rpb = 128 / m.tpr;
   const int row_in_block = threadIdx.x >> m.lg, tt = threadIdx.x & (m.tpr - 1);
 
-  float g_enc = 1.0f, g_dec = 1.0f;
+  float g_enc = 1.0f, g_dec = 1.0f, c6 = 1.0f;
   if constexpr (FMT == FMT_NV) {
     const float amax = p.act_amax > 0.0f ? p.act_amax : *reinterpret_cast<volatile const float*>(p.tensor);
     tensor_scales(amax, g_enc, g_dec);
+    c6 = __fdiv_rn(g_enc, 6.0f);
     fill_inv_table(inv_tab, g_enc);
     __syncthreads();
     if (blockIdx.x == 0 && threadIdx.x == 0) {
@@ -513,7 +584,10 @@ __global__ void __launch_bounds__(128, 6) prep_kernel(PrepParams p) {
     const bool real = r < p.t;
     const int64_t off = r * k;
     float rs = 1.0f;
-    if constexpr (NORM) rs = rstd_from_sumsq(row_sumsq<XBF16>(p.x, off, real, m, tt, row_in_block, red), k, p.eps);
+    if constexpr (NORM) {
+      if (p.rstd) rs = real ? __ldg(p.rstd + r) : 1.0f;  // row statistics from the amax pass
+      else rs = rstd_from_sumsq(row_sumsq<XBF16>(p.x, off, real, m, tt, row_in_block, red), k, p.eps);
+    }
 
     for (int j = 0; j < m.nj; j++) {
       const int u = tt + m.tpr * j;
@@ -525,14 +599,17 @@ __global__ void __launch_bounds__(128, 6) prep_kernel(PrepParams p) {
           float g[32];
           load_unit<XBF16>(p.gamma, (int64_t)u * 32, g);
 #pragma unroll
-          for (int i = 0; i < 32; i++) h[i] = __fmul_rn(__fmul_rn(h[i], rs), g[i]);
+          for (int i = 0; i < 32; i += 2) {
+            mul2(h[i], h[i + 1], rs, rs);
+            mul2(h[i], h[i + 1], g[i], g[i + 1]);
+          }
         }
       } else {
 #pragma unroll
         for (int i = 0; i < 32; i++) h[i] = 0.0f;
       }
       uint32_t meta, bc[4], bsc, rc[4], rsc0, rsc1;
-      quantize_unit<FMT, PAT>(h, g_enc, g_dec, inv_tab, meta, bc, bsc, rc, rsc0, rsc1);
+      quantize_unit<FMT, PAT>(h, c6, g_dec, inv_tab, meta, bc, bsc, rc, rsc0, rsc1);
       if (!active || !in_pad) continue;
 
       if constexpr (PAT == PAT_48P) {
@@ -606,7 +683,7 @@ __global__ void __launch_bounds__(256) weight_kernel(WeightParams p) {
     sc = (uint32_t)(e + 127);
     mul = pow2f(-e);
   } else {
-    sc = cvt_e4m3(__fmul_rn(__fdiv_rn(amax, 6.0f), g_enc));
+    sc = cvt_e4m3(__fmul_rn(amax, __fdiv_rn(g_enc, 6.0f)));
     const float sv = e4m3_value(sc);
     mul = sv == 0.0f ? 0.0f : __fdiv_rn(g_enc, sv);
   }

@@ -154,9 +154,9 @@ sharq_status launch_prep(const PrepParams& pp, cudaStream_t s) {
 
 template <bool NORM, bool XBF16>
 sharq_status launch_amax(const void* x, const void* gamma, float eps, int64_t t, int64_t k, float* out,
-                         cudaStream_t s) {
+                         float* rstd_out, cudaStream_t s) {
   auto kern = amax_kernel<NORM, XBF16>;
-  kern<<<row_grid(kern, t, k), 128, 0, s>>>(x, gamma, eps, t, k, out);
+  kern<<<row_grid(kern, t, k), 128, 0, s>>>(x, gamma, eps, t, k, out, rstd_out);
   return launched();
 }
 
@@ -321,7 +321,7 @@ sharq_status sharq_prepared_sizes(int64_t t, int64_t k, sharq_format fmt, sharq_
   if (bb_scales_bytes) *bb_scales_bytes = (size_t)tiled_sf_bytes(tp, pat == SHARQ_NM_8_16 ? k / b : k / (2 * b));
   if (res_codes_bytes) *res_codes_bytes = (size_t)(tp * k / 2);
   if (res_scales_bytes) *res_scales_bytes = (size_t)tiled_sf_bytes(tp, k / b);
-  if (workspace_bytes) *workspace_bytes = 0;
+  if (workspace_bytes) *workspace_bytes = (size_t)(tp * sizeof(float));  // per-row RMSNorm factors
   return SHARQ_OK;
 }
 
@@ -365,8 +365,6 @@ sharq_status sharq_quantize_weight(const void* w, sharq_dtype w_dt, sharq_weight
 
 sharq_status sharq_prepare(const void* x, sharq_dtype x_dt, const void* gamma, float eps, float act_amax,
                            sharq_prepared* out, void* workspace, size_t workspace_bytes, sharq_stream stream) {
-  (void)workspace;
-  (void)workspace_bytes;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   sharq_status st = check_prepared(out);
   if (st != SHARQ_OK) return st;
@@ -389,13 +387,19 @@ sharq_status sharq_prepare(const void* x, sharq_dtype x_dt, const void* gamma, f
   pp.res_scales = static_cast<uint8_t*>(out->res_scales);
   pp.tensor = out->tensor;
   pp.act_amax = act_amax > 0.0f ? act_amax : 0.0f;
+  pp.rstd = nullptr;
+  if (workspace && (workspace_bytes < (size_t)out->t * sizeof(float) || !aligned(workspace, 16)))
+    return fail(SHARQ_ERR_WORKSPACE, "workspace must hold t floats, 16-byte aligned");
   if (out->fmt == SHARQ_NVFP4 && !(act_amax > 0.0f)) {
+    // the amax pass already computes each row's RMSNorm factor: keep it for the prep pass
+    float* rstd = (norm && workspace) ? static_cast<float*>(workspace) : nullptr;
     SHARQ_CUDA(cudaMemsetAsync(out->tensor, 0, sizeof(float), s));
-    if (norm) st = bf16 ? launch_amax<true, true>(x, gamma, eps, out->t, out->k, out->tensor, s)
-                        : launch_amax<true, false>(x, gamma, eps, out->t, out->k, out->tensor, s);
-    else st = bf16 ? launch_amax<false, true>(x, gamma, eps, out->t, out->k, out->tensor, s)
-                   : launch_amax<false, false>(x, gamma, eps, out->t, out->k, out->tensor, s);
+    if (norm) st = bf16 ? launch_amax<true, true>(x, gamma, eps, out->t, out->k, out->tensor, rstd, s)
+                        : launch_amax<true, false>(x, gamma, eps, out->t, out->k, out->tensor, rstd, s);
+    else st = bf16 ? launch_amax<false, true>(x, gamma, eps, out->t, out->k, out->tensor, nullptr, s)
+                   : launch_amax<false, false>(x, gamma, eps, out->t, out->k, out->tensor, nullptr, s);
     if (st != SHARQ_OK) return st;
+    pp.rstd = rstd;
   }
   if (out->fmt == SHARQ_NVFP4) return prep_dispatch_p<FMT_NV>(pp, out->pat, norm, bf16, s);
   return prep_dispatch_p<FMT_MX>(pp, out->pat, norm, bf16, s);

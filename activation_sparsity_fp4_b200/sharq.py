@@ -223,15 +223,16 @@ class Prepared:
 
 
 def prepare(x: torch.Tensor, fmt, pat, gamma: torch.Tensor | None = None, eps: float = 1e-6, act_amax: float = 0.0,
-            out: Prepared | None = None, stream=None) -> Prepared:
-    """Fused preprocessing of x (t, k) on the GPU; returns (or fills) a Prepared."""
+            out: Prepared | None = None, stream=None, use_workspace: bool = True) -> Prepared:
+    """Fused preprocessing of x (t, k) on the GPU; returns (or fills) a Prepared.
+    use_workspace=False runs without the per-row scratch (same results)."""
     x = x.contiguous()
     t, k = x.shape
     if out is None:
         out = Prepared(t, k, fmt, pat, x.device)
     if gamma is not None:
         gamma = gamma.to(x.dtype).contiguous()
-    ws = out.workspace
+    ws = out.workspace if use_workspace else None
     sharq_prepare(x.data_ptr(), x.dtype, gamma.data_ptr() if gamma is not None else None, eps, act_amax, out.struct,
                   ws.data_ptr() if ws is not None else None, ws.numel() if ws is not None else 0, stream)
     return out

@@ -114,8 +114,10 @@ typedef struct {
 sharq_status sharq_weight_sizes(int64_t n, int64_t k, sharq_format fmt, size_t* codes_bytes,
                                 size_t* scales_dense_bytes, size_t* scales_sparse_bytes);
 
-/* Byte sizes of the prepared-activation buffers for t rows and of the
- * workspace sharq_prepare needs (0: it needs none). */
+/* Byte sizes of the prepared-activation buffers for t rows and of the optional
+ * workspace of sharq_prepare (t_pad floats: with RMSNorm and a device-computed
+ * NVFP4 amax, the amax pass leaves each row's RMSNorm factor there for the
+ * quantization pass, which then skips its own reduction). */
 sharq_status sharq_prepared_sizes(int64_t t, int64_t k, sharq_format fmt, sharq_pattern pat, size_t* meta_bytes,
                                   size_t* bb_codes_bytes, size_t* bb_scales_bytes, size_t* res_codes_bytes,
                                   size_t* res_scales_bytes, size_t* workspace_bytes);
@@ -135,7 +137,8 @@ sharq_status sharq_quantize_weight(const void* w, sharq_dtype w_dt, sharq_weight
  * x: t * k row-major values of dtype x_dt; gamma: k values of dtype x_dt or NULL.
  * act_amax > 0 gives the NVFP4 tensor amax; <= 0 computes max |h| on the device
  * (one extra read of x).  out->pointers, t, k, fmt, pat must be set by the caller.
- * workspace may be NULL when sharq_prepared_sizes reports 0. */
+ * workspace: NULL, or >= t floats (16-byte aligned) of scratch; results are the same
+ * either way.  Returns SHARQ_ERR_WORKSPACE for a non-NULL workspace that is too small. */
 sharq_status sharq_prepare(const void* x, sharq_dtype x_dt, const void* gamma, float eps, float act_amax,
                            sharq_prepared* out, void* workspace, size_t workspace_bytes, sharq_stream stream);
 

@@ -227,8 +227,9 @@ void orc_tensor_scale(float amax, float* g_enc, float* g_dec) {
  * Quantize n values that share one scale.  Writes n E2M1 codes, returns the
  * scale code.  MXFP4 (OCP MX rule): e = floor(log2 amax) - 2 clamped to
  * [-127, 127] (amax = 0 gives -127), code = e + 127, element = E2M1(v * 2^-e).
- * NVFP4: s = (amax / 6) * g_enc, S = E4M3(s); if S is 0 every code is +0,
- * else element = E2M1(v * (g_enc / S)).                                      */
+ * NVFP4: s = amax * c with the per-tensor constant c = g_enc / 6 (the two
+ * scalings folded into one rounding per block), S = E4M3(s); if S is 0 every
+ * code is +0, else element = E2M1(v * (g_enc / S)).                          */
 uint8_t orc_quant_block(const float* v, int n, int fmt, float g_enc, uint8_t* codes) {
   float amax = 0.0f;
   for (int i = 0; i < n; i++) amax = fmaxf(amax, fabsf(v[i]));
@@ -240,7 +241,8 @@ uint8_t orc_quant_block(const float* v, int n, int fmt, float g_enc, uint8_t* co
     for (int i = 0; i < n; i++) codes[i] = orc_e2m1_encode(v[i] * mul);
     return (uint8_t)(e + 127);
   }
-  float s32 = (amax / 6.0f) * g_enc;
+  const float c6 = g_enc / 6.0f;
+  float s32 = amax * c6;
   uint8_t sc = orc_e4m3_encode(s32);
   float sv = orc_e4m3_decode(sc);
   if (sv == 0.0f) {

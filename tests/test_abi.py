@@ -48,7 +48,7 @@ def test_prepared_sizes_pad_rows_to_128(L):
     m, bc, bs, rc, rs, ws = sharq.sharq_prepared_sizes(16, 256, "mxfp4", "2:4")
     assert (m, bc, rc) == (128 * 256 // 8, 128 * 256 // 4, 128 * 256 // 2)
     assert bs == 512 and rs == 128 * 8 // 4 * 4  # 256/64 = 4 scales; 256/32 = 8 scales per row
-    assert ws == 0
+    assert ws == 128 * 4  # one float per padded row
     m, bc, bs, rc, rs, ws = sharq.sharq_prepared_sizes(2048, 4096, "nvfp4", "4:8pair")
     assert m == 2048 * 4096 // 16 and bc == 2048 * 4096 // 4
     assert bs == 2048 * 4096 // 32 and rs == 2048 * 4096 // 16

@@ -64,6 +64,22 @@ def test_prep_single_row_and_zero_input(cuda_ok):
         assert_prep_equal(readback(gpu_prepare(z, "f32", fmt, "2:4", gamma=np.ones(512, np.float32))), ref, "2:4")
 
 
+@pytest.mark.parametrize("fmt", FMTS)
+def test_prep_workspace_gives_same_result(cuda_ok, fmt):
+    """With RMSNorm and a device amax the amax pass leaves each row's factor in
+    the workspace for the quantization pass; without it prep recomputes it."""
+    x = _x(8, 300, 2048)
+    gamma = workloads.to_bf16_values(np.random.default_rng(9).uniform(0.5, 1.5, 2048).astype(np.float32))
+    ref = oracle.prepare(x, fmt, "4:8pair", gamma=gamma)
+    from gpu_common import to_dev
+    xd, gd = to_dev(x, "bf16"), to_dev(gamma, "bf16")
+    a = sharq.prepare(xd, fmt, "4:8pair", gd, 1e-6, use_workspace=True)
+    b = sharq.prepare(xd, fmt, "4:8pair", gd, 1e-6, use_workspace=False)
+    sharq.sharq_sync_status()
+    assert_prep_equal(readback(a), ref, "4:8pair")
+    assert_prep_equal(readback(b), ref, "4:8pair")
+
+
 def test_prep_caller_amax(cuda_ok):
     x = _x(5, 130, 1024)
     amax = float(np.max(np.abs(x))) * 1.5
