@@ -292,6 +292,42 @@ sharq_status run_linear(const sharq_prepared* a, const sharq_weight* w, const in
 
 }  // namespace
 
+// Scratch of sharq_prepare_noalloc: one float (a row's RMSNorm factor) per row
+// for at most SHARQ_NOALLOC_MAX_ROWS rows, 256 KiB per device.  It is part of
+// the module image, so the driver places it when the module loads and no call
+// allocates it.  No entry of it has to start at zero: the amax pass writes the
+// factor of every row 0..t-1 before the quantization pass reads it, and rows
+// from t up are never read.
+static __device__ __align__(256) float g_noalloc_rstd[SHARQ_NOALLOC_MAX_ROWS];
+
+namespace {
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+float* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of the current device's copy of g_noalloc_rstd, looked up
+// once per device (with that device current) and cached.  The first lookup
+// may load the module on that device, which is why the first call on a device
+// has to come before any stream capture.
+sharq_status noalloc_scratch(float** out) {
+  int dev = -1;
+  SHARQ_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kNoAllocMaxDevices)
+    return fail(SHARQ_ERR_INVALID, "device %d is beyond the %d devices the static scratch tracks", dev,
+                kNoAllocMaxDevices);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    SHARQ_CUDA(cudaGetSymbolAddress(&p, g_noalloc_rstd));
+    g_noalloc_ptr[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return SHARQ_OK;
+}
+
+}  // namespace
+
 // =================================================================== C ABI
 extern "C" {
 
@@ -403,6 +439,20 @@ sharq_status sharq_prepare(const void* x, sharq_dtype x_dt, const void* gamma, f
   }
   if (out->fmt == SHARQ_NVFP4) return prep_dispatch_p<FMT_NV>(pp, out->pat, norm, bf16, s);
   return prep_dispatch_p<FMT_MX>(pp, out->pat, norm, bf16, s);
+}
+
+sharq_status sharq_prepare_noalloc(const void* x, sharq_dtype x_dt, const void* gamma, float eps, float act_amax,
+                                   sharq_prepared* out, sharq_stream stream) {
+  if (!out) return fail(SHARQ_ERR_INVALID, "out is NULL");
+  if (out->t > SHARQ_NOALLOC_MAX_ROWS)
+    return fail(SHARQ_ERR_WORKSPACE,
+                "sharq_prepare_noalloc: t = %lld rows exceeds its static scratch of %d rows; "
+                "call sharq_prepare with a caller workspace instead",
+                (long long)out->t, SHARQ_NOALLOC_MAX_ROWS);
+  float* scratch = nullptr;
+  sharq_status st = noalloc_scratch(&scratch);
+  if (st != SHARQ_OK) return st;
+  return sharq_prepare(x, x_dt, gamma, eps, act_amax, out, scratch, sizeof(float) * SHARQ_NOALLOC_MAX_ROWS, stream);
 }
 
 sharq_status sharq_linear(const sharq_prepared* a, const sharq_weight* w, void* y, sharq_dtype y_dt,

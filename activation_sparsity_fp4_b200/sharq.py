@@ -24,7 +24,8 @@ STATUS = {0: "SHARQ_OK", 1: "SHARQ_ERR_INVALID", 2: "SHARQ_ERR_UNSUPPORTED", 3: 
           4: "SHARQ_ERR_TIMEOUT", 5: "SHARQ_ERR_WORKSPACE"}
 SYMBOLS = ["sharq_weight_sizes", "sharq_prepared_sizes", "sharq_quantize_weight", "sharq_prepare", "sharq_linear",
            "sharq_linear_paths", "sharq_linear_grouped", "sharq_sync_status", "sharq_selftest_wait_timeout",
-           "sharq_last_error", "sharq_launch_count"]
+           "sharq_last_error", "sharq_launch_count", "sharq_prepare_noalloc"]
+NOALLOC_MAX_ROWS = 65536  # SHARQ_NOALLOC_MAX_ROWS of the C header
 
 
 class SharqError(RuntimeError):
@@ -68,6 +69,7 @@ def lib() -> ctypes.CDLL:
             "sharq_prepared_sizes": [I64, I64, I, I, SZ, SZ, SZ, SZ, SZ, SZ],
             "sharq_quantize_weight": [P, I, ctypes.POINTER(sharq_weight), P],
             "sharq_prepare": [P, I, P, F, F, ctypes.POINTER(sharq_prepared), P, ctypes.c_size_t, P],
+            "sharq_prepare_noalloc": [P, I, P, F, F, ctypes.POINTER(sharq_prepared), P],
             "sharq_linear": [ctypes.POINTER(sharq_prepared), ctypes.POINTER(sharq_weight), P, I, P],
             "sharq_linear_paths": [ctypes.POINTER(sharq_prepared), ctypes.POINTER(sharq_weight), P, I, I32, P],
             "sharq_linear_grouped": [ctypes.POINTER(sharq_prepared), ctypes.POINTER(sharq_weight), P, P, I, P],
@@ -140,6 +142,16 @@ def sharq_prepare(x_ptr: int, x_dt, gamma_ptr, eps: float, act_amax: float, out:
                                float(eps), float(act_amax), ctypes.byref(out),
                                ctypes.c_void_p(workspace_ptr) if workspace_ptr else None, workspace_bytes,
                                _stream(stream)), "sharq_prepare")
+
+
+def sharq_prepare_noalloc(x_ptr: int, x_dt, gamma_ptr, eps: float, act_amax: float, out: sharq_prepared,
+                          stream=None):
+    """sharq_prepare with the library's static per-row scratch: nothing is
+    allocated, t <= NOALLOC_MAX_ROWS, first call per device before any stream
+    capture, overlapping calls on one device race."""
+    _check(lib().sharq_prepare_noalloc(ctypes.c_void_p(x_ptr), _dt(x_dt),
+                                       ctypes.c_void_p(gamma_ptr) if gamma_ptr else None, float(eps), float(act_amax),
+                                       ctypes.byref(out), _stream(stream)), "sharq_prepare_noalloc")
 
 
 def sharq_linear(a: sharq_prepared, w: sharq_weight, y_ptr: int, y_dt, stream=None):

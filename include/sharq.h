@@ -13,7 +13,8 @@
  *  - All tensor arguments are DEVICE pointers on the current CUDA device,
  *    owned and allocated by the caller with the sizes the *_sizes queries
  *    return.  The library allocates no device memory and keeps no device
- *    state besides one error word per device.
+ *    state besides one error word per device and the static scratch of
+ *    sharq_prepare_noalloc.
  *  - Calls are asynchronous on the given stream.  Argument errors are found
  *    on the host and returned before anything is launched.  A device-side
  *    wait that runs out of time sets the error word; sharq_sync_status()
@@ -141,6 +142,35 @@ sharq_status sharq_quantize_weight(const void* w, sharq_dtype w_dt, sharq_weight
  * either way.  Returns SHARQ_ERR_WORKSPACE for a non-NULL workspace that is too small. */
 sharq_status sharq_prepare(const void* x, sharq_dtype x_dt, const void* gamma, float eps, float act_amax,
                            sharq_prepared* out, void* workspace, size_t workspace_bytes, sharq_stream stream);
+
+/* Largest t that sharq_prepare_noalloc accepts (its static scratch holds one float per row). */
+#define SHARQ_NOALLOC_MAX_ROWS 65536
+
+/* sharq_prepare without a caller workspace and without any allocation: the
+ * per-row scratch (each row's RMSNorm factor, which the NVFP4 amax pass hands
+ * to the quantization pass) is a static device array inside this library,
+ * SHARQ_NOALLOC_MAX_ROWS floats (256 KiB) per device.  Arguments, outputs and
+ * results are those of sharq_prepare with a workspace; the SharQ pages have no
+ * counterpart of this call, which exists for callers that cannot allocate:
+ *   - a host whose device memory is sized once at start-up and may not grow
+ *     (a fixed pool, no allocator reachable from the calling code);
+ *   - a plug-in or kernel interface with a fixed signature that has no room for a
+ *     workspace pointer.
+ * Such callers would otherwise lose the shortcut, and their NVFP4 + RMSNorm prepare
+ * would recompute every row's statistics in the quantization pass.
+ * Limits and rules:
+ *   - t > SHARQ_NOALLOC_MAX_ROWS returns SHARQ_ERR_WORKSPACE before anything runs;
+ *     use sharq_prepare with a workspace for larger t.
+ *   - The first call on a device looks up the scratch's address with that device
+ *     current (this may load the library's module there); make it before any
+ *     stream capture.  Later calls do no set-up.
+ *   - Nothing in the scratch needs to start at zero (every row read was written by
+ *     the same call); the amax accumulator, out->tensor[0], is zeroed on the stream
+ *     as in sharq_prepare.
+ *   - One scratch per device: calls that overlap on one device (several streams or
+ *     host threads) race on it.  Keep them in one stream order. */
+sharq_status sharq_prepare_noalloc(const void* x, sharq_dtype x_dt, const void* gamma, float eps, float act_amax,
+                                   sharq_prepared* out, sharq_stream stream);
 
 /* The two GEMMs of the layer (SharQ abstract, Section 1): a sparse FP4 GEMM over
  * the compressed backbone and its metadata, and a dense FP4 GEMM over R that

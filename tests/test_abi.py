@@ -93,3 +93,15 @@ def test_product_path_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(sharq, "_lib", None)
     with pytest.raises(RuntimeError, match="no CPU fallback"):
         sharq.lib()
+
+
+def test_noalloc_limit_matches_header_and_rejects_on_host(L):
+    text = open(HEADER).read()
+    m = re.search(r"#define\s+SHARQ_NOALLOC_MAX_ROWS\s+(\d+)", text)
+    assert m and int(m.group(1)) == sharq.NOALLOC_MAX_ROWS
+    before = sharq.sharq_launch_count()
+    a = sharq.sharq_prepared(16, 16, 16, 16, 16, 16, sharq.NOALLOC_MAX_ROWS + 1, 256, 1, 1)
+    with pytest.raises(sharq.SharqError) as ei:
+        sharq.sharq_prepare_noalloc(16, sharq.BF16, None, 1e-6, 0.0, a, 0)
+    assert ei.value.status == 5 and "static scratch" in str(ei.value)
+    assert sharq.sharq_launch_count() == before
