@@ -109,6 +109,31 @@ __device__ __forceinline__ uint32_t top2of4(float a0, float a1, float a2, float 
   const int n3 = b03 + b13 + b23;
   return (uint32_t)(n0 < 2) | ((uint32_t)(n1 < 2) << 1) | ((uint32_t)(n2 < 2) << 2) | ((uint32_t)(n3 < 2) << 3);
 }
+// 0xFFFFFFFF if a >= b, else 0: a comparison whose result can be combined bitwise.
+__device__ __forceinline__ uint32_t ge_mask(float a, float b) {
+  uint32_t r;
+  asm("set.ge.u32.f32 %0, %1, %2;" : "=r"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t maj3(uint32_t a, uint32_t b, uint32_t c) { return (a & b) | (c & (a | b)); }
+// The same top-2-of-4 rule as four masks (0 or ~0), from bitwise majorities of
+// the comparison masks: entry p wins against q < p when s_p > s_q and against
+// q > p when s_p >= s_q, and is kept iff it wins at least two of its three
+// comparisons (used where byte masks are wanted, the 4:8 pair pattern).
+__device__ __forceinline__ void top2of4_masks(float s0, float s1, float s2, float s3, uint32_t (&k)[4]) {
+  const uint32_t b01 = ge_mask(s0, s1), b02 = ge_mask(s0, s2), b03 = ge_mask(s0, s3);
+  const uint32_t b12 = ge_mask(s1, s2), b13 = ge_mask(s1, s3), b23 = ge_mask(s2, s3);
+  k[0] = maj3(b01, b02, b03);
+  k[1] = maj3(~b01, b12, b13);
+  k[2] = maj3(~b02, ~b12, b23);
+  k[3] = maj3(~b03, ~b13, ~b23);
+}
+// Metadata nibble i0 | i1 << 2 (kept indices i0 < i1) of two-of-four keep masks.
+__device__ __forceinline__ uint32_t kept_nibble(const uint32_t (&k)[4]) {
+  const uint32_t i0 = (~k[0] & 1u) + (~k[0] & ~k[1] & 1u);
+  const uint32_t i1 = 1u + ((k[2] | k[3]) & 1u) + (k[3] & 1u);
+  return i0 | (i1 << 2);
+}
 // metadata nibble (i0 | i1 << 2) of a 4-bit mask with exactly two bits set
 __device__ __forceinline__ uint32_t pair_nibble(uint32_t kp) {
   // kp: 0b0011 -> 4, 0b0101 -> 8, 0b0110 -> 9, 0b1001 -> 12, 0b1010 -> 13, 0b1100 -> 14
@@ -429,9 +454,10 @@ __device__ __forceinline__ void quantize_unit(float (&h)[32], float c6, float g_
       const float s0 = fmaxf(fabsf(hg[0]), fabsf(hg[1])), s1 = fmaxf(fabsf(hg[2]), fabsf(hg[3]));
       const float s2 = fmaxf(fabsf(hg[4]), fabsf(hg[5])), s3 = fmaxf(fabsf(hg[6]), fabsf(hg[7]));
       bamax = fmaxf(bamax, fmaxf(fmaxf(s0, s1), fmaxf(s2, s3)));
-      const uint32_t kp = top2of4(s0, s1, s2, s3);
-      meta |= pair_nibble(kp) << (4 * g);
-      keepw[g] = pair_byte_mask(kp);
+      uint32_t kk[4];
+      top2of4_masks(s0, s1, s2, s3, kk);
+      meta |= kept_nibble(kk) << (4 * g);
+      keepw[g] = (kk[0] & 0x000000FFu) | (kk[1] & 0x0000FF00u) | (kk[2] & 0x00FF0000u) | (kk[3] & 0xFF000000u);
     }
   } else if constexpr (PAT == PAT_24) {
 #pragma unroll

@@ -243,7 +243,7 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
 // even with saturation.
 __device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
   uint32_t out;
-  asm volatile(
+  asm(
       "{\n\t.reg .b8 t;\n\t"
       "cvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\t"
       "cvt.u32.u8 %0, t;\n\t}"
@@ -254,7 +254,7 @@ __device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
 // Eight fp32 -> eight E2M1 codes packed in 32 bits (element i in nibble i).
 __device__ __forceinline__ uint32_t cvt_e2m1x8(const float* v) {
   uint32_t out;
-  asm volatile(
+  asm(
       "{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
       "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
       "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
@@ -274,14 +274,14 @@ __device__ __forceinline__ float e2m1_value(uint32_t code) {
 // fp32 -> E4M3 code (round to nearest even, saturate to 448).
 __device__ __forceinline__ uint32_t cvt_e4m3(float v) {
   uint16_t out;
-  asm volatile("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(0.0f), "f"(v));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(0.0f), "f"(v));
   return out & 0xFF;
 }
 // Value of an E4M3 code (exact; codes here are never NaN).
 __device__ __forceinline__ float e4m3_value(uint32_t code) {
   uint32_t h2;
   uint16_t in = (uint16_t)(code & 0xFF);
-  asm volatile("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
   return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFF)));
 }
 
