@@ -83,15 +83,15 @@ struct GemmCfg {
   // transaction bytes: unpacking loads count the packed (global) size, half their smem footprint
   static constexpr uint32_t kTx = (kWBytes + kRBytes + kBBytes) / (kUnpacked ? 2 : 1) + kEBytes + kSfaR + kSfbD + kSfaB +
                                   kSfbS;
-  // tensor memory columns: accumulator, then two slots of scales + metadata
+  // tensor memory columns: accumulator, then one slot of scales + metadata per stage
   static constexpr int cSfaR = 0;
   static constexpr int cSfbD = cSfaR + 4 * kChunksR;
   static constexpr int cSfaB = cSfbD + 4 * kNRB * kChunksR;
   static constexpr int cSfbS = cSfaB + 4 * kChunksB;
   static constexpr int cE = cSfbS + (SPARSE ? 4 * kNRB * kChunksB : 0);
   static constexpr int kSlotCols = cE + 4 * kEBoxes;
-  static constexpr int kTmemCols = BN + 2 * kSlotCols <= 256 ? 256 : 512;
-  static_assert(BN + 2 * kSlotCols <= kTmemCols, "tensor memory budget");
+  static constexpr int kTmemCols = BN + kStages * kSlotCols <= 256 ? 256 : 512;
+  static_assert(BN + kStages * kSlotCols <= kTmemCols, "tensor memory budget");
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   // instruction descriptor (block-scaled kinds): E2M1 x E2M1, K-major, M=128, N=BN
@@ -137,7 +137,8 @@ __global__ void __launch_bounds__(192, 1) gemm_kernel(const __grid_constant__ Ge
   uint64_t* acc_full = empty + C::kStages;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain = acc_empty + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* sf_ready = drain + 1;  // per stage: its scale slot is in tensor memory
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sf_ready + C::kStages);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -147,6 +148,7 @@ __global__ void __launch_bounds__(192, 1) gemm_kernel(const __grid_constant__ Ge
     for (int s = 0; s < C::kStages; s++) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&sf_ready[s], 4);
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 4);
@@ -269,7 +271,7 @@ __global__ void __launch_bounds__(192, 1) gemm_kernel(const __grid_constant__ Ge
       int it = 0;
       const uint32_t acc = tmem_base;
       // descriptor halves: start addresses in 16-byte units (stage 0), constant high words
-      constexpr uint32_t kHi128 = desc_hi(1024, 2), kHi64 = desc_hi(512, 4), kHiCp = desc_hi(128, 0);
+      constexpr uint32_t kHi128 = desc_hi(1024, 2), kHi64 = desc_hi(512, 4);
       constexpr uint32_t kHiB = (SPARSE && !C::kUnpacked) ? kHi64 : kHi128;  // backbone rows of 64 or 128 bytes
       constexpr uint32_t kLbo = 1u << 16;  // 16-byte leading offset (ignored by swizzled K-major layouts)
       const uint32_t lo0 = smem_u32(smem) >> 4;
@@ -284,30 +286,10 @@ __global__ void __launch_bounds__(192, 1) gemm_kernel(const __grid_constant__ Ge
           if (!mbar_wait(&full[stage], phase, p.timeout_ns, abort_flag)) { *abort_flag = 1; break; }
           tc_fence_after();
           const uint32_t ls = lo0 + (uint32_t)(stage * (C::kStageBytes >> 4));  // stage base, 16-byte units
-          const uint32_t slot = tmem_base + C::BN + (uint32_t)((kt & 1) * C::kSlotCols);
-          // scale factors and metadata -> tensor memory
-#pragma unroll
-          for (int c = 0; c < C::kChunksR; c++) {
-            tc_cp_32x128b_warpx4(slot + C::cSfaR + 4 * c, desc_lohi(ls + (C::oSfaR >> 4) + 32 * c, kHiCp));
-#pragma unroll
-            for (int rb = 0; rb < C::kNRB; rb++)
-              tc_cp_32x128b_warpx4(slot + C::cSfbD + 4 * C::kNRB * c + 4 * rb,
-                                   desc_lohi(ls + ((C::oSfbD + rb * C::kChunksR * 512) >> 4) + 32 * c, kHiCp));
-          }
-#pragma unroll
-          for (int c = 0; c < C::kChunksB; c++) {
-            tc_cp_32x128b_warpx4(slot + C::cSfaB + 4 * c, desc_lohi(ls + (C::oSfaB >> 4) + 32 * c, kHiCp));
-            if constexpr (SPARSE) {
-#pragma unroll
-              for (int rb = 0; rb < C::kNRB; rb++)
-                tc_cp_32x128b_warpx4(slot + C::cSfbS + 4 * C::kNRB * c + 4 * rb,
-                                     desc_lohi(ls + ((C::oSfbS + rb * C::kChunksB * 512) >> 4) + 32 * c, kHiCp));
-            }
-          }
-#pragma unroll
-          for (int bx = 0; bx < C::kEBoxes; bx++)
-            tc_cp_128x128b(slot + C::cE + 4 * bx, desc_lohi(ls + ((C::oE + bx * C::BM * 16) >> 4), kHiCp));
-
+          // scale factors and metadata of this stage were written to its slot by the epilogue warps
+          if (!mbar_wait(&sf_ready[stage], phase, p.timeout_ns, abort_flag)) { *abort_flag = 1; break; }
+          tc_fence_after();
+          const uint32_t slot = tmem_base + C::BN + (uint32_t)(stage * C::kSlotCols);
           if (run_sparse) {
             if constexpr (SPARSE) {
               // backbone: sparse MMAs (32 bytes of compressed A, 64 bytes of W per MMA)
@@ -379,12 +361,52 @@ __global__ void __launch_bounds__(192, 1) gemm_kernel(const __grid_constant__ Ge
   } else {
     // ---------------------------------------------------------- epilogue
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16);
     int it = 0;
+    int stage = 0;
+    uint32_t phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, it++) {
       const int mt = tile % m_tiles, nt = tile / m_tiles;
       const int64_t m0 = (int64_t)mt * C::BM;
       const int e = tile_expert(m0);
       if (e < 0) { it--; continue; }
+      // scale factors and metadata of each K tile: shared memory -> this warp's
+      // quadrant of the stage's tensor-memory slot (the layout tcgen05.cp
+      // .32x128b.warpx4 and .128x128b would produce), so that the tensor pipe
+      // runs MMAs only
+      for (int kt = 0; kt < k_tiles; kt++) {
+        if (!mbar_wait(&full[stage], phase, p.timeout_ns, abort_flag)) { *abort_flag = 1; break; }
+        const uint8_t* sb = smem + stage * C::kStageBytes;
+        const uint32_t slot = tq + C::BN + (uint32_t)(stage * C::kSlotCols);
+#pragma unroll
+        for (int c = 0; c < C::kChunksR; c++) {
+          tmem_st4(slot + C::cSfaR + 4 * c, *reinterpret_cast<const uint4*>(sb + C::oSfaR + 512 * c + 16 * lane));
+#pragma unroll
+          for (int rb = 0; rb < C::kNRB; rb++)
+            tmem_st4(slot + C::cSfbD + 4 * C::kNRB * c + 4 * rb,
+                     *reinterpret_cast<const uint4*>(sb + C::oSfbD + rb * C::kChunksR * 512 + 512 * c + 16 * lane));
+        }
+#pragma unroll
+        for (int c = 0; c < C::kChunksB; c++) {
+          tmem_st4(slot + C::cSfaB + 4 * c, *reinterpret_cast<const uint4*>(sb + C::oSfaB + 512 * c + 16 * lane));
+          if constexpr (SPARSE) {
+#pragma unroll
+            for (int rb = 0; rb < C::kNRB; rb++)
+              tmem_st4(slot + C::cSfbS + 4 * C::kNRB * c + 4 * rb,
+                       *reinterpret_cast<const uint4*>(sb + C::oSfbS + rb * C::kChunksB * 512 + 512 * c + 16 * lane));
+          }
+        }
+#pragma unroll
+        for (int bx = 0; bx < C::kEBoxes; bx++)  // metadata: tile row 32q + lane
+          tmem_st4(slot + C::cE + 4 * bx,
+                   *reinterpret_cast<const uint4*>(sb + C::oE + bx * C::BM * 16 + 16 * (32 * q + lane)));
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sf_ready[stage]);
+        if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+      }
+      if (*abort_flag) break;
       if (!mbar_wait(acc_full, it & 1, p.timeout_ns, abort_flag)) { *abort_flag = 1; break; }
       if (*abort_flag) break;
       tc_fence_after();
@@ -393,9 +415,15 @@ __global__ void __launch_bounds__(192, 1) gemm_kernel(const __grid_constant__ Ge
       const bool st = row < p.t;
       const int64_t n0 = (int64_t)nt * C::BN;
 #pragma unroll 1
-      for (int c = 0; c < C::BN / 32; c++) {
-        uint32_t v[32];
-        tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(32 * c), v);
+      for (int c2 = 0; c2 < C::BN / 32; c2 += 2) {
+        uint32_t vv[2][32];
+        tmem_ld32_nowait(tq + (uint32_t)(32 * c2), vv[0]);
+        tmem_ld32_nowait(tq + (uint32_t)(32 * c2 + 32), vv[1]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int h = 0; h < 2; h++) {
+        const int c = c2 + h;
+        const uint32_t (&v)[32] = vv[h];
         if (st) {
           if (p.y_bf16) {
             uint32_t pk[16];
@@ -417,6 +445,7 @@ __global__ void __launch_bounds__(192, 1) gemm_kernel(const __grid_constant__ Ge
                                    __fmul_rn(__uint_as_float(v[4 * j + 2]), alpha),
                                    __fmul_rn(__uint_as_float(v[4 * j + 3]), alpha));
           }
+        }
         }
       }
       tc_fence_before();
