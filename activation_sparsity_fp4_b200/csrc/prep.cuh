@@ -76,6 +76,19 @@ __device__ __forceinline__ void load_unit(const void* base, int64_t off, float (
   }
 }
 
+// 32 bf16 values (4 x 16 bytes, element i in the low half first) -> fp32.
+__device__ __forceinline__ void unpack_bf16_unit(const uint4 (&w4)[4], float (&v)[32]) {
+#pragma unroll
+  for (int q = 0; q < 4; q++) {
+    const uint32_t ws[4] = {w4[q].x, w4[q].y, w4[q].z, w4[q].w};
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+      v[8 * q + 2 * j] = __uint_as_float(ws[j] << 16);
+      v[8 * q + 2 * j + 1] = __uint_as_float(ws[j] & 0xFFFF0000u);
+    }
+  }
+}
+
 // Two E2M1 codes (low nibble = first element) -> exact fp32 values.
 __device__ __forceinline__ void e2m1x2_values(uint32_t c, float& lo, float& hi) {
   uint32_t h2;
@@ -392,6 +405,84 @@ __global__ void __launch_bounds__(128) amax_kernel(const void* x, const void* ga
   if (threadIdx.x == 0) {
     const float mm = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
     atomicMax(reinterpret_cast<unsigned int*>(amax_out), __float_as_uint(mm));
+  }
+}
+
+// Amax pass for bf16 rows of k <= 4096 (at most 4 units per lane), one warp
+// per row and no block barrier: lane l owns the units l, l + 32, l + 64,
+// l + 96, so each 32-unit slab is one coalesced 2 KB read, and the whole row
+// is loaded into registers before any arithmetic.  The sum of squares follows
+// row_sumsq's fixed order: 16-element chunk sums, the pair of a unit,
+// butterflies over the 32 units of a slab, then the slab sums pairwise, zero
+// padded to 4.
+template <bool NORM>
+__global__ void __launch_bounds__(128, 4) amax_rows_kernel(const void* x, const void* gamma, float eps, int64_t t,
+                                                           int64_t k, float* amax_out, float* rstd_out) {
+  __shared__ float wmax[4];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int64_t r = (int64_t)blockIdx.x * 4 + w;
+  const int units = (int)(k / 32);
+  const int nj = (units + 31) >> 5;
+  float my = 0.0f;
+  if (r < t) {
+    const int64_t off = r * k;
+    uint4 raw[4][4];
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+      const int u = lane + 32 * j;
+      const bool on = j < nj && u < units;
+      const uint4* p4 = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x) + off + (int64_t)u * 32);
+#pragma unroll
+      for (int q = 0; q < 4; q++) raw[j][q] = on ? __ldg(p4 + q) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    float rs = 1.0f;
+    if constexpr (NORM) {
+      float sl[4];
+#pragma unroll
+      for (int j = 0; j < 4; j++) {
+        float v[32];
+        unpack_bf16_unit(raw[j], v);
+        float c0 = 0.0f, c1 = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; i++) c0 = __fmaf_rn(v[i], v[i], c0);
+#pragma unroll
+        for (int i = 16; i < 32; i++) c1 = __fmaf_rn(v[i], v[i], c1);
+        float a = __fadd_rn(c0, c1);
+#pragma unroll
+        for (int msk = 1; msk < 32; msk <<= 1) a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, msk));
+        sl[j] = j < nj ? a : 0.0f;
+      }
+      rs = rstd_from_sumsq(__fadd_rn(__fadd_rn(sl[0], sl[1]), __fadd_rn(sl[2], sl[3])), k, eps);
+      if (rstd_out && lane == 0) rstd_out[r] = rs;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+      const int u = lane + 32 * j;
+      if (j >= nj || u >= units) continue;
+      float v[32];
+      unpack_bf16_unit(raw[j], v);
+      if constexpr (NORM) {
+        float g[32];
+        load_unit<true>(gamma, (int64_t)u * 32, g);
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          mul2(v[i], v[i + 1], rs, rs);
+          mul2(v[i], v[i + 1], g[i], g[i + 1]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 32; i++) my = fmaxf(my, fabsf(v[i]));
+    }
+  }
+#pragma unroll
+  for (int msk = 16; msk >= 1; msk >>= 1) my = fmaxf(my, __shfl_xor_sync(0xffffffffu, my, msk));
+  if (lane == 0) wmax[w] = my;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const float mm = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
+    // non-negative floats order like their bit patterns; skip the atomic when it cannot raise the maximum
+    if (__float_as_uint(mm) > *reinterpret_cast<volatile unsigned int*>(amax_out))
+      atomicMax(reinterpret_cast<unsigned int*>(amax_out), __float_as_uint(mm));
   }
 }
 
