@@ -88,7 +88,7 @@ class ClockSampler:
                 self.samples.append((sm, rs))
             except Exception:
                 pass
-            time.sleep(0.002)
+            time.sleep(0.0002)
 
     def __enter__(self):
         import threading
