@@ -13,6 +13,7 @@
 
 #include "../../include/sharq.h"
 #include "gemm.cuh"
+#include "gemm_pair.cuh"
 #include "prep.cuh"
 
 using namespace sharq;
@@ -57,6 +58,15 @@ uint64_t wait_timeout_ns() {
   static uint64_t v = [] {
     const char* s = getenv("SHARQ_WAIT_TIMEOUT_NS");
     return s ? strtoull(s, nullptr, 10) : 2000000000ull;
+  }();
+  return v;
+}
+
+// SHARQ_GEMM_PAIRS=0 runs every GEMM on the single-CTA kernel (for comparison).
+bool pair_enabled() {
+  static const bool v = [] {
+    const char* e = getenv("SHARQ_GEMM_PAIRS");
+    return !(e && e[0] == '0');
   }();
   return v;
 }
@@ -225,6 +235,34 @@ sharq_status check_weight(const sharq_weight* w) {
   return SHARQ_OK;
 }
 
+// CTA-pair GEMM: clusters of 2 CTAs, one per SM, persistent over 256 x 256 tiles.
+template <int KIND>
+sharq_status launch_pair(const GemmMaps& maps, const GemmParams& gp, cudaStream_t s) {
+  using C = PairCfg<KIND>;
+  static bool configured = false;
+  if (!configured) {
+    SHARQ_CUDA(cudaFuncSetAttribute(gemm_pair_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    C::kSmemBytes));
+    configured = true;
+  }
+  const int tiles = (int)(gp.t_pad / 256) * (int)(gp.n / C::BN);
+  const int pairs = sm_count() / 2;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * (tiles < pairs ? tiles : pairs)));
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  SHARQ_CUDA(cudaLaunchKernelEx(&cfg, gemm_pair_kernel<KIND>, maps, gp));
+  return launched();
+}
+
 sharq_status run_linear(const sharq_prepared* a, const sharq_weight* w, const int32_t* offsets, void* y,
                         sharq_dtype y_dt, int32_t paths, cudaStream_t s) {
   sharq_status st = check_prepared(a);
@@ -288,6 +326,12 @@ sharq_status run_linear(const sharq_prepared* a, const sharq_weight* w, const in
   gp.y_bf16 = y_dt == SHARQ_BF16;
   gp.paths = paths;
   gp.timeout_ns = wait_timeout_ns();
+  if (sparse && !unpacked && offsets == nullptr && t_pad % 256 == 0 && pair_enabled()) {
+    // CTA pairs: each SM loads half of every weight tile (128-row weight boxes)
+    st = make_map(&maps.w, w->codes, w->k / 2, w->n, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != SHARQ_OK) return st;
+    return a->fmt == SHARQ_NVFP4 ? launch_pair<GK_NVF4>(maps, gp, s) : launch_pair<GK_MXF4>(maps, gp, s);
+  }
   if (a->fmt == SHARQ_NVFP4)
     return sparse ? launch_gemm<GK_NVF4, true>(maps, gp, s) : launch_gemm<GK_NVF4, false>(maps, gp, s);
   if (unpacked) return launch_gemm<GK_MXF8, true>(maps, gp, s);

@@ -107,6 +107,24 @@ def test_linear_each_path_separately(cuda_ok, fmt, pat):
         assert_close_gemm(y, ref, f"{fmt} {pat} paths={paths}")
 
 
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4"])
+def test_linear_cta_pairs(cuda_ok, fmt):
+    """Row counts whose 128-row padding is a multiple of 256 run on CTA pairs
+    (a 256 x 256 tile per pair of SMs): several pair tiles in M and N, ragged
+    rows, fewer K tiles than pipeline stages, and each path alone."""
+    t, k, n = 700, 768, 768  # padded to 768 rows = 3 pair tiles, 3 column tiles, 3 K tiles
+    x, w = _x(8, t, k), _w(9, n, k)
+    prep, wq = _ref(x, w, fmt, "4:8pair")
+    _, _, y = _run_linear(x, w, fmt, "4:8pair")
+    assert_close_gemm(y, oracle.linear_ref(prep, wq), f"{fmt} 4:8pair pairs")
+    bu, ru = oracle.decode_prepared(prep)
+    wu = oracle.decode_weight(wq)
+    alpha = float(prep["tensor"][2]) * float(wq["tensor"][2])
+    for paths, ref in ((1, alpha * bu @ wu.T), (2, alpha * ru @ wu.T)):
+        _, _, y = _run_linear(x, w, fmt, "4:8pair", paths=paths)
+        assert_close_gemm(y, ref, f"{fmt} 4:8pair pairs paths={paths}")
+
+
 def test_linear_bf16_output_and_single_row(cuda_ok):
     k, n = 512, 256
     w = _w(6, n, k)
