@@ -125,6 +125,7 @@ struct GemmParams {
 
 struct GemmMaps {
   CUtensorMap w, r, b, e;
+  CUtensorMap y;  // bf16 output, 32 x 32 boxes (CTA-pair kernel only)
 };
 
 template <int KIND, bool SPARSE>

@@ -12,7 +12,7 @@
 // Each SM therefore loads half a weight tile per stage instead of a whole one
 // (51 KB per stage instead of 67 KB), which leaves room for a fourth stage.
 //
-// Per CTA (192 threads, one CTA per SM):
+// Per CTA (448 threads, one CTA per SM):
 //   warp 0      TMA producer: weight half, residual and backbone tiles with the
 //               pair form of the tensor load, whose completion is counted on
 //               the leader's full[] barrier; metadata and scale factors on this
@@ -20,9 +20,12 @@
 //   warp 1      tensor-memory allocation for the pair; in the leader, the MMA
 //               issuer (one thread), committing to empty[] and acc_full of both
 //               CTAs;
-//   warps 2-5   scale factors and metadata of this CTA -> its tensor-memory
-//               slot (its own 128 activation rows, all 256 weight rows), then
-//               the accumulator drain of its 128 output rows.
+//   warps 2-9   the accumulator drain of its 128 output rows, two warps per
+//               32-lane quadrant, 128 columns each (bf16 output: the columns
+//               into registers first, then the accumulator is released and
+//               the stores drain under the next tile's MMAs);
+//   warps 10-13 scale factors and metadata of this CTA -> its tensor-memory
+//               slot (its own 128 activation rows, all 256 weight rows).
 // Four shared-memory stages, three tensor-memory scale slots (a slot is
 // rewritten once the MMAs of the K tile that used it have retired).  Every
 // wait is bounded in time; the abort flag of both CTAs is set on any timeout.
@@ -61,7 +64,8 @@ struct PairCfg {
   static constexpr int kSlotCols = cE + 4;
   static constexpr int kTmemCols = 512;
   static_assert(BN + kSlots * kSlotCols <= kTmemCols, "tensor memory budget");
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int kYBuf = 8 * 2048;  // bf16 output staging: 32 rows x 32 columns per epilogue warp
+  static constexpr int kSmemBytes = kStages * kStageBytes + kYBuf + 1024 /*align*/ + 256 /*barriers*/;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   // E2M1 x E2M1, K-major, M = 256 (the pair), N = 256
   static constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
@@ -74,11 +78,12 @@ __device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v
 }
 
 template <int KIND>
-__global__ void __launch_bounds__(192, 1) gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
+__global__ void __launch_bounds__(448, 1) gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
   using C = PairCfg<KIND>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);  // leader: both CTAs' tiles
+  uint8_t* ybuf = smem + C::kStages * C::kStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(ybuf + C::kYBuf);  // leader: both CTAs' tiles
   uint64_t* empty = full + C::kStages;       // this CTA: the stage's MMAs have retired
   uint64_t* sfull = empty + C::kStages;      // this CTA: its metadata and scale factors have landed
   uint64_t* sf_ready = sfull + C::kStages;   // leader: both CTAs' scale slots are in tensor memory
@@ -99,9 +104,9 @@ __global__ void __launch_bounds__(192, 1) gemm_pair_kernel(const __grid_constant
       mbar_init(&empty[s], 1);
       mbar_init(&sfull[s], 1);
     }
-    for (int j = 0; j < C::kSlots; j++) mbar_init(&sf_ready[j], 8);  // 4 warps x 2 CTAs
+    for (int j = 0; j < C::kSlots; j++) mbar_init(&sf_ready[j], 8);  // 4 staging warps x 2 CTAs
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 8);
+    mbar_init(acc_empty, 16);  // 8 epilogue warps x 2 CTAs
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -253,59 +258,66 @@ __global__ void __launch_bounds__(192, 1) gemm_pair_kernel(const __grid_constant
       tc_commit_pair(smem_u32(drain));
       (void)mbar_wait(drain, 0, 1000000000ull, nullptr, true);
     }
-  } else {
-    // -------------------------------------------- scale slots, then epilogue
-    const int q = warp & 3;
-    const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16);
-    const uint32_t sf_ready_leader = mapa_u32(smem_u32(sf_ready), 0);
+  } else if (warp < 10) {
+    // ------------------------------------------------------------- epilogue
+    // accumulator lanes 32q..32q+31 (this CTA's output rows), columns
+    // 128h..128h+127
+    constexpr int kCols = C::BN / 2;
+    const int q = warp & 3, hcol = (warp - 2) >> 2;
+    const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(kCols * hcol);
     const uint32_t acc_empty_leader = mapa_u32(smem_u32(acc_empty), 0);
-    uint32_t g = 0;
     int it = 0;
-    for (int tile = cluster; tile < num_tiles; tile += nclusters, it++) {
+    for (int tile = cluster; tile < num_tiles && !*abort_flag; tile += nclusters, it++) {
       const int mt = tile % m_pairs, nt = tile / m_pairs;
-      for (int kt = 0; kt < k_tiles; kt++, g++) {
-        const int stage = (int)(g % C::kStages), slot = (int)(g % C::kSlots);
-        if (g >= (uint32_t)C::kSlots) {  // the slot's previous K tile has been consumed by its MMAs
-          const uint32_t gp = g - C::kSlots;
-          if (!mbar_wait(&empty[gp % C::kStages], (gp / C::kStages) & 1u, p.timeout_ns, abort_flag)) {
-            abort_both();
-            break;
-          }
-        }
-        if (!mbar_wait(&sfull[stage], (g / C::kStages) & 1u, p.timeout_ns, abort_flag)) { abort_both(); break; }
-        const uint8_t* sb = smem + stage * C::kStageBytes;
-        const uint32_t st = tq + C::BN + (uint32_t)(slot * C::kSlotCols);
-#pragma unroll
-        for (int c = 0; c < C::kChunksR; c++) {
-          tmem_st4(st + C::cSfaR + 4 * c, *reinterpret_cast<const uint4*>(sb + C::oSfaR + 512 * c + 16 * lane));
-#pragma unroll
-          for (int rb = 0; rb < C::kNRB; rb++)
-            tmem_st4(st + C::cSfbD + 4 * C::kNRB * c + 4 * rb,
-                     *reinterpret_cast<const uint4*>(sb + C::oSfbD + rb * C::kChunksR * 512 + 512 * c + 16 * lane));
-        }
-#pragma unroll
-        for (int c = 0; c < C::kChunksB; c++) {
-          tmem_st4(st + C::cSfaB + 4 * c, *reinterpret_cast<const uint4*>(sb + C::oSfaB + 512 * c + 16 * lane));
-#pragma unroll
-          for (int rb = 0; rb < C::kNRB; rb++)
-            tmem_st4(st + C::cSfbS + 4 * C::kNRB * c + 4 * rb,
-                     *reinterpret_cast<const uint4*>(sb + C::oSfbS + rb * C::kChunksB * 512 + 512 * c + 16 * lane));
-        }
-        tmem_st4(st + C::cE, *reinterpret_cast<const uint4*>(sb + C::oE + 16 * (32 * q + lane)));
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_remote(sf_ready_leader + (uint32_t)(slot * 8));
-      }
-      if (*abort_flag) break;
       if (!mbar_wait(acc_full, (uint32_t)(it & 1), p.timeout_ns, abort_flag)) { abort_both(); break; }
       tc_fence_after();
       const float alpha = __fmul_rn(__ldg(p.tensor_x + 2), __ldg(p.tensor_w + 2));
       const int64_t row = (int64_t)mt * 256 + 128 * (int64_t)rank + 32 * q + lane;
       const bool store = row < p.t;
-      const int64_t n0 = (int64_t)nt * C::BN;
+      const int64_t n0 = (int64_t)nt * C::BN + kCols * hcol;
+      if (p.y_bf16) {
+        // this warp's columns into registers as bf16, then release the
+        // accumulator so the next tile's MMAs start while the stores drain
+        uint32_t pk[kCols / 2];
+#pragma unroll
+        for (int c = 0; c < kCols / 32; c++) {
+          uint32_t v[32];
+          tmem_ld32(tq + (uint32_t)(32 * c), v);
+#pragma unroll
+          for (int j = 0; j < 16; j++) {
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[2 * j]), alpha),
+                                                      __fmul_rn(__uint_as_float(v[2 * j + 1]), alpha));
+            pk[16 * c + j] = *reinterpret_cast<uint32_t*>(&h2);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(acc_empty_leader);
+        // 32 rows x 32 columns at a time through shared memory, written by a
+        // TMA store (whole lines; rows at or beyond t are clipped by the map)
+        (void)store;
+        uint8_t* yb = ybuf + (warp - 2) * 2048;
+        const int32_t row0 = (int32_t)(row - lane);
+        if (row0 >= p.t) continue;  // padding rows only: nothing to write
+#pragma unroll
+        for (int c = 0; c < kCols / 32; c++) {
+          if (lane == 0) bulk_wait_group_read0();  // the previous store has read the buffer
+          __syncwarp();
+          uint4* d = reinterpret_cast<uint4*>(yb + 64 * lane);
+#pragma unroll
+          for (int j = 0; j < 4; j++)
+            d[j] = make_uint4(pk[16 * c + 4 * j], pk[16 * c + 4 * j + 1], pk[16 * c + 4 * j + 2], pk[16 * c + 4 * j + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&maps.y, smem_u32(yb), (int32_t)(2 * (n0 + 32 * c)), row0);  // x in bytes
+            bulk_commit_group();
+          }
+        }
+        continue;
+      }
 #pragma unroll 1
-      for (int c2 = 0; c2 < C::BN / 32; c2 += 2) {
+      for (int c2 = 0; c2 < kCols / 32; c2 += 2) {
         uint32_t vv[2][32];
         tmem_ld32_nowait(tq + (uint32_t)(32 * c2), vv[0]);
         tmem_ld32_nowait(tq + (uint32_t)(32 * c2 + 32), vv[1]);
@@ -341,7 +353,52 @@ __global__ void __launch_bounds__(192, 1) gemm_pair_kernel(const __grid_constant
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(acc_empty_leader);
     }
+  } else {
+    // ------------------------------------------------ scale-slot staging
+    // warps 10-13, one per tensor-memory lane quadrant
+    const int q = warp & 3;
+    const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16);
+    const uint32_t sf_ready_leader = mapa_u32(smem_u32(sf_ready), 0);
+    uint32_t g = 0;
+    for (int tile = cluster; tile < num_tiles && !*abort_flag; tile += nclusters) {
+      for (int kt = 0; kt < k_tiles; kt++, g++) {
+        const int stage = (int)(g % C::kStages), slot = (int)(g % C::kSlots);
+        if (g >= (uint32_t)C::kSlots) {  // the slot's previous K tile has been consumed by its MMAs
+          const uint32_t gp = g - C::kSlots;
+          if (!mbar_wait(&empty[gp % C::kStages], (gp / C::kStages) & 1u, p.timeout_ns, abort_flag)) {
+            abort_both();
+            break;
+          }
+        }
+        if (!mbar_wait(&sfull[stage], (g / C::kStages) & 1u, p.timeout_ns, abort_flag)) { abort_both(); break; }
+        const uint8_t* sb = smem + stage * C::kStageBytes;
+        const uint32_t st = tq + C::BN + (uint32_t)(slot * C::kSlotCols);
+#pragma unroll
+        for (int c = 0; c < C::kChunksR; c++) {
+          tmem_st4(st + C::cSfaR + 4 * c, *reinterpret_cast<const uint4*>(sb + C::oSfaR + 512 * c + 16 * lane));
+#pragma unroll
+          for (int rb = 0; rb < C::kNRB; rb++)
+            tmem_st4(st + C::cSfbD + 4 * C::kNRB * c + 4 * rb,
+                     *reinterpret_cast<const uint4*>(sb + C::oSfbD + rb * C::kChunksR * 512 + 512 * c + 16 * lane));
+        }
+#pragma unroll
+        for (int c = 0; c < C::kChunksB; c++) {
+          tmem_st4(st + C::cSfaB + 4 * c, *reinterpret_cast<const uint4*>(sb + C::oSfaB + 512 * c + 16 * lane));
+#pragma unroll
+          for (int rb = 0; rb < C::kNRB; rb++)
+            tmem_st4(st + C::cSfbS + 4 * C::kNRB * c + 4 * rb,
+                     *reinterpret_cast<const uint4*>(sb + C::oSfbS + rb * C::kChunksB * 512 + 512 * c + 16 * lane));
+        }
+        tmem_st4(st + C::cE, *reinterpret_cast<const uint4*>(sb + C::oE + 16 * (32 * q + lane)));
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(sf_ready_leader + (uint32_t)(slot * 8));
+      }
+    }
   }
+
+  if (warp >= 2 && warp < 10 && lane == 0) bulk_wait_group0();  // output stores complete
 
   // the leader's MMAs read this CTA's shared memory and write its tensor
   // memory: neither CTA frees tensor memory or exits before both are done

@@ -345,6 +345,25 @@ __device__ __forceinline__ void mma_mxf4_sp_pair(uint32_t d, uint64_t a, uint64_
       : "memory");
 }
 
+// Shared -> global tile store (TMA; elements outside the tensor are not written).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t smem_src, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_src), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until the stores this thread committed have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_group_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Wait until the stores this thread committed are complete.
+__device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Make this thread's generic-proxy shared-memory writes visible to the async proxy (TMA).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Descriptor from its two 32-bit halves: lo = start >> 4 | (LBO >> 4) << 16,
 // hi = SBO >> 4 | version 1 << 14 | layout << 29.
 __device__ __forceinline__ uint64_t desc_lohi(uint32_t lo, uint32_t hi) {

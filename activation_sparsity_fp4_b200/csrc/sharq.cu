@@ -249,7 +249,7 @@ sharq_status launch_pair(const GemmMaps& maps, const GemmParams& gp, cudaStream_
   const int pairs = sm_count() / 2;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(2 * (tiles < pairs ? tiles : pairs)));
-  cfg.blockDim = dim3(192);
+  cfg.blockDim = dim3(448);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -330,6 +330,10 @@ sharq_status run_linear(const sharq_prepared* a, const sharq_weight* w, const in
     // CTA pairs: each SM loads half of every weight tile (128-row weight boxes)
     st = make_map(&maps.w, w->codes, w->k / 2, w->n, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != SHARQ_OK) return st;
+    if (y_dt == SHARQ_BF16) {  // output tiles of 32 rows x 32 bf16 columns; rows t.. are outside the map
+      st = make_map(&maps.y, y, w->n * 2, a->t, 64, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
+      if (st != SHARQ_OK) return st;
+    }
     return a->fmt == SHARQ_NVFP4 ? launch_pair<GK_NVF4>(maps, gp, s) : launch_pair<GK_MXF4>(maps, gp, s);
   }
   if (a->fmt == SHARQ_NVFP4)
