@@ -9,14 +9,19 @@
 // scale-factor view of the weight (one scale per 2b logical K for the sparse
 // MMA, the same scales repeated per b for the dense MMA).
 //
-// Structure (one CTA per SM, 6 warps):
+// Structure (one CTA per SM, 14 warps):
 //   warp 0      TMA producer: weight, residual, backbone and metadata tiles by
 //               cp.async.bulk.tensor, scale factors by 1-D cp.async.bulk;
-//   warp 1      TMEM owner and MMA issuer (one thread): tcgen05.cp of scales and
-//               metadata into tensor memory, tcgen05.mma.sp over the backbone,
-//               tcgen05.mma over the residual, tcgen05.commit to free stages;
-//   warps 2-5   epilogue: tcgen05.ld of the fp32 accumulator, times the tensor
-//               scales g_dec(x) * g_dec(w), stores y (bf16 or fp32).
+//   warp 1      TMEM owner and MMA issuer (one thread): tcgen05.mma.sp over the
+//               backbone, tcgen05.mma over the residual, tcgen05.commit to free
+//               stages and to hand the accumulator to the epilogue;
+//   warps 2-9   epilogue, two warps per 32-lane quadrant, half the columns
+//               each: tcgen05.ld of the fp32 accumulator, times the tensor
+//               scales g_dec(x) * g_dec(w); bf16 output is packed into
+//               registers, the accumulator released, and the tile written by
+//               TMA stores through shared memory; fp32 output is stored directly;
+//   warps 10-13 scale factors and metadata of each K tile, shared memory ->
+//               the stage's tensor-memory slot (tcgen05.st), one warp per quadrant.
 // Tiles are 128 x 256 outputs; a stage is 256 logical K.  Every wait is
 // bounded in time and reports through the device error word.
 #pragma once
@@ -92,7 +97,9 @@ struct GemmCfg {
   static constexpr int kSlotCols = cE + 4 * kEBoxes;
   static constexpr int kTmemCols = BN + kStages * kSlotCols <= 256 ? 256 : 512;
   static_assert(BN + kStages * kSlotCols <= kTmemCols, "tensor memory budget");
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int kYCols = 16;                // bf16 output staged 32 rows x 16 columns at a time
+  static constexpr int kYBuf = 8 * 32 * kYCols * 2;  // one chunk per epilogue warp
+  static constexpr int kSmemBytes = kStages * kStageBytes + kYBuf + 1024 /*align*/ + 256 /*barriers*/;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   // instruction descriptor (block-scaled kinds): E2M1 x E2M1, K-major, M=128, N=BN
   static constexpr uint32_t kFmt = kUnpacked ? 5u : 1u;
@@ -129,11 +136,12 @@ struct GemmMaps {
 };
 
 template <int KIND, bool SPARSE>
-__global__ void __launch_bounds__(192, 1) gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
+__global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
   using C = GemmCfg<KIND, SPARSE>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  uint8_t* ybuf = smem + C::kStages * C::kStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(ybuf + C::kYBuf);
   uint64_t* empty = full + C::kStages;
   uint64_t* acc_full = empty + C::kStages;
   uint64_t* acc_empty = acc_full + 1;
@@ -152,7 +160,7 @@ __global__ void __launch_bounds__(192, 1) gemm_kernel(const __grid_constant__ Ge
       mbar_init(&sf_ready[s], 4);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 4);
+    mbar_init(acc_empty, 8);  // 8 epilogue warps
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -359,22 +367,101 @@ __global__ void __launch_bounds__(192, 1) gemm_kernel(const __grid_constant__ Ge
       tc_commit(drain);
       (void)mbar_wait(drain, 0, 1000000000ull, nullptr, true);
     }
-  } else {
+  } else if (warp < 10) {
     // ---------------------------------------------------------- epilogue
-    const int q = warp & 3;  // TMEM lane quadrant this warp may access
-    const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16);
+    // accumulator lanes 32q..32q+31 (output rows), columns kCols*hcol ..
+    constexpr int kCols = C::BN / 2;
+    const int q = warp & 3, hcol = (warp - 2) >> 2;
+    const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(kCols * hcol);
+    uint8_t* yb = ybuf + (warp - 2) * (32 * C::kYCols * 2);
     int it = 0;
-    int stage = 0;
-    uint32_t phase = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, it++) {
+    for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x, it++) {
       const int mt = tile % m_tiles, nt = tile / m_tiles;
       const int64_t m0 = (int64_t)mt * C::BM;
       const int e = tile_expert(m0);
       if (e < 0) { it--; continue; }
-      // scale factors and metadata of each K tile: shared memory -> this warp's
-      // quadrant of the stage's tensor-memory slot (the layout tcgen05.cp
-      // .32x128b.warpx4 and .128x128b would produce), so that the tensor pipe
-      // runs MMAs only
+      if (!mbar_wait(acc_full, it & 1, p.timeout_ns, abort_flag)) { *abort_flag = 1; break; }
+      tc_fence_after();
+      const float alpha = __fmul_rn(__ldg(p.tensor_x + 2), __ldg(p.tensor_w + 3 * e + 2));
+      const int64_t row = m0 + 32 * q + lane;
+      const bool st = row < p.t;
+      const int64_t n0 = (int64_t)nt * C::BN + kCols * hcol;
+      if (p.y_bf16) {
+        // this warp's columns into registers as bf16, release the accumulator
+        // so the next tile's MMAs start, then 32 x 16 tiles through shared
+        // memory with TMA stores (rows at or beyond t are outside the map)
+        uint32_t pk[kCols / 2];
+#pragma unroll
+        for (int c = 0; c < kCols / 32; c++) {
+          uint32_t v[32];
+          tmem_ld32(tq + (uint32_t)(32 * c), v);
+#pragma unroll
+          for (int j = 0; j < 16; j++) {
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[2 * j]), alpha),
+                                                      __fmul_rn(__uint_as_float(v[2 * j + 1]), alpha));
+            pk[16 * c + j] = *reinterpret_cast<uint32_t*>(&h2);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty);
+        const int32_t row0 = (int32_t)(m0 + 32 * q);
+        if (row0 >= p.t) continue;  // padding rows only: nothing to write
+#pragma unroll
+        for (int c = 0; c < kCols / C::kYCols; c++) {
+          constexpr int kW = C::kYCols / 2;  // packed words per row and chunk
+          if (lane == 0) bulk_wait_group_read0();  // the previous store has read the buffer
+          __syncwarp();
+          uint4* d = reinterpret_cast<uint4*>(yb + C::kYCols * 2 * lane);
+#pragma unroll
+          for (int j = 0; j < kW / 4; j++)
+            d[j] = make_uint4(pk[kW * c + 4 * j], pk[kW * c + 4 * j + 1], pk[kW * c + 4 * j + 2], pk[kW * c + 4 * j + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&maps.y, smem_u32(yb), (int32_t)(2 * (n0 + C::kYCols * c)), row0);  // x in bytes
+            bulk_commit_group();
+          }
+        }
+        continue;
+      }
+#pragma unroll 1
+      for (int c2 = 0; c2 < kCols / 32; c2 += 2) {
+        uint32_t vv[2][32];
+        tmem_ld32_nowait(tq + (uint32_t)(32 * c2), vv[0]);
+        tmem_ld32_nowait(tq + (uint32_t)(32 * c2 + 32), vv[1]);
+        tmem_ld_wait();
+        if (!st) continue;
+#pragma unroll
+        for (int h = 0; h < 2; h++) {
+          const uint32_t(&v)[32] = vv[h];
+          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.y) + row * p.n + n0 + 32 * (c2 + h));
+#pragma unroll
+          for (int j = 0; j < 8; j++)
+            dst[j] = make_float4(__fmul_rn(__uint_as_float(v[4 * j]), alpha),
+                                 __fmul_rn(__uint_as_float(v[4 * j + 1]), alpha),
+                                 __fmul_rn(__uint_as_float(v[4 * j + 2]), alpha),
+                                 __fmul_rn(__uint_as_float(v[4 * j + 3]), alpha));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+    }
+    if (lane == 0) bulk_wait_group0();  // output stores complete
+  } else {
+    // ------------------------------------------------ scale-slot staging
+    // warps 10-13, one per tensor-memory lane quadrant: scale factors and
+    // metadata of each K tile, shared memory -> this warp's quadrant of the
+    // stage's tensor-memory slot (the layout tcgen05.cp .32x128b.warpx4 and
+    // .128x128b would produce), so that the tensor pipe runs MMAs only
+    const int q = warp & 3;
+    const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16);
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x) {
+      const int mt = tile % m_tiles;
+      if (tile_expert((int64_t)mt * C::BM) < 0) continue;
       for (int kt = 0; kt < k_tiles; kt++) {
         if (!mbar_wait(&full[stage], phase, p.timeout_ns, abort_flag)) { *abort_flag = 1; break; }
         const uint8_t* sb = smem + stage * C::kStageBytes;
@@ -407,51 +494,6 @@ __global__ void __launch_bounds__(192, 1) gemm_kernel(const __grid_constant__ Ge
         if (lane == 0) mbar_arrive(&sf_ready[stage]);
         if (++stage == C::kStages) { stage = 0; phase ^= 1; }
       }
-      if (*abort_flag) break;
-      if (!mbar_wait(acc_full, it & 1, p.timeout_ns, abort_flag)) { *abort_flag = 1; break; }
-      if (*abort_flag) break;
-      tc_fence_after();
-      const float alpha = __fmul_rn(__ldg(p.tensor_x + 2), __ldg(p.tensor_w + 3 * e + 2));
-      const int64_t row = m0 + 32 * q + lane;
-      const bool st = row < p.t;
-      const int64_t n0 = (int64_t)nt * C::BN;
-#pragma unroll 1
-      for (int c2 = 0; c2 < C::BN / 32; c2 += 2) {
-        uint32_t vv[2][32];
-        tmem_ld32_nowait(tq + (uint32_t)(32 * c2), vv[0]);
-        tmem_ld32_nowait(tq + (uint32_t)(32 * c2 + 32), vv[1]);
-        tmem_ld_wait();
-#pragma unroll
-        for (int h = 0; h < 2; h++) {
-        const int c = c2 + h;
-        const uint32_t (&v)[32] = vv[h];
-        if (st) {
-          if (p.y_bf16) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int j = 0; j < 16; j++) {
-              __nv_bfloat162 h2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[2 * j]), alpha),
-                                                        __fmul_rn(__uint_as_float(v[2 * j + 1]), alpha));
-              pk[j] = *reinterpret_cast<uint32_t*>(&h2);
-            }
-            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.y) + row * p.n + n0 + 32 * c);
-#pragma unroll
-            for (int j = 0; j < 4; j++) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-          } else {
-            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.y) + row * p.n + n0 + 32 * c);
-#pragma unroll
-            for (int j = 0; j < 8; j++)
-              dst[j] = make_float4(__fmul_rn(__uint_as_float(v[4 * j]), alpha),
-                                   __fmul_rn(__uint_as_float(v[4 * j + 1]), alpha),
-                                   __fmul_rn(__uint_as_float(v[4 * j + 2]), alpha),
-                                   __fmul_rn(__uint_as_float(v[4 * j + 3]), alpha));
-          }
-        }
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
     }
   }
 

@@ -203,7 +203,7 @@ sharq_status launch_gemm(const GemmMaps& maps, const GemmParams& gp, cudaStream_
   const int tiles = (int)(gp.t_pad / C::BM) * (int)(gp.n / C::BN);
   const int sms = sm_count();
   dim3 grid(tiles < sms ? tiles : sms);
-  gemm_kernel<KIND, SPARSE><<<grid, 192, C::kSmemBytes, s>>>(maps, gp);
+  gemm_kernel<KIND, SPARSE><<<grid, 448, C::kSmemBytes, s>>>(maps, gp);
   return launched();
 }
 
@@ -309,6 +309,12 @@ sharq_status run_linear(const sharq_prepared* a, const sharq_weight* w, const in
       if (st != SHARQ_OK) return st;
     }
   }
+  const bool pairs = sparse && !unpacked && offsets == nullptr && t_pad % 256 == 0 && pair_enabled();
+  if (y_dt == SHARQ_BF16) {
+    // output tiles of 32 rows x 32 (CTA pairs) or 16 bf16 columns; rows t.. are outside the map
+    st = make_map(&maps.y, y, w->n * 2, a->t, pairs ? 64 : 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != SHARQ_OK) return st;
+  }
   GemmParams gp;
   gp.t = a->t;
   gp.t_pad = t_pad;
@@ -326,14 +332,10 @@ sharq_status run_linear(const sharq_prepared* a, const sharq_weight* w, const in
   gp.y_bf16 = y_dt == SHARQ_BF16;
   gp.paths = paths;
   gp.timeout_ns = wait_timeout_ns();
-  if (sparse && !unpacked && offsets == nullptr && t_pad % 256 == 0 && pair_enabled()) {
+  if (pairs) {
     // CTA pairs: each SM loads half of every weight tile (128-row weight boxes)
     st = make_map(&maps.w, w->codes, w->k / 2, w->n, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != SHARQ_OK) return st;
-    if (y_dt == SHARQ_BF16) {  // output tiles of 32 rows x 32 bf16 columns; rows t.. are outside the map
-      st = make_map(&maps.y, y, w->n * 2, a->t, 64, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
-      if (st != SHARQ_OK) return st;
-    }
     return a->fmt == SHARQ_NVFP4 ? launch_pair<GK_NVF4>(maps, gp, s) : launch_pair<GK_MXF4>(maps, gp, s);
   }
   if (a->fmt == SHARQ_NVFP4)
