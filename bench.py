@@ -8,6 +8,10 @@ W 4096 x 4096), synthetic seeded data.  The weight is quantized once, outside
 the timed region (it is an offline step of the layer).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sharq|reference]
+                  [--workload q_proj|down_proj|wan|wan_816|qwen_moe_gate_up]
+
+The default workload is q_proj; the others measure the remaining layer shapes
+the pages evaluate (one JSON line each, same keys).
 
 Prints ONE JSON line (rank 0).  value = effective TFLOP/s = 2*T*N*K per step
 summed over ranks / max-over-ranks time; L2 is flushed (256 MB write) before
@@ -28,11 +32,61 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "effective TFLOP/s of sparse+dense FP4 linear (1 B200) + prep GB/s vs roofline"
-T, K, N = 2048, 4096, 4096
-WORKLOAD = "Llama-3.1-8B q_proj: X 2048x4096 bf16 (0.5*t3 + 8 outlier channels x100), RMSNorm, W 4096x4096; NVFP4, 4:8 pair"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 FP4_OVER_BF16 = 9.0 / 2.25          # nominal dense FP4 / dense BF16 ratio
-PREP_BYTES_PER_ELEM = 2.0 + 0.25 + 1 / 16 + 1 / 32 + 0.5 + 1 / 16  # bf16 in; bb codes, meta, bb sf, res codes, res sf
+FP8_OVER_BF16 = 4.5 / 2.25          # nominal dense FP8 / dense BF16 ratio
+
+WORKLOADS = {
+    "q_proj": "Llama-3.1-8B q_proj: X 2048x4096 bf16 (0.5*t3 + 8 outlier channels x100), RMSNorm, W 4096x4096; "
+              "NVFP4, 4:8 pair",
+    "down_proj": "Llama-3.1-8B down_proj: X 2048x14336 bf16 = SiLU(a)*b, a,b ~N(0,1); W 4096x14336 ~N(0,0.01^2); "
+                 "MXFP4, 2:4",
+    "wan": "Wan2.2-14B DiT linear: X 32768x5120 bf16 ~N(0,1) + 16 outlier channels x50, RMSNorm; W 5120x5120; "
+           "NVFP4, 4:8 pair",
+    "wan_816": "Wan2.2-14B DiT linear: X 32768x5120 bf16 ~N(0,1) + 16 outlier channels x50, RMSNorm; W 5120x5120; "
+               "NVFP4, 8:16",
+    "qwen_moe_gate_up": "Qwen3-30B-A3B MoE gate/up: 4096 tokens top-8 of 128 experts -> 32768 routed rows (each expert "
+                        "padded to 128 rows), hidden 2048; per expert W 1536x2048; NVFP4, 4:8 pair, no norm; grouped",
+}
+
+
+def prep_bytes_per_elem(fmt: str, pat: str, x_bytes: int = 2) -> float:
+    """Algorithmic bytes of sharq_prepare per element of X: X read, then backbone codes, metadata,
+    backbone scales, residual codes and residual scales written (layouts of sharq.h)."""
+    b = 16 if fmt == "nvfp4" else 32
+    meta = 1 / 16 if pat == "4:8pair" else 1 / 8
+    bb_codes = 0.5 if pat == "8:16" else 0.25
+    bb_sf = 1 / b if pat == "8:16" else 1 / (2 * b)  # 8:16 keeps the dense view (each scale twice)
+    return x_bytes + bb_codes + meta + bb_sf + 0.5 + 1 / b
+
+
+def make_workload(name: str) -> dict:
+    """Inputs and roofline terms of one bench workload (host arrays; nothing of the method here)."""
+    from activation_sparsity_fp4_b200 import workloads
+    if name == "qwen_moe_gate_up":
+        c = workloads.qwen_moe()
+        t, k = c["x"].shape
+        n = c["w_gu"].shape[1]
+        return dict(name=name, desc=WORKLOADS[name], x=c["x"], gamma=None, eps=1e-6, w=c["w_gu"], fmt="nvfp4",
+                    pat="4:8pair", offsets=c["offsets"], t=t, k=k, n=n, real_rows=int(c["counts"].sum()),
+                    first_group=(int(c["offsets"][0]), int(c["offsets"][1])))
+    c = {"q_proj": workloads.q_proj, "down_proj": workloads.down_proj, "wan": workloads.wan,
+         "wan_816": lambda: workloads.wan(pat="8:16")}[name]()
+    t, k = c["x"].shape
+    return dict(name=name, desc=WORKLOADS[name], x=c["x"], gamma=c["gamma"], eps=c["eps"], w=c["w"],
+                fmt=c["fmt"], pat=c["pat"], offsets=None, t=t, k=k, n=c["w"].shape[0], real_rows=t,
+                first_group=None)
+
+
+def gemm_roofline(wl: dict):
+    """(work per launch in FP4- or FP8-dense-equivalent flops, peak kind, description)."""
+    rows, n, k = wl["real_rows"], wl["n"], wl["k"]
+    if wl["pat"] == "8:16":
+        return 4.0 * rows * n * k, "fp4", "4*T*N*K: dense backbone 2TNK + dense residual 2TNK (kind::mxf4nvf4)"
+    if wl["fmt"] == "mxfp4" and wl["pat"] == "2:4":
+        return (3.0 * rows * n * k, "fp8",
+                "3*T*N*K FP8-dense-equivalent: sparse 2TNK at 2x + dense 2TNK, both kind::mxf8f6f4")
+    return 3.0 * rows * n * k, "fp4", "3*T*N*K FP4-dense-equivalent (sparse 2TNK at 2x rate + dense 2TNK)"
 
 
 def peaks():
@@ -142,38 +196,42 @@ def committed_traffic():
 _ORACLE_SETUP = {}
 
 
-def _oracle_setup():
+def _oracle_setup(name: str):
     """Workload and the offline weight quantization for the oracle (untimed, once)."""
-    if not _ORACLE_SETUP:
+    if _ORACLE_SETUP.get("name") != name:
         import oracle
-        from activation_sparsity_fp4_b200 import workloads
-        cfg = workloads.q_proj()
-        wq = oracle.quantize_weight(cfg["w"], "nvfp4")
-        _ORACLE_SETUP.update(cfg=cfg, wq=wq, wu=oracle.decode_weight(wq))
+        wl = make_workload(name)
+        w = wl["w"][0] if wl["offsets"] is not None else wl["w"]  # grouped: the first expert's weight
+        wq = oracle.quantize_weight(w, wl["fmt"])
+        _ORACLE_SETUP.clear()
+        _ORACLE_SETUP.update(name=name, wl=wl, wq=wq, wu=oracle.decode_weight(wq))
     return _ORACLE_SETUP
 
 
-def cpu_baseline(rows: int = T):
-    """The oracle, as it stands, on the host cores: tensor amax over all rows,
-    prep of the first `rows` rows and the fp64 reference GEMM of those rows;
-    scaled to effective TFLOP/s (2 * rows * N * K / time)."""
+def cpu_baseline(name: str = "q_proj", rows: int = 2048):
+    """The oracle, as it stands, on the host cores: the tensor amax over all rows
+    (NVFP4), prep of `rows` rows (grouped: rows of the first expert) and the fp64
+    reference GEMM of those rows; scaled to effective TFLOP/s (2 * rows * N * K / time)."""
     import numpy as np
 
     import oracle
 
-    st = _oracle_setup()
-    cfg, wq, wu = st["cfg"], st["wq"], st["wu"]
+    st = _oracle_setup(name)
+    wl, wq, wu = st["wl"], st["wq"], st["wu"]
+    x = wl["x"]
+    r0 = wl["first_group"][0] if wl["first_group"] else 0
+    rows = min(rows, (wl["first_group"][1] - r0) if wl["first_group"] else wl["t"])
     cores = len(os.sched_getaffinity(0))
     t0 = time.perf_counter()
-    amax = oracle.rows_amax(cfg["x"], cfg["gamma"], cfg["eps"])
-    prep = oracle.prepare(cfg["x"][:rows], "nvfp4", "4:8pair", gamma=cfg["gamma"], eps=cfg["eps"], act_amax=amax,
+    amax = oracle.rows_amax(x, wl["gamma"], wl["eps"]) if wl["fmt"] == "nvfp4" else 0.0
+    prep = oracle.prepare(x[r0:r0 + rows], wl["fmt"], wl["pat"], gamma=wl["gamma"], eps=wl["eps"], act_amax=amax,
                           threads=cores)
     y = oracle.linear_ref(prep, wq, wu=wu)
     dt = time.perf_counter() - t0
     assert np.isfinite(y).all()
-    value = 2.0 * rows * N * K / dt / 1e12
+    value = 2.0 * rows * wl["n"] * wl["k"] / dt / 1e12
     return {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": f"{rows} of {T} rows: tensor amax over all rows, prep of those rows with {cores} threads, "
+            "sample": f"{rows} of {wl['t']} rows: tensor amax over all rows, prep of those rows with {cores} threads, "
                       f"fp64 numpy GEMM of those rows ({dt:.2f} s)"}, dt
 
 
@@ -182,7 +240,7 @@ def run_sharq(args):
     import numpy as np
     import torch
 
-    from activation_sparsity_fp4_b200 import sharq, workloads
+    from activation_sparsity_fp4_b200 import sharq
 
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
@@ -195,22 +253,34 @@ def run_sharq(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         pg = dist
 
-    cfg = workloads.q_proj()
-    x_host = torch.from_numpy(cfg["x"]).to(torch.bfloat16).pin_memory()
+    wl = make_workload(args.workload)
+    T, K, N, fmt, pat = wl["t"], wl["k"], wl["n"], wl["fmt"], wl["pat"]
+    x_host = torch.from_numpy(wl["x"]).to(torch.bfloat16).pin_memory()
     x = x_host.to(dev)
-    gamma = torch.from_numpy(cfg["gamma"]).to(torch.bfloat16).to(dev)
-    w = torch.from_numpy(cfg["w"]).to(torch.bfloat16).to(dev)
-    wq = sharq.FP4Weight.quantize(w, "nvfp4")
-    prep = sharq.Prepared(T, K, "nvfp4", "4:8pair", dev)
-    y = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
+    gamma = torch.from_numpy(wl["gamma"]).to(torch.bfloat16).to(dev) if wl["gamma"] is not None else None
+    w = torch.from_numpy(wl["w"]).to(torch.bfloat16).to(dev)
+    wq = sharq.FP4Weight.quantize(w, fmt)
+    del w
+    offsets = torch.from_numpy(wl["offsets"]).to(torch.int32).to(dev) if wl["offsets"] is not None else None
+    prep = sharq.Prepared(T, K, fmt, pat, dev)
+    y = torch.zeros((T, N), dtype=torch.bfloat16, device=dev)
     y_host = torch.empty((T, N), dtype=torch.bfloat16).pin_memory()
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     sharq.sharq_sync_status()
 
+    def do_prep(act_amax=0.0):
+        sharq.prepare(x, fmt, pat, gamma, wl["eps"], act_amax=act_amax, out=prep)
+
+    def do_gemm():
+        if offsets is None:
+            sharq.linear(prep, wq, out=y)
+        else:
+            sharq.linear_grouped(prep, wq, offsets, out=y)
+
     def step():
-        sharq.prepare(x, "nvfp4", "4:8pair", gamma, cfg["eps"], out=prep)
-        sharq.linear(prep, wq, out=y)
+        do_prep()
+        do_gemm()
 
     for _ in range(args.warmup):
         flush.fill_(1)
@@ -222,9 +292,9 @@ def run_sharq(args):
     g_prep, g_gemm = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
     sharq.sharq_launch_count(reset=True)
     with torch.cuda.graph(g_prep):
-        sharq.prepare(x, "nvfp4", "4:8pair", gamma, cfg["eps"], out=prep)
+        do_prep()
     with torch.cuda.graph(g_gemm):
-        sharq.linear(prep, wq, out=y)
+        do_gemm()
     launches_per_step = sharq.sharq_launch_count()
     for _ in range(args.warmup):
         flush.fill_(1)
@@ -262,7 +332,7 @@ def run_sharq(args):
     for i in range(args.steps):
         flush.fill_(1)
         pev[i][0].record(stream)
-        sharq.prepare(x, "nvfp4", "4:8pair", gamma, cfg["eps"], act_amax=amax, out=prep)
+        do_prep(amax if fmt == "nvfp4" else 0.0)
         pev[i][1].record(stream)
     torch.cuda.synchronize()
     prep_given_ms = statistics.mean(a.elapsed_time(b) for a, b in pev)
@@ -287,15 +357,22 @@ def run_sharq(args):
 
     if rank == 0:
         pk, src = peaks()
-        flops = 2.0 * T * N * K
+        flops = 2.0 * wl["real_rows"] * N * K
         value = world * flops * args.steps / (total_ms / 1e3) / 1e12
         gemm_avg = statistics.mean(gemm_ms) / 1e3
-        fp4_peak = pk["bf16_tflops"] * FP4_OVER_BF16
-        achieved = 3.0 * T * N * K / gemm_avg / 1e12   # FP4-dense-equivalent work of the pair
-        prep_bytes = PREP_BYTES_PER_ELEM * T * K
+        work, kind, work_desc = gemm_roofline(wl)
+        ratio = FP4_OVER_BF16 if kind == "fp4" else FP8_OVER_BF16
+        peak = pk["bf16_tflops"] * ratio
+        achieved = work / gemm_avg / 1e12
+        bpe = prep_bytes_per_elem(fmt, pat)
+        prep_bytes = bpe * T * K
         prep_gbs = prep_bytes / (statistics.mean(prep_ms) / 1e3) / 1e9
         prep_given_gbs = prep_bytes / (prep_given_ms / 1e3) / 1e9
         clocks = clk.summary()
+        grouped = offsets is not None
+        kernel = {"4:8pair": "sparse", "2:4": "sparse", "8:16": "dense backbone"}[pat]
+        kname = ("gemm_pair_kernel" if (not grouped and pat == "4:8pair" and T % 256 == 0) else "gemm_kernel")
+        kkind = "MXF8" if (fmt == "mxfp4" and pat == "2:4") else ("NVF4" if fmt == "nvfp4" else "MXF4")
         out = {
             "metric": METRIC,
             "value": round(value, 2),
@@ -307,21 +384,23 @@ def run_sharq(args):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": "nvfp4 (e2m1 x e4m3 block-16 scales, fp32 accumulate)",
-            "data": "synthetic (seeded, shaped like the pages' Llama-3.1-8B q_proj layer)",
-            "config": {"workload": WORKLOAD, "t": T, "k": K, "n": N, "fmt": "nvfp4", "pattern": "4:8 pair",
-                       "norm": "rmsnorm", "y_dtype": "bf16", "parallelism": f"replicas x{world}",
+            "dtype": (f"{fmt} (e2m1 x {'e4m3 block-16' if fmt == 'nvfp4' else 'e8m0 block-32'} scales, "
+                      "fp32 accumulate)"),
+            "data": f"synthetic (seeded, shaped like the pages' {args.workload} layer)",
+            "config": {"workload": wl["desc"], "t": T, "k": K, "n": N, "fmt": fmt, "pattern": pat,
+                       "norm": "rmsnorm" if gamma is not None else "none", "y_dtype": "bf16",
+                       "parallelism": f"replicas x{world}",
                        "l2": "flushed (256 MB write) before every timed step"},
-            "roofline": {"bound": "tensor", "kernel": "gemm_kernel<NVF4, sparse>",
-                         "achieved": round(achieved, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
-                         "frac": round(achieved / fp4_peak, 4), "traffic": committed_traffic(),
-                         "peak_source": f"{src}: bf16 burst x {FP4_OVER_BF16:g} (nominal FP4/BF16)",
-                         "work": "3*T*N*K FP4-dense-equivalent flops per launch (sparse 2TNK at 2x rate + dense 2TNK)",
-                         "avg_launch_us": round(gemm_avg * 1e6, 2)},
+            "roofline": {"bound": "tensor", "kernel": f"{kname}<{kkind}, {kernel}>",
+                         "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
+                         "frac": round(achieved / peak, 4),
+                         "traffic": committed_traffic() if args.workload == "q_proj" else None,
+                         "peak_source": f"{src}: bf16 burst x {ratio:g} (nominal {kind.upper()}/BF16)",
+                         "work": work_desc, "avg_launch_us": round(gemm_avg * 1e6, 2)},
             "prep": {"gbs_device_amax": round(prep_gbs, 1), "gbs_given_amax": round(prep_given_gbs, 1),
                      "peak_gbs": pk["hbm_gbs"], "frac_given_amax": round(prep_given_gbs / pk["hbm_gbs"], 4),
                      "frac_device_amax": round(prep_gbs / pk["hbm_gbs"], 4),
-                     "bytes_per_elem": PREP_BYTES_PER_ELEM, "avg_us": round(statistics.mean(prep_ms) * 1e3, 2),
+                     "bytes_per_elem": bpe, "avg_us": round(statistics.mean(prep_ms) * 1e3, 2),
                      "avg_us_given_amax": round(prep_given_ms * 1e3, 2)},
             "e2e": {"value": round(world * flops * args.steps / (e2e_ms / 1e3) / 1e12, 3), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": int(x_host.numel() * 2), "d2h_bytes_per_step": int(y_host.numel() * 2)},
@@ -329,8 +408,11 @@ def run_sharq(args):
             "launch_mode": "CUDA graphs (prep graph + GEMM graph per step); e2e uses direct API calls",
             "clocks": clocks,
         }
+        if grouped:
+            out["config"]["routed_rows"] = wl["real_rows"]
+            out["config"]["experts"] = int(wl["w"].shape[0])
         if not args.no_cpu_baseline and world == 1:
-            out["cpu_baseline"], _ = cpu_baseline()
+            out["cpu_baseline"], _ = cpu_baseline(args.workload)
         print(json.dumps(out), flush=True)
     if pg:
         pg.barrier()
@@ -345,21 +427,22 @@ def run_reference(args):
         return
     rows = 256
     for _ in range(args.warmup):
-        cpu_baseline(rows)
+        cpu_baseline(args.workload, rows)
     times = []
     base = None
     for _ in range(args.steps):
-        base, dt = cpu_baseline(rows)
+        base, dt = cpu_baseline(args.workload, rows)
         times.append(dt)
+    wl = _ORACLE_SETUP["wl"]
     total = sum(times)
-    value = 2.0 * rows * N * K * args.steps / total / 1e12
+    value = 2.0 * rows * wl["n"] * wl["k"] * args.steps / total / 1e12
     base["value"] = value
     out = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32 prep / f64 GEMM (CPU oracle)",
         "data": "synthetic", "impl": "reference",
-        "config": {"workload": WORKLOAD, "t": T, "k": K, "n": N, "sample_rows_per_step": rows},
+        "config": {"workload": wl["desc"], "t": wl["t"], "k": wl["k"], "n": wl["n"], "sample_rows_per_step": rows},
         "cpu_baseline": base,
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -373,6 +456,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["sharq", "reference"], default="sharq")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="q_proj")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
