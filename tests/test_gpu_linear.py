@@ -125,6 +125,53 @@ def test_linear_cta_pairs(cuda_ok, fmt):
         assert_close_gemm(y, ref, f"{fmt} 4:8pair pairs paths={paths}")
 
 
+def _bf16_round(a: np.ndarray) -> np.ndarray:
+    """fp32 -> the nearest bf16 value (ties to even), as float32."""
+    return workloads.to_bf16_values(np.asarray(a, dtype=np.float32))
+
+
+@pytest.mark.parametrize("fmt,pat", LINEAR_CASES)
+@pytest.mark.parametrize("t", [300, 700])
+def test_linear_bf16_output_equals_rounded_fp32(cuda_ok, fmt, pat, t):
+    """bf16 output (written through shared memory by TMA stores) equals the fp32
+    output of the same operands rounded to bf16, element for element, on both
+    GEMM kernels (t=300 pads to 384 rows: single-CTA; t=700 pads to 768: CTA
+    pairs for 4:8 pair) with several column tiles; rows past t stay untouched."""
+    k, n = 512, 768
+    x, w = _x(10, t, k), _w(11, n, k)
+    p = gpu_prepare(x, "bf16", fmt, pat)
+    wq = gpu_weight(w, "bf16", fmt)
+    y32 = sharq.linear(p, wq, out_dtype=torch.float32)
+    guard = torch.full((t + 64, n), 7.0, dtype=torch.bfloat16, device="cuda")
+    sharq.linear(p, wq, out=guard[:t])
+    sharq.sharq_sync_status()
+    y16 = guard[:t].float().cpu().numpy()
+    ref = _bf16_round(y32.cpu().numpy())
+    bad = np.argwhere(y16 != ref)
+    assert bad.size == 0, f"{fmt} {pat} t={t}: {len(bad)} bf16 outputs differ, first {bad[:3].tolist()}"
+    assert bool((guard[t:] == 7.0).all()), "rows past t were written"
+
+
+def test_linear_grouped_bf16_output_equals_rounded_fp32(cuda_ok):
+    """The grouped launch's bf16 output equals its fp32 output rounded to bf16."""
+    rng = np.random.default_rng(12)
+    experts, k, n = 3, 512, 512
+    counts = [128, 256, 128]
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    t = int(offsets[-1])
+    x = _x(13, t, k)
+    w = workloads.to_bf16_values((rng.standard_normal((experts, n, k)) * 0.02).astype(np.float32))
+    p = gpu_prepare(x, "bf16", "nvfp4", "4:8pair")
+    wq = sharq.FP4Weight.quantize(to_dev(w, "bf16"), "nvfp4")
+    off_dev = torch.from_numpy(offsets).cuda()
+    y32 = sharq.linear_grouped(p, wq, off_dev, out_dtype=torch.float32)
+    y16 = sharq.linear_grouped(p, wq, off_dev, out_dtype=torch.bfloat16)
+    sharq.sharq_sync_status()
+    ref = _bf16_round(y32.cpu().numpy())
+    bad = np.argwhere(y16.float().cpu().numpy() != ref)
+    assert bad.size == 0, f"grouped: {len(bad)} bf16 outputs differ, first {bad[:3].tolist()}"
+
+
 def test_linear_bf16_output_and_single_row(cuda_ok):
     k, n = 512, 256
     w = _w(6, n, k)
