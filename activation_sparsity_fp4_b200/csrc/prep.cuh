@@ -408,62 +408,79 @@ __global__ void __launch_bounds__(128) amax_kernel(const void* x, const void* ga
   }
 }
 
-// Amax pass for bf16 rows of k <= 4096 (at most 4 units per lane), one warp
-// per row and no block barrier: lane l owns the units l, l + 32, l + 64,
-// l + 96, so each 32-unit slab is one coalesced 2 KB read, and the whole row
-// is loaded into registers before any arithmetic.  The sum of squares follows
+// Amax pass for bf16 rows of k <= 4096 (at most 4 units per lane).  Two rows
+// per block, two warps per row: lane l of warp h holds the units
+// l + 32 (2h) and l + 32 (2h + 1), so each 32-unit slab is one coalesced
+// 2 KB read, and all of a row's loads are issued before any arithmetic;
+// gamma is copied into shared memory meanwhile.  The sum of squares follows
 // row_sumsq's fixed order: 16-element chunk sums, the pair of a unit,
-// butterflies over the 32 units of a slab, then the slab sums pairwise, zero
-// padded to 4.
+// butterflies over the 32 units of a slab, then the slab sums pairwise
+// ((s0 + s1) + (s2 + s3), zero padded), the halves exchanged through
+// shared memory at the one block barrier.
 template <bool NORM>
-__global__ void __launch_bounds__(128, 4) amax_rows_kernel(const void* x, const void* gamma, float eps, int64_t t,
+__global__ void __launch_bounds__(128, 7) amax_rows_kernel(const void* x, const void* gamma, float eps, int64_t t,
                                                            int64_t k, float* amax_out, float* rstd_out) {
   __shared__ float wmax[4];
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int64_t r = (int64_t)blockIdx.x * 4 + w;
+  __shared__ float ssum[4];
+  __shared__ uint4 gs[4096 / 8];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, hw = w & 1;
+  const int64_t r = (int64_t)blockIdx.x * 2 + (w >> 1);
+  const bool have = r < t;
   const int units = (int)(k / 32);
   const int nj = (units + 31) >> 5;
+  const int64_t off = r * k;
+  uint4 raw[2][4];
+#pragma unroll
+  for (int jj = 0; jj < 2; jj++) {
+    const int j = 2 * hw + jj;
+    const int u = lane + 32 * j;
+    const bool on = have && j < nj && u < units;
+    const uint4* p4 = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x) + (on ? off + (int64_t)u * 32 : 0));
+#pragma unroll
+    for (int q = 0; q < 4; q++) raw[jj][q] = on ? __ldg(p4 + q) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  if constexpr (NORM) {
+    const uint4* g4 = static_cast<const uint4*>(gamma);
+    for (int i = threadIdx.x; i < (int)(k / 8); i += 128) gs[i] = __ldg(g4 + i);
+  }
+  float rs = 1.0f;
+  if constexpr (NORM) {
+    float sl[2];
+#pragma unroll
+    for (int jj = 0; jj < 2; jj++) {
+      float v[32];
+      unpack_bf16_unit(raw[jj], v);
+      float c0 = 0.0f, c1 = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 16; i++) c0 = __fmaf_rn(v[i], v[i], c0);
+#pragma unroll
+      for (int i = 16; i < 32; i++) c1 = __fmaf_rn(v[i], v[i], c1);
+      float a = __fadd_rn(c0, c1);
+#pragma unroll
+      for (int msk = 1; msk < 32; msk <<= 1) a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, msk));
+      sl[jj] = (2 * hw + jj) < nj ? a : 0.0f;
+    }
+    if (lane == 0) ssum[w] = __fadd_rn(sl[0], sl[1]);
+  }
+  __syncthreads();  // every thread: gamma in shared memory, half-row sums exchanged
   float my = 0.0f;
-  if (r < t) {
-    const int64_t off = r * k;
-    uint4 raw[4][4];
-#pragma unroll
-    for (int j = 0; j < 4; j++) {
-      const int u = lane + 32 * j;
-      const bool on = j < nj && u < units;
-      const uint4* p4 = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x) + off + (int64_t)u * 32);
-#pragma unroll
-      for (int q = 0; q < 4; q++) raw[j][q] = on ? __ldg(p4 + q) : make_uint4(0u, 0u, 0u, 0u);
-    }
-    float rs = 1.0f;
+  if (have) {
     if constexpr (NORM) {
-      float sl[4];
-#pragma unroll
-      for (int j = 0; j < 4; j++) {
-        float v[32];
-        unpack_bf16_unit(raw[j], v);
-        float c0 = 0.0f, c1 = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 16; i++) c0 = __fmaf_rn(v[i], v[i], c0);
-#pragma unroll
-        for (int i = 16; i < 32; i++) c1 = __fmaf_rn(v[i], v[i], c1);
-        float a = __fadd_rn(c0, c1);
-#pragma unroll
-        for (int msk = 1; msk < 32; msk <<= 1) a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, msk));
-        sl[j] = j < nj ? a : 0.0f;
-      }
-      rs = rstd_from_sumsq(__fadd_rn(__fadd_rn(sl[0], sl[1]), __fadd_rn(sl[2], sl[3])), k, eps);
-      if (rstd_out && lane == 0) rstd_out[r] = rs;
+      const int w0 = w & ~1;
+      rs = rstd_from_sumsq(__fadd_rn(ssum[w0], ssum[w0 + 1]), k, eps);
+      if (rstd_out && lane == 0 && hw == 0) rstd_out[r] = rs;
     }
 #pragma unroll
-    for (int j = 0; j < 4; j++) {
+    for (int jj = 0; jj < 2; jj++) {
+      const int j = 2 * hw + jj;
       const int u = lane + 32 * j;
       if (j >= nj || u >= units) continue;
       float v[32];
-      unpack_bf16_unit(raw[j], v);
+      unpack_bf16_unit(raw[jj], v);
       if constexpr (NORM) {
         float g[32];
-        load_unit<true>(gamma, (int64_t)u * 32, g);
+        const uint4 g4[4] = {gs[4 * u], gs[4 * u + 1], gs[4 * u + 2], gs[4 * u + 3]};
+        unpack_bf16_unit(g4, g);
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
           mul2(v[i], v[i + 1], rs, rs);
@@ -480,7 +497,6 @@ __global__ void __launch_bounds__(128, 4) amax_rows_kernel(const void* x, const 
   __syncthreads();
   if (threadIdx.x == 0) {
     const float mm = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
-    // non-negative floats order like their bit patterns; skip the atomic when it cannot raise the maximum
     if (__float_as_uint(mm) > *reinterpret_cast<volatile unsigned int*>(amax_out))
       atomicMax(reinterpret_cast<unsigned int*>(amax_out), __float_as_uint(mm));
   }

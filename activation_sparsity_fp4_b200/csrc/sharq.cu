@@ -165,8 +165,8 @@ sharq_status launch_prep(const PrepParams& pp, cudaStream_t s) {
 template <bool NORM, bool XBF16>
 sharq_status launch_amax(const void* x, const void* gamma, float eps, int64_t t, int64_t k, float* out,
                          float* rstd_out, cudaStream_t s) {
-  if (XBF16 && k <= 4096) {  // one warp per row, the row in registers, four rows per block
-    amax_rows_kernel<NORM><<<(unsigned)((t + 3) / 4), 128, 0, s>>>(x, gamma, eps, t, k, out, rstd_out);
+  if (XBF16 && k <= 4096) {  // two warps per row, the row in registers, two rows per block
+    amax_rows_kernel<NORM><<<(unsigned)((t + 1) / 2), 128, 0, s>>>(x, gamma, eps, t, k, out, rstd_out);
     return launched();
   }
   auto kern = amax_kernel<NORM, XBF16>;
