@@ -76,6 +76,9 @@ def _load():
             "orc_decode_prepared": (None, [P, P, P, P, P, I64, I64, I, I, P, P]),
             "orc_decode_weight": (None, [P, P, I64, I64, I, P]),
             "orc_meta_bytes_per_row": (I64, [I64, I]),
+            "orc_exp": (F, [F]),
+            "orc_silu": (F, [F]),
+            "orc_swiglu": (None, [P, P, I64, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -180,6 +183,28 @@ def rows_amax(x, gamma=None, eps: float = 1e-6) -> float:
     x = _f32(x)
     g = None if gamma is None else _f32(gamma)
     return float(_load().orc_rows_amax(_ptr(x), x.shape[0], x.shape[1], _ptr(g), eps))
+
+
+def exp(x) -> np.ndarray:
+    """The oracle's fp32 exponential (Cody-Waite reduction + degree-7 Taylor), elementwise."""
+    lib = _load()
+    x = _f32(x)
+    return np.array([lib.orc_exp(float(v)) for v in x.ravel()], np.float32).reshape(x.shape)
+
+
+def swiglu(gate, up) -> np.ndarray:
+    """h = SiLU(gate) * up in the oracle's fixed fp32 steps (inputs converted exactly to fp32)."""
+    a, b = _f32(gate), _f32(up)
+    assert a.shape == b.shape
+    h = np.empty_like(a)
+    _load().orc_swiglu(_ptr(a), _ptr(b), a.size, _ptr(h))
+    return h
+
+
+def prepare_swiglu(gate, up, fmt, pat, act_amax: float = 0.0, *, threads: int = 1, want_float: bool = False) -> dict:
+    """Preprocessing of a down projection's input formed on the fly: h = SiLU(gate) * up
+    (no RMSNorm), then the mask, backbone and residual of ``prepare``."""
+    return prepare(swiglu(gate, up), fmt, pat, None, 1e-6, act_amax, threads=threads, want_float=want_float)
 
 
 def prepare(x, fmt, pat, gamma=None, eps: float = 1e-6, act_amax: float = 0.0, *, threads: int = 1,

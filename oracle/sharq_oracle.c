@@ -140,6 +140,60 @@ float orc_rms_rstd(const float* x, int64_t k, float eps) {
   return r;
 }
 
+/* -------------------------------------------------------------- SwiGLU ----
+ * Gated activation feeding a down projection: h = SiLU(gate) * up, fused into
+ * the preprocessing so that h never goes to memory (an extension of the SharQ
+ * abstract's fusing of the layer norm into the preprocessing op; the pages
+ * give no formula).  Fixed fp32 steps, each rounded once:
+ *   SiLU(a) = a / (1 + E(-a)),   h = SiLU(a) * b,
+ * with E the exponential below.
+ *
+ * E(x) = e^x by Cody and Waite's range reduction and a Taylor polynomial:
+ *   x is clamped to [-104, 89] (outside, e^x is 0 or inf in fp32 anyway);
+ *   n = rint(x * log2(e))                        (nearest integer, ties to even);
+ *   r = fmaf(-n, LN2_HI, x), r = fmaf(-n, LN2_LO, r)   (|r| <= ln(2)/2 + tiny;
+ *       LN2_HI = ln 2 to 15 significant bits, LN2_LO = ln 2 - LN2_HI rounded:
+ *       ln 2 carried to about 39 bits across the two fused steps);
+ *   p = sum_{i=0..7} r^i / i!  by Horner, p = fmaf(p, r, 1/i!) from i = 7 down;
+ *   E = (p * 2^n1) * 2^n2 with n1 = n / 2, n2 = n - n1 (exact scalings while the
+ *       result stays normal).
+ * The truncation error of the degree-7 polynomial on |r| <= 0.35 is below
+ * 1e-8 relative, so E is within a few ulp of e^x.                           */
+static const float ORC_LOG2E = 1.44269502162933349609375f;     /* log2(e) rounded to fp32 */
+static const float ORC_LN2_HI = 0.693145751953125f;            /* 0x3F317200 */
+static const float ORC_LN2_LO = 1.428606765330187045037746429443359375e-06f;
+
+static float pow2i(int e) { /* exact 2^e for -126 <= e <= 127 */
+  uint32_t bits = (uint32_t)(e + 127) << 23;
+  float f;
+  memcpy(&f, &bits, sizeof(f));
+  return f;
+}
+
+float orc_exp(float x) {
+  x = fminf(fmaxf(x, -104.0f), 89.0f);
+  float nf = rintf(x * ORC_LOG2E);
+  int n = (int)nf;
+  float r = fmaf(-nf, ORC_LN2_HI, x);
+  r = fmaf(-nf, ORC_LN2_LO, r);
+  float p = 1.0f / 5040.0f;
+  p = fmaf(p, r, 1.0f / 720.0f);
+  p = fmaf(p, r, 1.0f / 120.0f);
+  p = fmaf(p, r, 1.0f / 24.0f);
+  p = fmaf(p, r, 1.0f / 6.0f);
+  p = fmaf(p, r, 0.5f);
+  p = fmaf(p, r, 1.0f);
+  p = fmaf(p, r, 1.0f);
+  int n1 = n / 2, n2 = n - n1;
+  return (p * pow2i(n1)) * pow2i(n2);
+}
+
+float orc_silu(float a) { return a / (1.0f + orc_exp(-a)); }
+
+void orc_swiglu(const float* gate, const float* up, int64_t n, float* h) {
+  for (int64_t i = 0; i < n; i++) h[i] = orc_silu(gate[i]) * up[i];
+}
+
 /* ------------------------------------------------------------------ mask --
  * Top-N by magnitude per group of M consecutive K elements; ties go to the
  * lower index.  For the 4:8 pair pattern the unit is an adjacent pair (2p,
