@@ -34,7 +34,8 @@ __host__ __device__ __forceinline__ int64_t tiled_sf_bytes(int64_t rows, int64_t
 }
 
 struct PrepParams {
-  const void* x;
+  const void* x;     // activations (SwiGLU form: the gate input)
+  const void* x2;    // SwiGLU form: the up input (same layout and dtype as x); else null
   const void* gamma;
   float eps;
   int64_t t, t_pad, k;
@@ -87,6 +88,45 @@ __device__ __forceinline__ void unpack_bf16_unit(const uint4 (&w4)[4], float (&v
       v[8 * q + 2 * j + 1] = __uint_as_float(ws[j] & 0xFFFF0000u);
     }
   }
+}
+
+// --------------------------------------------------------------- SwiGLU
+// h = SiLU(gate) * up with SiLU(a) = a / (1 + E(-a)), every step a single
+// IEEE round-to-nearest fp32 operation.  E is this project's exponential:
+// Cody and Waite's range reduction by ln 2 (split in two fp32 constants) and
+// the degree-7 Taylor polynomial evaluated by Horner with fused multiply-adds,
+// then an exact scaling by 2^n in two halves; the input is clamped to
+// [-104, 89], beyond which e^x is 0 or infinite in fp32 anyway.
+__device__ __forceinline__ float pow2i_dev(int e) {  // exact 2^e, -126 <= e <= 127
+  return __int_as_float((e + 127) << 23);
+}
+__device__ __forceinline__ float dev_exp(float x) {
+  x = fminf(fmaxf(x, -104.0f), 89.0f);
+  const float nf = rintf(__fmul_rn(x, 1.44269502162933349609375f));  // log2(e) rounded to fp32
+  const int n = (int)nf;
+  float r = __fmaf_rn(-nf, 0.693145751953125f, x);                   // ln 2, high 15 bits
+  r = __fmaf_rn(-nf, 1.428606765330187045037746429443359375e-06f, r);  // ln 2 - high part, rounded
+  float p = 1.0f / 5040.0f;
+  p = __fmaf_rn(p, r, 1.0f / 720.0f);
+  p = __fmaf_rn(p, r, 1.0f / 120.0f);
+  p = __fmaf_rn(p, r, 1.0f / 24.0f);
+  p = __fmaf_rn(p, r, 1.0f / 6.0f);
+  p = __fmaf_rn(p, r, 0.5f);
+  p = __fmaf_rn(p, r, 1.0f);
+  p = __fmaf_rn(p, r, 1.0f);
+  const int n1 = n / 2, n2 = n - n1;
+  return __fmul_rn(__fmul_rn(p, pow2i_dev(n1)), pow2i_dev(n2));
+}
+__device__ __forceinline__ float dev_silu(float a) { return __fdiv_rn(a, __fadd_rn(1.0f, dev_exp(-a))); }
+
+// h of one unit in the SwiGLU form.
+template <bool XBF16>
+__device__ __forceinline__ void swiglu_unit(const void* gate, const void* up, int64_t off, float (&h)[32]) {
+  float a[32], b[32];
+  load_unit<XBF16>(gate, off, a);
+  load_unit<XBF16>(up, off, b);
+#pragma unroll
+  for (int i = 0; i < 32; i++) h[i] = __fmul_rn(dev_silu(a[i]), b[i]);
 }
 
 // Two E2M1 codes (low nibble = first element) -> exact fp32 values.
@@ -362,9 +402,10 @@ __device__ __forceinline__ void sub2(float& a, float& b, float c, float d) {  //
 // ------------------------------------------------------------ stats kernel
 // Per row: rstd (RMSNorm) into rstd_out (if non-null) and max |h| folded into
 // amax_out[0] (zeroed beforehand) with one atomic per block.
-template <bool NORM, bool XBF16>
+template <bool NORM, bool XBF16, bool ACT = false>
 __global__ void __launch_bounds__(128) amax_kernel(const void* x, const void* gamma, float eps, int64_t t, int64_t k,
-                                                   float* amax_out, float* rstd_out) {
+                                                   float* amax_out, float* rstd_out, const void* x2 = nullptr) {
+  static_assert(!(NORM && ACT), "the SwiGLU form has no RMSNorm");
   __shared__ float red[32 * 16];
   __shared__ float wmax[4];
   const RowMap m = row_map(k);
@@ -384,7 +425,8 @@ __global__ void __launch_bounds__(128) amax_kernel(const void* x, const void* ga
       const int u = tt + m.tpr * j;
       if (!real || u >= m.units) continue;
       float v[32];
-      load_unit<XBF16>(x, off + (int64_t)u * 32, v);
+      if constexpr (ACT) swiglu_unit<XBF16>(x, x2, off + (int64_t)u * 32, v);
+      else load_unit<XBF16>(x, off + (int64_t)u * 32, v);
       if constexpr (NORM) {
         float g[32];
         load_unit<XBF16>(gamma, (int64_t)u * 32, g);
@@ -681,8 +723,9 @@ __device__ __forceinline__ void quantize_unit(float (&h)[32], float c6, float g_
   }
 }
 
-template <int FMT, int PAT, bool NORM, bool XBF16>
+template <int FMT, int PAT, bool NORM, bool XBF16, bool ACT = false>
 __global__ void __launch_bounds__(128, 6) prep_kernel(PrepParams p) {
+  static_assert(!(NORM && ACT), "the SwiGLU form has no RMSNorm");
   __shared__ float inv_tab[128];
   __shared__ float red[32 * 16];
   const int64_t k = p.k;
@@ -727,7 +770,8 @@ __global__ void __launch_bounds__(128, 6) prep_kernel(PrepParams p) {
       const bool active = u < m.units;
       float h[32];
       if (real && active) {
-        load_unit<XBF16>(p.x, off + (int64_t)u * 32, h);
+        if constexpr (ACT) swiglu_unit<XBF16>(p.x, p.x2, off + (int64_t)u * 32, h);
+        else load_unit<XBF16>(p.x, off + (int64_t)u * 32, h);
         if constexpr (NORM) {
           float g[32];
           load_unit<XBF16>(p.gamma, (int64_t)u * 32, g);

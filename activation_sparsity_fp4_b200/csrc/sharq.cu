@@ -170,7 +170,7 @@ sharq_status launch_amax(const void* x, const void* gamma, float eps, int64_t t,
     return launched();
   }
   auto kern = amax_kernel<NORM, XBF16>;
-  kern<<<row_grid(kern, t, k), 128, 0, s>>>(x, gamma, eps, t, k, out, rstd_out);
+  kern<<<row_grid(kern, t, k), 128, 0, s>>>(x, gamma, eps, t, k, out, rstd_out, nullptr);
   return launched();
 }
 
@@ -189,6 +189,32 @@ sharq_status prep_dispatch_p(const PrepParams& pp, int pat, bool norm, bool xbf1
     case PAT_48P: return prep_dispatch_n<FMT, PAT_48P>(pp, norm, xbf16, s);
     default: return prep_dispatch_n<FMT, PAT_816>(pp, norm, xbf16, s);
   }
+}
+
+// SwiGLU form (no RMSNorm): h = SiLU(x) * x2 inside the prep and amax kernels.
+template <int FMT, int PAT, bool XBF16>
+sharq_status launch_prep_swiglu(const PrepParams& pp, cudaStream_t s) {
+  auto kern = prep_kernel<FMT, PAT, false, XBF16, true>;
+  kern<<<row_grid(kern, pp.t_pad, pp.k), 128, 0, s>>>(pp);
+  return launched();
+}
+template <int FMT, int PAT>
+sharq_status swiglu_dispatch_x(const PrepParams& pp, bool xbf16, cudaStream_t s) {
+  return xbf16 ? launch_prep_swiglu<FMT, PAT, true>(pp, s) : launch_prep_swiglu<FMT, PAT, false>(pp, s);
+}
+template <int FMT>
+sharq_status swiglu_dispatch_p(const PrepParams& pp, int pat, bool xbf16, cudaStream_t s) {
+  switch (pat) {
+    case PAT_24: return swiglu_dispatch_x<FMT, PAT_24>(pp, xbf16, s);
+    case PAT_48P: return swiglu_dispatch_x<FMT, PAT_48P>(pp, xbf16, s);
+    default: return swiglu_dispatch_x<FMT, PAT_816>(pp, xbf16, s);
+  }
+}
+template <bool XBF16>
+sharq_status launch_amax_swiglu(const void* gate, const void* up, int64_t t, int64_t k, float* out, cudaStream_t s) {
+  auto kern = amax_kernel<false, XBF16, true>;
+  kern<<<row_grid(kern, t, k), 128, 0, s>>>(gate, nullptr, 0.0f, t, k, out, nullptr, up);
+  return launched();
 }
 
 template <int KIND, bool SPARSE>
@@ -465,6 +491,7 @@ sharq_status sharq_prepare(const void* x, sharq_dtype x_dt, const void* gamma, f
   const bool bf16 = x_dt == SHARQ_BF16, norm = gamma != nullptr;
   PrepParams pp;
   pp.x = x;
+  pp.x2 = nullptr;
   pp.gamma = gamma;
   pp.eps = eps;
   pp.t = out->t;
@@ -493,6 +520,41 @@ sharq_status sharq_prepare(const void* x, sharq_dtype x_dt, const void* gamma, f
   }
   if (out->fmt == SHARQ_NVFP4) return prep_dispatch_p<FMT_NV>(pp, out->pat, norm, bf16, s);
   return prep_dispatch_p<FMT_MX>(pp, out->pat, norm, bf16, s);
+}
+
+sharq_status sharq_prepare_swiglu(const void* gate, const void* up, sharq_dtype dt, float act_amax,
+                                  sharq_prepared* out, sharq_stream stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  sharq_status st = check_prepared(out);
+  if (st != SHARQ_OK) return st;
+  if (!gate || !aligned(gate, 16)) return fail(SHARQ_ERR_INVALID, "gate must be a 16-byte aligned device pointer");
+  if (!up || !aligned(up, 16)) return fail(SHARQ_ERR_INVALID, "up must be a 16-byte aligned device pointer");
+  if (dt != SHARQ_F32 && dt != SHARQ_BF16) return fail(SHARQ_ERR_INVALID, "bad dtype %d", (int)dt);
+  const bool bf16 = dt == SHARQ_BF16;
+  PrepParams pp;
+  pp.x = gate;
+  pp.x2 = up;
+  pp.gamma = nullptr;
+  pp.eps = 0.0f;
+  pp.t = out->t;
+  pp.t_pad = round_up(out->t, 128);
+  pp.k = out->k;
+  pp.meta = static_cast<uint8_t*>(out->meta);
+  pp.bb_codes = static_cast<uint8_t*>(out->bb_codes);
+  pp.bb_scales = static_cast<uint8_t*>(out->bb_scales);
+  pp.res_codes = static_cast<uint8_t*>(out->res_codes);
+  pp.res_scales = static_cast<uint8_t*>(out->res_scales);
+  pp.tensor = out->tensor;
+  pp.act_amax = act_amax > 0.0f ? act_amax : 0.0f;
+  pp.rstd = nullptr;
+  if (out->fmt == SHARQ_NVFP4 && !(act_amax > 0.0f)) {
+    SHARQ_CUDA(cudaMemsetAsync(out->tensor, 0, sizeof(float), s));
+    st = bf16 ? launch_amax_swiglu<true>(gate, up, out->t, out->k, out->tensor, s)
+              : launch_amax_swiglu<false>(gate, up, out->t, out->k, out->tensor, s);
+    if (st != SHARQ_OK) return st;
+  }
+  if (out->fmt == SHARQ_NVFP4) return swiglu_dispatch_p<FMT_NV>(pp, out->pat, bf16, s);
+  return swiglu_dispatch_p<FMT_MX>(pp, out->pat, bf16, s);
 }
 
 sharq_status sharq_prepare_noalloc(const void* x, sharq_dtype x_dt, const void* gamma, float eps, float act_amax,

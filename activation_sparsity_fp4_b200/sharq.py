@@ -24,7 +24,7 @@ STATUS = {0: "SHARQ_OK", 1: "SHARQ_ERR_INVALID", 2: "SHARQ_ERR_UNSUPPORTED", 3: 
           4: "SHARQ_ERR_TIMEOUT", 5: "SHARQ_ERR_WORKSPACE"}
 SYMBOLS = ["sharq_weight_sizes", "sharq_prepared_sizes", "sharq_quantize_weight", "sharq_prepare", "sharq_linear",
            "sharq_linear_paths", "sharq_linear_grouped", "sharq_sync_status", "sharq_selftest_wait_timeout",
-           "sharq_last_error", "sharq_launch_count", "sharq_prepare_noalloc"]
+           "sharq_last_error", "sharq_launch_count", "sharq_prepare_noalloc", "sharq_prepare_swiglu"]
 NOALLOC_MAX_ROWS = 65536  # SHARQ_NOALLOC_MAX_ROWS of the C header
 
 
@@ -70,6 +70,7 @@ def lib() -> ctypes.CDLL:
             "sharq_quantize_weight": [P, I, ctypes.POINTER(sharq_weight), P],
             "sharq_prepare": [P, I, P, F, F, ctypes.POINTER(sharq_prepared), P, ctypes.c_size_t, P],
             "sharq_prepare_noalloc": [P, I, P, F, F, ctypes.POINTER(sharq_prepared), P],
+            "sharq_prepare_swiglu": [P, P, I, F, ctypes.POINTER(sharq_prepared), P],
             "sharq_linear": [ctypes.POINTER(sharq_prepared), ctypes.POINTER(sharq_weight), P, I, P],
             "sharq_linear_paths": [ctypes.POINTER(sharq_prepared), ctypes.POINTER(sharq_weight), P, I, I32, P],
             "sharq_linear_grouped": [ctypes.POINTER(sharq_prepared), ctypes.POINTER(sharq_weight), P, P, I, P],
@@ -152,6 +153,11 @@ def sharq_prepare_noalloc(x_ptr: int, x_dt, gamma_ptr, eps: float, act_amax: flo
     _check(lib().sharq_prepare_noalloc(ctypes.c_void_p(x_ptr), _dt(x_dt),
                                        ctypes.c_void_p(gamma_ptr) if gamma_ptr else None, float(eps), float(act_amax),
                                        ctypes.byref(out), _stream(stream)), "sharq_prepare_noalloc")
+
+
+def sharq_prepare_swiglu(gate_ptr: int, up_ptr: int, dt, act_amax: float, out: sharq_prepared, stream=None):
+    _check(lib().sharq_prepare_swiglu(ctypes.c_void_p(gate_ptr), ctypes.c_void_p(up_ptr), _dt(dt), float(act_amax),
+                                      ctypes.byref(out), _stream(stream)), "sharq_prepare_swiglu")
 
 
 def sharq_linear(a: sharq_prepared, w: sharq_weight, y_ptr: int, y_dt, stream=None):
@@ -247,6 +253,18 @@ def prepare(x: torch.Tensor, fmt, pat, gamma: torch.Tensor | None = None, eps: f
     ws = out.workspace if use_workspace else None
     sharq_prepare(x.data_ptr(), x.dtype, gamma.data_ptr() if gamma is not None else None, eps, act_amax, out.struct,
                   ws.data_ptr() if ws is not None else None, ws.numel() if ws is not None else 0, stream)
+    return out
+
+
+def prepare_swiglu(gate: torch.Tensor, up: torch.Tensor, fmt, pat, act_amax: float = 0.0,
+                   out: Prepared | None = None, stream=None) -> Prepared:
+    """Preprocessing of h = SiLU(gate) * up (t, k), formed inside the kernel."""
+    gate, up = gate.contiguous(), up.to(gate.dtype).contiguous()
+    assert gate.shape == up.shape
+    t, k = gate.shape
+    if out is None:
+        out = Prepared(t, k, fmt, pat, gate.device)
+    sharq_prepare_swiglu(gate.data_ptr(), up.data_ptr(), gate.dtype, act_amax, out.struct, stream)
     return out
 
 

@@ -17,7 +17,8 @@ them by shape and value distribution only:
                  entries of a seeded permutation of K); RMSNorm gamma ~U(0.5, 1.5) bf16, eps 1e-6;
                  W 4096x4096 ~N(0, 0.02^2); NVFP4, 4:8 pair.
 * ``down_proj``  X T x 14336 bf16 = SiLU(a) * b with a, b ~N(0,1) (computed in fp32);
-                 W 4096x14336 ~N(0, 0.01^2); MXFP4, 2:4; T in {1, 16, 64, 256, 2048}.
+                 W 4096x14336 ~N(0, 0.01^2); MXFP4, 2:4; T in {1, 16, 64, 256, 2048}; also
+                 gate = a and up = b rounded to bf16, the inputs of the SwiGLU form.
 * ``wan``        X 32768x5120 bf16 ~N(0,1), 16 outlier channels x50; RMSNorm gamma ~U(0.5, 1.5);
                  W 5120x5120 ~N(0, 0.02^2); NVFP4, 4:8 pair (and 8:16).
 * ``qwen_moe``   4096 tokens, hidden 2048, 0.5 * Student-t(3) bf16; router logits 4096x128 ~N(0,1),
@@ -75,8 +76,10 @@ def down_proj(seed: int = SEED, t: int = 2048) -> dict:
     x = (a / (np.float32(1.0) + np.exp(-a))) * b
     x = to_bf16_values(x.astype(np.float32))
     w = to_bf16_values(rng.standard_normal((n, k), dtype=np.float32) * np.float32(0.01))
+    # the gate and up projections as a bf16 model hands them over, for the form of the
+    # preprocessing that builds the down projection's input itself
     return dict(name="down_proj", x=x, x_dtype="bf16", gamma=None, eps=1e-6, w=w, w_dtype="bf16",
-                fmt="mxfp4", pat="2:4")
+                fmt="mxfp4", pat="2:4", gate=to_bf16_values(a), up=to_bf16_values(b))
 
 
 def wan(seed: int = SEED, t: int = 32768, pat: str = "4:8pair") -> dict:

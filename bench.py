@@ -45,6 +45,8 @@ WORKLOADS = {
            "NVFP4, 4:8 pair",
     "wan_816": "Wan2.2-14B DiT linear: X 32768x5120 bf16 ~N(0,1) + 16 outlier channels x50, RMSNorm; W 5120x5120; "
                "NVFP4, 8:16",
+    "down_proj_swiglu": "Llama-3.1-8B down_proj from its gate and up inputs: gate, up 2048x14336 bf16 ~N(0,1), "
+                        "h = SiLU(gate)*up formed inside the prep kernel; W 4096x14336 ~N(0,0.01^2); MXFP4, 2:4",
     "qwen_moe_gate_up": "Qwen3-30B-A3B MoE gate/up: 4096 tokens top-8 of 128 experts -> 32768 routed rows (each expert "
                         "padded to 128 rows), hidden 2048; per expert W 1536x2048; NVFP4, 4:8 pair, no norm; grouped",
 }
@@ -69,13 +71,16 @@ def make_workload(name: str) -> dict:
         n = c["w_gu"].shape[1]
         return dict(name=name, desc=WORKLOADS[name], x=c["x"], gamma=None, eps=1e-6, w=c["w_gu"], fmt="nvfp4",
                     pat="4:8pair", offsets=c["offsets"], t=t, k=k, n=n, real_rows=int(c["counts"].sum()),
-                    first_group=(int(c["offsets"][0]), int(c["offsets"][1])))
-    c = {"q_proj": workloads.q_proj, "down_proj": workloads.down_proj, "wan": workloads.wan,
-         "wan_816": lambda: workloads.wan(pat="8:16")}[name]()
+                    first_group=(int(c["offsets"][0]), int(c["offsets"][1])), gate=None, up=None)
+    c = {"q_proj": workloads.q_proj, "down_proj": workloads.down_proj, "down_proj_swiglu": workloads.down_proj,
+         "wan": workloads.wan, "wan_816": lambda: workloads.wan(pat="8:16")}[name]()
     t, k = c["x"].shape
-    return dict(name=name, desc=WORKLOADS[name], x=c["x"], gamma=c["gamma"], eps=c["eps"], w=c["w"],
-                fmt=c["fmt"], pat=c["pat"], offsets=None, t=t, k=k, n=c["w"].shape[0], real_rows=t,
-                first_group=None)
+    wl = dict(name=name, desc=WORKLOADS[name], x=c["x"], gamma=c["gamma"], eps=c["eps"], w=c["w"],
+              fmt=c["fmt"], pat=c["pat"], offsets=None, t=t, k=k, n=c["w"].shape[0], real_rows=t,
+              first_group=None, gate=None, up=None)
+    if name == "down_proj_swiglu":
+        wl.update(x=None, gate=c["gate"], up=c["up"])
+    return wl
 
 
 def gemm_roofline(wl: dict):
@@ -223,9 +228,12 @@ def cpu_baseline(name: str = "q_proj", rows: int = 2048):
     rows = min(rows, (wl["first_group"][1] - r0) if wl["first_group"] else wl["t"])
     cores = len(os.sched_getaffinity(0))
     t0 = time.perf_counter()
-    amax = oracle.rows_amax(x, wl["gamma"], wl["eps"]) if wl["fmt"] == "nvfp4" else 0.0
-    prep = oracle.prepare(x[r0:r0 + rows], wl["fmt"], wl["pat"], gamma=wl["gamma"], eps=wl["eps"], act_amax=amax,
-                          threads=cores)
+    if wl["gate"] is not None:  # SwiGLU form (MXFP4: no tensor amax)
+        prep = oracle.prepare_swiglu(wl["gate"][:rows], wl["up"][:rows], wl["fmt"], wl["pat"], threads=cores)
+    else:
+        amax = oracle.rows_amax(x, wl["gamma"], wl["eps"]) if wl["fmt"] == "nvfp4" else 0.0
+        prep = oracle.prepare(x[r0:r0 + rows], wl["fmt"], wl["pat"], gamma=wl["gamma"], eps=wl["eps"],
+                              act_amax=amax, threads=cores)
     y = oracle.linear_ref(prep, wq, wu=wu)
     dt = time.perf_counter() - t0
     assert np.isfinite(y).all()
@@ -255,8 +263,11 @@ def run_sharq(args):
 
     wl = make_workload(args.workload)
     T, K, N, fmt, pat = wl["t"], wl["k"], wl["n"], wl["fmt"], wl["pat"]
-    x_host = torch.from_numpy(wl["x"]).to(torch.bfloat16).pin_memory()
+    swiglu = wl["gate"] is not None
+    x_host = torch.from_numpy(wl["gate"] if swiglu else wl["x"]).to(torch.bfloat16).pin_memory()
     x = x_host.to(dev)
+    up_host = torch.from_numpy(wl["up"]).to(torch.bfloat16).pin_memory() if swiglu else None
+    up = up_host.to(dev) if swiglu else None
     gamma = torch.from_numpy(wl["gamma"]).to(torch.bfloat16).to(dev) if wl["gamma"] is not None else None
     w = torch.from_numpy(wl["w"]).to(torch.bfloat16).to(dev)
     wq = sharq.FP4Weight.quantize(w, fmt)
@@ -270,7 +281,10 @@ def run_sharq(args):
     sharq.sharq_sync_status()
 
     def do_prep(act_amax=0.0):
-        sharq.prepare(x, fmt, pat, gamma, wl["eps"], act_amax=act_amax, out=prep)
+        if swiglu:
+            sharq.prepare_swiglu(x, up, fmt, pat, act_amax=act_amax, out=prep)
+        else:
+            sharq.prepare(x, fmt, pat, gamma, wl["eps"], act_amax=act_amax, out=prep)
 
     def do_gemm():
         if offsets is None:
@@ -343,6 +357,8 @@ def run_sharq(args):
         flush.fill_(1)
         eev[i][0].record(stream)
         x.copy_(x_host, non_blocking=True)
+        if swiglu:
+            up.copy_(up_host, non_blocking=True)
         step()
         y_host.copy_(y, non_blocking=True)
         eev[i][1].record(stream)
@@ -364,7 +380,7 @@ def run_sharq(args):
         ratio = FP4_OVER_BF16 if kind == "fp4" else FP8_OVER_BF16
         peak = pk["bf16_tflops"] * ratio
         achieved = work / gemm_avg / 1e12
-        bpe = prep_bytes_per_elem(fmt, pat)
+        bpe = prep_bytes_per_elem(fmt, pat, 4 if swiglu else 2)
         prep_bytes = bpe * T * K
         prep_gbs = prep_bytes / (statistics.mean(prep_ms) / 1e3) / 1e9
         prep_given_gbs = prep_bytes / (prep_given_ms / 1e3) / 1e9
@@ -403,7 +419,8 @@ def run_sharq(args):
                      "bytes_per_elem": bpe, "avg_us": round(statistics.mean(prep_ms) * 1e3, 2),
                      "avg_us_given_amax": round(prep_given_ms * 1e3, 2)},
             "e2e": {"value": round(world * flops * args.steps / (e2e_ms / 1e3) / 1e12, 3), "unit": "TFLOP/s",
-                    "h2d_bytes_per_step": int(x_host.numel() * 2), "d2h_bytes_per_step": int(y_host.numel() * 2)},
+                    "h2d_bytes_per_step": int(x_host.numel() * 2 * (2 if swiglu else 1)),
+                    "d2h_bytes_per_step": int(y_host.numel() * 2)},
             "gpu_launches": int(launches),
             "launch_mode": "CUDA graphs (prep graph + GEMM graph per step); e2e uses direct API calls",
             "clocks": clocks,

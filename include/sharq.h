@@ -143,6 +143,20 @@ sharq_status sharq_quantize_weight(const void* w, sharq_dtype w_dt, sharq_weight
 sharq_status sharq_prepare(const void* x, sharq_dtype x_dt, const void* gamma, float eps, float act_amax,
                            sharq_prepared* out, void* workspace, size_t workspace_bytes, sharq_stream stream);
 
+/* Fused preprocessing of a down projection's input formed on the fly from a gated
+ * MLP: h = SiLU(gate) * up, then the mask, backbone and residual of sharq_prepare (no
+ * RMSNorm).  The SharQ abstract fuses the layer norm into the preprocessing op; this
+ * extends the same fusion to the activation in front of the down projection, so h is
+ * never written to or read from memory.  In fp32, each step rounded once:
+ *   SiLU(a) = a / (1 + E(-a)),  h = SiLU(a) * b,
+ * where E is the library's exponential: reduction by ln 2 in two fp32 steps (Cody and
+ * Waite), the degree-7 Taylor polynomial by Horner with fused multiply-adds, exact
+ * scaling by 2^n; inputs clamped to [-104, 89]; within one ulp of e^x.
+ * gate, up: t * k row-major values of dtype dt (DEVICE).  act_amax as in sharq_prepare
+ * (<= 0: the NVFP4 tensor amax of h is computed on the device).  out: as sharq_prepare. */
+sharq_status sharq_prepare_swiglu(const void* gate, const void* up, sharq_dtype dt, float act_amax,
+                                  sharq_prepared* out, sharq_stream stream);
+
 /* Largest t that sharq_prepare_noalloc accepts (its static scratch holds one float per row). */
 #define SHARQ_NOALLOC_MAX_ROWS 65536
 
