@@ -819,6 +819,53 @@ __global__ void __launch_bounds__(128, 6) prep_kernel(PrepParams p) {
   }
 }
 
+// --------------------------------------------------------- row gather
+// Prepared activations laid out again by row: destination row r takes source
+// row rows[r] (r < t) -- metadata, backbone and residual codes as contiguous
+// row segments (16-byte copies), the tiled scales as 32-bit words of four
+// scales -- or, for rows[r] < 0 and for the padding rows t..t_pad-1, the
+// encoding of an all-zero input row: no element beats another, so the mask
+// keeps the first N of every group (nibble i0 | i1 << 2 = 4 for 2:4 and the
+// 4:8 pair, mask 0x00FF for 8:16), and every code and scale is 0.
+struct GatherParams {
+  const uint8_t *s_meta, *s_bbc, *s_bbs, *s_rc, *s_rs;
+  uint8_t *d_meta, *d_bbc, *d_bbs, *d_rc, *d_rs;
+  const int32_t* rows;
+  int64_t src_t, t, t_pad;
+  int64_t meta_row, bbc_row, rc_row;  // bytes per row
+  int64_t bbs_per_row, rs_per_row;    // scales per row (multiples of 4)
+  uint32_t zero_meta;                 // 4 bytes of the zero row's metadata
+};
+
+__global__ void __launch_bounds__(256) gather_rows_kernel(const GatherParams p) {
+  const int lane = threadIdx.x & 31;
+  const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (r >= p.t_pad) return;
+  int64_t src = r < p.t ? (int64_t)__ldg(p.rows + r) : -1;
+  if (src >= p.src_t) src = -1;  // out of range: treated as a zero row (the host checks nothing on the device data)
+  auto seg = [&](const uint8_t* sb, uint8_t* db, int64_t row_bytes, uint32_t fill) {
+    uint4* d = reinterpret_cast<uint4*>(db + r * row_bytes);
+    const int64_t n = row_bytes / 16;
+    if (src >= 0) {
+      const uint4* s4 = reinterpret_cast<const uint4*>(sb + src * row_bytes);
+      for (int64_t i = lane; i < n; i += 32) d[i] = __ldg(s4 + i);
+    } else {
+      for (int64_t i = lane; i < n; i += 32) d[i] = make_uint4(fill, fill, fill, fill);
+    }
+  };
+  seg(p.s_meta, p.d_meta, p.meta_row, p.zero_meta);
+  seg(p.s_bbc, p.d_bbc, p.bbc_row, 0u);
+  seg(p.s_rc, p.d_rc, p.rc_row, 0u);
+  auto scales = [&](const uint8_t* sb, uint8_t* db, int64_t per_row) {
+    for (int64_t s4 = lane; s4 < per_row / 4; s4 += 32) {
+      const uint32_t v = src >= 0 ? __ldg(reinterpret_cast<const uint32_t*>(sb + tiled_sf_offset(src, 4 * s4, per_row))) : 0u;
+      *reinterpret_cast<uint32_t*>(db + tiled_sf_offset(r, 4 * s4, per_row)) = v;
+    }
+  };
+  scales(p.s_bbs, p.d_bbs, p.bbs_per_row);
+  scales(p.s_rs, p.d_rs, p.rs_per_row);
+}
+
 // --------------------------------------------------------- weight kernel
 // One thread quantizes 32 consecutive K values of a weight row; a scale block
 // is 2b logical K (NVFP4: this unit; MXFP4: the unit and its neighbour lane).

@@ -557,6 +557,47 @@ sharq_status sharq_prepare_swiglu(const void* gate, const void* up, sharq_dtype 
   return swiglu_dispatch_p<FMT_MX>(pp, out->pat, bf16, s);
 }
 
+sharq_status sharq_gather_prepared(const sharq_prepared* src, const int32_t* rows, sharq_prepared* dst,
+                                   sharq_stream stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  sharq_status st = check_prepared(src);
+  if (st != SHARQ_OK) return st;
+  st = check_prepared(dst);
+  if (st != SHARQ_OK) return st;
+  if (src->k != dst->k || src->fmt != dst->fmt || src->pat != dst->pat)
+    return fail(SHARQ_ERR_INVALID, "source and destination differ in k, format or pattern");
+  if (dst->t > 0 && (!rows || !aligned(rows, 4))) return fail(SHARQ_ERR_INVALID, "rows must be a device int32 array");
+  const int64_t k = dst->k;
+  const int b = fmt_block(dst->fmt);
+  const bool d816 = dst->pat == SHARQ_NM_8_16;
+  GatherParams gp;
+  gp.s_meta = static_cast<const uint8_t*>(src->meta);
+  gp.s_bbc = static_cast<const uint8_t*>(src->bb_codes);
+  gp.s_bbs = static_cast<const uint8_t*>(src->bb_scales);
+  gp.s_rc = static_cast<const uint8_t*>(src->res_codes);
+  gp.s_rs = static_cast<const uint8_t*>(src->res_scales);
+  gp.d_meta = static_cast<uint8_t*>(dst->meta);
+  gp.d_bbc = static_cast<uint8_t*>(dst->bb_codes);
+  gp.d_bbs = static_cast<uint8_t*>(dst->bb_scales);
+  gp.d_rc = static_cast<uint8_t*>(dst->res_codes);
+  gp.d_rs = static_cast<uint8_t*>(dst->res_scales);
+  gp.rows = rows;
+  gp.src_t = src->t;
+  gp.t = dst->t;
+  gp.t_pad = round_up(dst->t, 128);
+  gp.meta_row = meta_row_bytes(k, dst->pat);
+  gp.bbc_row = d816 ? k / 2 : k / 4;
+  gp.rc_row = k / 2;
+  gp.bbs_per_row = d816 ? k / b : k / (2 * b);
+  gp.rs_per_row = k / b;
+  gp.zero_meta = d816 ? 0x00FF00FFu : 0x44444444u;
+  gather_rows_kernel<<<(unsigned)((gp.t_pad + 7) / 8), 256, 0, s>>>(gp);
+  st = launched();
+  if (st != SHARQ_OK) return st;
+  SHARQ_CUDA(cudaMemcpyAsync(dst->tensor, src->tensor, 3 * sizeof(float), cudaMemcpyDeviceToDevice, s));
+  return SHARQ_OK;
+}
+
 sharq_status sharq_prepare_noalloc(const void* x, sharq_dtype x_dt, const void* gamma, float eps, float act_amax,
                                    sharq_prepared* out, sharq_stream stream) {
   if (!out) return fail(SHARQ_ERR_INVALID, "out is NULL");

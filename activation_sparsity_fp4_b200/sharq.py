@@ -24,7 +24,8 @@ STATUS = {0: "SHARQ_OK", 1: "SHARQ_ERR_INVALID", 2: "SHARQ_ERR_UNSUPPORTED", 3: 
           4: "SHARQ_ERR_TIMEOUT", 5: "SHARQ_ERR_WORKSPACE"}
 SYMBOLS = ["sharq_weight_sizes", "sharq_prepared_sizes", "sharq_quantize_weight", "sharq_prepare", "sharq_linear",
            "sharq_linear_paths", "sharq_linear_grouped", "sharq_sync_status", "sharq_selftest_wait_timeout",
-           "sharq_last_error", "sharq_launch_count", "sharq_prepare_noalloc", "sharq_prepare_swiglu"]
+           "sharq_last_error", "sharq_launch_count", "sharq_prepare_noalloc", "sharq_prepare_swiglu",
+           "sharq_gather_prepared"]
 NOALLOC_MAX_ROWS = 65536  # SHARQ_NOALLOC_MAX_ROWS of the C header
 
 
@@ -71,6 +72,7 @@ def lib() -> ctypes.CDLL:
             "sharq_prepare": [P, I, P, F, F, ctypes.POINTER(sharq_prepared), P, ctypes.c_size_t, P],
             "sharq_prepare_noalloc": [P, I, P, F, F, ctypes.POINTER(sharq_prepared), P],
             "sharq_prepare_swiglu": [P, P, I, F, ctypes.POINTER(sharq_prepared), P],
+            "sharq_gather_prepared": [ctypes.POINTER(sharq_prepared), P, ctypes.POINTER(sharq_prepared), P],
             "sharq_linear": [ctypes.POINTER(sharq_prepared), ctypes.POINTER(sharq_weight), P, I, P],
             "sharq_linear_paths": [ctypes.POINTER(sharq_prepared), ctypes.POINTER(sharq_weight), P, I, I32, P],
             "sharq_linear_grouped": [ctypes.POINTER(sharq_prepared), ctypes.POINTER(sharq_weight), P, P, I, P],
@@ -158,6 +160,11 @@ def sharq_prepare_noalloc(x_ptr: int, x_dt, gamma_ptr, eps: float, act_amax: flo
 def sharq_prepare_swiglu(gate_ptr: int, up_ptr: int, dt, act_amax: float, out: sharq_prepared, stream=None):
     _check(lib().sharq_prepare_swiglu(ctypes.c_void_p(gate_ptr), ctypes.c_void_p(up_ptr), _dt(dt), float(act_amax),
                                       ctypes.byref(out), _stream(stream)), "sharq_prepare_swiglu")
+
+
+def sharq_gather_prepared(src: sharq_prepared, rows_ptr: int, dst: sharq_prepared, stream=None):
+    _check(lib().sharq_gather_prepared(ctypes.byref(src), ctypes.c_void_p(rows_ptr), ctypes.byref(dst),
+                                       _stream(stream)), "sharq_gather_prepared")
 
 
 def sharq_linear(a: sharq_prepared, w: sharq_weight, y_ptr: int, y_dt, stream=None):
@@ -265,6 +272,16 @@ def prepare_swiglu(gate: torch.Tensor, up: torch.Tensor, fmt, pat, act_amax: flo
     if out is None:
         out = Prepared(t, k, fmt, pat, gate.device)
     sharq_prepare_swiglu(gate.data_ptr(), up.data_ptr(), gate.dtype, act_amax, out.struct, stream)
+    return out
+
+
+def gather_prepared(src: Prepared, rows: torch.Tensor, out: Prepared | None = None, stream=None) -> Prepared:
+    """Prepared rows laid out again: row i of the result is src row rows[i] (a zero row for
+    rows[i] < 0)."""
+    rows = rows.to(torch.int32).contiguous()
+    if out is None:
+        out = Prepared(rows.numel(), src.k, src.fmt, src.pat, src.meta.device)
+    sharq_gather_prepared(src.struct, rows.data_ptr(), out.struct, stream)
     return out
 
 

@@ -105,23 +105,31 @@ def route_top_k(logits: np.ndarray, top_k: int) -> np.ndarray:
     return order[:, :top_k]
 
 
+def expert_rows(experts: np.ndarray, n_experts: int, align: int = 128):
+    """Routed-row layout of a top-k assignment: each expert's rows contiguous, in token
+    order, padded to a multiple of align.  Returns (counts, offsets (n_experts+1),
+    gather = token index per routed row, -1 for a padding row)."""
+    counts = np.bincount(experts.ravel(), minlength=n_experts)
+    padded = ((counts + align - 1) // align) * align
+    offsets = np.zeros(n_experts + 1, np.int64)
+    offsets[1:] = np.cumsum(padded)
+    gather = np.full(int(offsets[-1]), -1, np.int64)
+    fill = offsets[:-1].copy()
+    for tok in range(experts.shape[0]):
+        for e in experts[tok]:
+            gather[fill[e]] = tok
+            fill[e] += 1
+    return counts, offsets, gather
+
+
 def qwen_moe(seed: int = SEED, tokens: int = 4096, n_experts: int = 128, top_k: int = 8,
              hidden: int = 2048, inter: int = 768, align: int = 128) -> dict:
     rng = np.random.default_rng(seed)
     x_tok = to_bf16_values((0.5 * rng.standard_t(3, size=(tokens, hidden))).astype(np.float32))
     logits = rng.standard_normal((tokens, n_experts))
     experts = route_top_k(logits, top_k)
-    counts = np.bincount(experts.ravel(), minlength=n_experts)
-    padded = ((counts + align - 1) // align) * align
-    offsets = np.zeros(n_experts + 1, np.int64)
-    offsets[1:] = np.cumsum(padded)
+    counts, offsets, gather = expert_rows(experts, n_experts, align)
     rows = int(offsets[-1])
-    gather = np.full(rows, -1, np.int64)  # token index per routed row, -1 = padding row
-    fill = offsets[:-1].copy()
-    for tok in range(tokens):
-        for e in experts[tok]:
-            gather[fill[e]] = tok
-            fill[e] += 1
     x_routed = np.zeros((rows, hidden), np.float32)
     valid = gather >= 0
     x_routed[valid] = x_tok[gather[valid]]
@@ -131,7 +139,7 @@ def qwen_moe(seed: int = SEED, tokens: int = 4096, n_experts: int = 128, top_k: 
     w_d = to_bf16_values(rng.standard_normal((n_experts, hidden, inter), dtype=np.float32) * np.float32(0.02))
     return dict(name="qwen_moe", x=x_routed, x_down=x_down, x_dtype="bf16", gamma=None, eps=1e-6,
                 w_gu=w_gu, w_d=w_d, w_dtype="bf16", fmt="nvfp4", pat="4:8pair", counts=counts,
-                offsets=offsets, gather=gather, n_experts=n_experts)
+                offsets=offsets, gather=gather, n_experts=n_experts, x_tok=x_tok)
 
 
 CONFIGS = {

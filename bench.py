@@ -8,7 +8,7 @@ W 4096 x 4096), synthetic seeded data.  The weight is quantized once, outside
 the timed region (it is an offline step of the layer).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sharq|reference]
-                  [--workload q_proj|down_proj|wan|wan_816|qwen_moe_gate_up]
+                  [--workload NAME]
 
 The default workload is q_proj; the others measure the remaining layer shapes
 the pages evaluate (one JSON line each, same keys).
@@ -49,6 +49,8 @@ WORKLOADS = {
                         "h = SiLU(gate)*up formed inside the prep kernel; W 4096x14336 ~N(0,0.01^2); MXFP4, 2:4",
     "qwen_moe_gate_up": "Qwen3-30B-A3B MoE gate/up: 4096 tokens top-8 of 128 experts -> 32768 routed rows (each expert "
                         "padded to 128 rows), hidden 2048; per expert W 1536x2048; NVFP4, 4:8 pair, no norm; grouped",
+    "qwen_moe_gate_up_gather": "Qwen3-30B-A3B MoE gate/up as qwen_moe_gate_up, but each of the 4096 tokens prepared "
+                               "once and its prepared row gathered into the 32768 routed rows; grouped",
 }
 
 
@@ -65,13 +67,16 @@ def prep_bytes_per_elem(fmt: str, pat: str, x_bytes: int = 2) -> float:
 def make_workload(name: str) -> dict:
     """Inputs and roofline terms of one bench workload (host arrays; nothing of the method here)."""
     from activation_sparsity_fp4_b200 import workloads
-    if name == "qwen_moe_gate_up":
+    if name in ("qwen_moe_gate_up", "qwen_moe_gate_up_gather"):
         c = workloads.qwen_moe()
         t, k = c["x"].shape
         n = c["w_gu"].shape[1]
-        return dict(name=name, desc=WORKLOADS[name], x=c["x"], gamma=None, eps=1e-6, w=c["w_gu"], fmt="nvfp4",
-                    pat="4:8pair", offsets=c["offsets"], t=t, k=k, n=n, real_rows=int(c["counts"].sum()),
-                    first_group=(int(c["offsets"][0]), int(c["offsets"][1])), gate=None, up=None)
+        wl = dict(name=name, desc=WORKLOADS[name], x=c["x"], gamma=None, eps=1e-6, w=c["w_gu"], fmt="nvfp4",
+                  pat="4:8pair", offsets=c["offsets"], t=t, k=k, n=n, real_rows=int(c["counts"].sum()),
+                  first_group=(int(c["offsets"][0]), int(c["offsets"][1])), gate=None, up=None)
+        if name.endswith("_gather"):
+            wl.update(tokens=c["x_tok"], gather=c["gather"])
+        return wl
     c = {"q_proj": workloads.q_proj, "down_proj": workloads.down_proj, "down_proj_swiglu": workloads.down_proj,
          "wan": workloads.wan, "wan_816": lambda: workloads.wan(pat="8:16")}[name]()
     t, k = c["x"].shape
@@ -264,7 +269,9 @@ def run_sharq(args):
     wl = make_workload(args.workload)
     T, K, N, fmt, pat = wl["t"], wl["k"], wl["n"], wl["fmt"], wl["pat"]
     swiglu = wl["gate"] is not None
-    x_host = torch.from_numpy(wl["gate"] if swiglu else wl["x"]).to(torch.bfloat16).pin_memory()
+    gathered = wl.get("gather") is not None  # prep of the tokens, then their prepared rows gathered
+    x_src = wl["gate"] if swiglu else (wl["tokens"] if gathered else wl["x"])
+    x_host = torch.from_numpy(x_src).to(torch.bfloat16).pin_memory()
     x = x_host.to(dev)
     up_host = torch.from_numpy(wl["up"]).to(torch.bfloat16).pin_memory() if swiglu else None
     up = up_host.to(dev) if swiglu else None
@@ -274,6 +281,10 @@ def run_sharq(args):
     del w
     offsets = torch.from_numpy(wl["offsets"]).to(torch.int32).to(dev) if wl["offsets"] is not None else None
     prep = sharq.Prepared(T, K, fmt, pat, dev)
+    if gathered:
+        rows_host = torch.from_numpy(wl["gather"]).to(torch.int32).pin_memory()
+        rows = rows_host.to(dev)
+        prep_tok = sharq.Prepared(x_host.shape[0], K, fmt, pat, dev)
     y = torch.zeros((T, N), dtype=torch.bfloat16, device=dev)
     y_host = torch.empty((T, N), dtype=torch.bfloat16).pin_memory()
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
@@ -283,6 +294,9 @@ def run_sharq(args):
     def do_prep(act_amax=0.0):
         if swiglu:
             sharq.prepare_swiglu(x, up, fmt, pat, act_amax=act_amax, out=prep)
+        elif gathered:
+            sharq.prepare(x, fmt, pat, gamma, wl["eps"], act_amax=act_amax, out=prep_tok)
+            sharq.gather_prepared(prep_tok, rows, out=prep)
         else:
             sharq.prepare(x, fmt, pat, gamma, wl["eps"], act_amax=act_amax, out=prep)
 
@@ -359,6 +373,8 @@ def run_sharq(args):
         x.copy_(x_host, non_blocking=True)
         if swiglu:
             up.copy_(up_host, non_blocking=True)
+        if gathered:
+            rows.copy_(rows_host, non_blocking=True)
         step()
         y_host.copy_(y, non_blocking=True)
         eev[i][1].record(stream)
@@ -382,6 +398,8 @@ def run_sharq(args):
         achieved = work / gemm_avg / 1e12
         bpe = prep_bytes_per_elem(fmt, pat, 4 if swiglu else 2)
         prep_bytes = bpe * T * K
+        if gathered:  # prep of the tokens, then each routed row's prepared bytes read and written once
+            prep_bytes = bpe * x_host.shape[0] * K + 2 * (bpe - 2) * T * K + 4 * T
         prep_gbs = prep_bytes / (statistics.mean(prep_ms) / 1e3) / 1e9
         prep_given_gbs = prep_bytes / (prep_given_ms / 1e3) / 1e9
         clocks = clk.summary()
@@ -419,7 +437,8 @@ def run_sharq(args):
                      "bytes_per_elem": bpe, "avg_us": round(statistics.mean(prep_ms) * 1e3, 2),
                      "avg_us_given_amax": round(prep_given_ms * 1e3, 2)},
             "e2e": {"value": round(world * flops * args.steps / (e2e_ms / 1e3) / 1e12, 3), "unit": "TFLOP/s",
-                    "h2d_bytes_per_step": int(x_host.numel() * 2 * (2 if swiglu else 1)),
+                    "h2d_bytes_per_step": int(x_host.numel() * 2 * (2 if swiglu else 1)
+                                              + (rows_host.numel() * 4 if gathered else 0)),
                     "d2h_bytes_per_step": int(y_host.numel() * 2)},
             "gpu_launches": int(launches),
             "launch_mode": "CUDA graphs (prep graph + GEMM graph per step); e2e uses direct API calls",

@@ -157,6 +157,19 @@ sharq_status sharq_prepare(const void* x, sharq_dtype x_dt, const void* gamma, f
 sharq_status sharq_prepare_swiglu(const void* gate, const void* up, sharq_dtype dt, float act_amax,
                                   sharq_prepared* out, sharq_stream stream);
 
+/* Row gather of prepared activations, for a mixture-of-experts layer: prepare every token
+ * once, then lay its prepared row out once per expert it is routed to (SharQ evaluates
+ * Qwen3-30B-A3B; each token goes to several experts, so preparing the routed rows
+ * repeats the per-row work for every copy).  dst row i is src row rows[i] for rows[i]
+ * in [0, src->t), else (rows[i] < 0, and every padding row up to t_pad) the encoding of
+ * an all-zero input row.  rows: DEVICE, dst->t int32 values.  src and dst share k, fmt
+ * and pat; dst->tensor receives src->tensor.  The result equals preparing the gathered
+ * rows directly whenever the NVFP4 tensor amax is the same (routed rows hold the tokens'
+ * values and zeros).  Index values are not checked on the host: one at or beyond src->t
+ * is treated as a zero row. */
+sharq_status sharq_gather_prepared(const sharq_prepared* src, const int32_t* rows, sharq_prepared* dst,
+                                   sharq_stream stream);
+
 /* Largest t that sharq_prepare_noalloc accepts (its static scratch holds one float per row). */
 #define SHARQ_NOALLOC_MAX_ROWS 65536
 

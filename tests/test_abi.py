@@ -105,3 +105,18 @@ def test_noalloc_limit_matches_header_and_rejects_on_host(L):
         sharq.sharq_prepare_noalloc(16, sharq.BF16, None, 1e-6, 0.0, a, 0)
     assert ei.value.status == 5 and "static scratch" in str(ei.value)
     assert sharq.sharq_launch_count() == before
+
+
+def test_gather_prepared_rejects_mismatch_on_host(L):
+    """Source and destination must agree on k, format and pattern; checked before any launch."""
+    before = sharq.sharq_launch_count()
+    src = sharq.sharq_prepared(16, 16, 16, 16, 16, 16, 256, 512, 1, 1)
+    for dst in (sharq.sharq_prepared(16, 16, 16, 16, 16, 16, 128, 256, 1, 1),
+                sharq.sharq_prepared(16, 16, 16, 16, 16, 16, 128, 512, 0, 1),
+                sharq.sharq_prepared(16, 16, 16, 16, 16, 16, 128, 512, 1, 2)):
+        with pytest.raises(sharq.SharqError) as ei:
+            sharq.sharq_gather_prepared(src, 16, dst, 0)
+        assert ei.value.status == 1
+    with pytest.raises(sharq.SharqError):  # no index array
+        sharq.sharq_gather_prepared(src, 0, sharq.sharq_prepared(16, 16, 16, 16, 16, 16, 128, 512, 1, 1), 0)
+    assert sharq.sharq_launch_count() == before
