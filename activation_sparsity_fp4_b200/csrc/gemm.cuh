@@ -124,6 +124,7 @@ struct GemmParams {
   const uint8_t* sf_w_sparse;    // per expert tiled, n rows, k/(2b)
   const float* tensor_x;         // [amax, g_enc, g_dec]
   const float* tensor_w;         // experts * 3
+  const void* w_codes;           // packed weight codes, row-major [experts * n][k / 2] (L2 warm-up only)
   void* y;
   int y_bf16;
   int paths;          // bit 0 sparse backbone, bit 1 dense residual
@@ -184,6 +185,17 @@ __global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ Ge
   const int n_tiles = (int)(p.n / C::BN);
   const int num_tiles = m_tiles * n_tiles;
   const int k_tiles = (int)(p.k / C::BK);
+  if (warp == 0 && lane == 0 && p.experts <= 1 && (int)blockIdx.x < num_tiles) {
+    // while the kernel before this one finishes: warm L2 with this CTA's share
+    // of the weight rows of its first tile (the CTAs on one column of tiles
+    // split them); the weight is not written by the preparation kernels
+    const int mt = (int)blockIdx.x % m_tiles, nt = (int)blockIdx.x / m_tiles;
+    const int per = (C::BN + m_tiles - 1) / m_tiles;
+    const int64_t row_bytes = p.k / 2;
+    const uint8_t* w0 = static_cast<const uint8_t*>(p.w_codes) + ((int64_t)nt * C::BN + (int64_t)mt * per) * row_bytes;
+    for (int r = 0; r < per && mt * per + r < C::BN; r++) prefetch_l2(w0 + r * row_bytes, (uint32_t)row_bytes);
+  }
+  grid_dep_wait();  // the prepared activations (and scales) are complete
   const int64_t sd_per_row = p.k / C::kVecDense;                    // dense-view scales per row
   const int64_t sb_per_row = SPARSE ? p.k / C::kVecSparse : sd_per_row;
   const int64_t wsd_bytes = tiled_sf_bytes(p.n, sd_per_row);

@@ -135,6 +135,18 @@ __global__ void __launch_bounds__(448, 1) gemm_pair_kernel(const __grid_constant
   const int n_tiles = (int)(p.n / C::BN);
   const int num_tiles = m_pairs * n_tiles;
   const int k_tiles = (int)(p.k / C::BK);
+  if (warp == 0 && lane == 0 && cluster < num_tiles) {
+    // while the kernel before this one finishes: warm L2 with this CTA's share
+    // of the weight rows of its first tile (the pairs on one column of tiles
+    // split them); the weight is not written by the preparation kernels
+    const int mt = cluster % m_pairs, nt = cluster / m_pairs;
+    const int per = (C::BNh + m_pairs - 1) / m_pairs;
+    const int64_t row_bytes = p.k / 2;
+    const uint8_t* w0 = static_cast<const uint8_t*>(p.w_codes) +
+                        ((int64_t)nt * C::BN + C::BNh * (int64_t)rank + (int64_t)mt * per) * row_bytes;
+    for (int r = 0; r < per && mt * per + r < C::BNh; r++) prefetch_l2(w0 + r * row_bytes, (uint32_t)row_bytes);
+  }
+  grid_dep_wait();  // the prepared activations (and scales) are complete
   const int64_t sd_blocks = (p.k / C::kVecDense + 3) / 4;   // 512-byte blocks per 128-row block, dense view
   const int64_t sb_blocks = (p.k / C::kVecSparse + 3) / 4;  // backbone / sparse view
   const bool run_sparse = (p.paths & 1) != 0;

@@ -408,6 +408,7 @@ __global__ void __launch_bounds__(128) amax_kernel(const void* x, const void* ga
   static_assert(!(NORM && ACT), "the SwiGLU form has no RMSNorm");
   __shared__ float red[32 * 16];
   __shared__ float wmax[4];
+  grid_dep_launch();
   const RowMap m = row_map(k);
   const int rpb = 128 / m.tpr;
   const int row_in_block = threadIdx.x >> m.lg, tt = threadIdx.x & (m.tpr - 1);
@@ -465,6 +466,7 @@ __global__ void __launch_bounds__(128, 7) amax_rows_kernel(const void* x, const 
   __shared__ float wmax[4];
   __shared__ float ssum[4];
   __shared__ uint4 gs[4096 / 8];
+  grid_dep_launch();
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, hw = w & 1;
   const int64_t r = (int64_t)blockIdx.x * 2 + (w >> 1);
   const bool have = r < t;
@@ -724,7 +726,7 @@ __device__ __forceinline__ void quantize_unit(float (&h)[32], float c6, float g_
 }
 
 template <int FMT, int PAT, bool NORM, bool XBF16, bool ACT = false>
-__global__ void __launch_bounds__(128, 6) prep_kernel(PrepParams p) {
+__global__ void __launch_bounds__(128, ACT ? 6 : 7) prep_kernel(PrepParams p) {
   static_assert(!(NORM && ACT), "the SwiGLU form has no RMSNorm");
   __shared__ float inv_tab[128];
   __shared__ float red[32 * 16];
@@ -732,6 +734,8 @@ __global__ void __launch_bounds__(128, 6) prep_kernel(PrepParams p) {
   const RowMap m = row_map(k);
   const int rpb = 128 / m.tpr;
   const int row_in_block = threadIdx.x >> m.lg, tt = threadIdx.x & (m.tpr - 1);
+  grid_dep_wait();    // the amax pass (or whatever wrote x) has completed
+  grid_dep_launch();  // the GEMM may be scheduled; it waits for this grid in turn
 
   float g_enc = 1.0f, g_dec = 1.0f, c6 = 1.0f;
   if constexpr (FMT == FMT_NV) {
@@ -840,6 +844,8 @@ struct GatherParams {
 __global__ void __launch_bounds__(256) gather_rows_kernel(const GatherParams p) {
   const int lane = threadIdx.x & 31;
   const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  grid_dep_wait();
+  grid_dep_launch();
   if (r >= p.t_pad) return;
   int64_t src = r < p.t ? (int64_t)__ldg(p.rows + r) : -1;
   if (src >= p.src_t) src = -1;  // out of range: treated as a zero row (the host checks nothing on the device data)

@@ -23,6 +23,23 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
+// ------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while the
+// kernel before it in the stream is still running.  grid_dep_wait blocks until
+// that kernel has completed and its memory writes are visible; every such
+// kernel calls it before its first access to global memory that another kernel
+// may write.  grid_dep_launch lets the next such kernel be scheduled now (it
+// still runs its own grid_dep_wait before touching this kernel's outputs).
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Warm L2 with [p, p + bytes) (16-byte aligned, a multiple of 16 bytes); no data
+// reaches the issuing thread.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+               : "memory");
+}
+
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");

@@ -71,6 +71,48 @@ bool pair_enabled() {
   return v;
 }
 
+// SHARQ_PDL=0 launches every kernel with plain stream order (for comparison).
+bool pdl_enabled() {
+  static const bool v = [] {
+    const char* e = getenv("SHARQ_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return v;
+}
+
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous kernel in the stream still runs; it calls grid_dep_wait
+// before touching global memory another kernel writes.  cluster > 1 also sets
+// the cluster shape.
+template <typename... KArgs, typename... Args>
+sharq_status launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, unsigned cluster,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (pdl_enabled()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    n++;
+  }
+  if (cluster > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    n++;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+  if (e != cudaSuccess) return fail(SHARQ_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e));
+  return launched();
+}
+
 int sm_count() {
   int dev = 0, n = 0;
   cudaGetDevice(&dev);
@@ -158,8 +200,7 @@ unsigned row_grid(Kern kern, int64_t rows, int64_t k) {
 template <int FMT, int PAT, bool NORM, bool XBF16>
 sharq_status launch_prep(const PrepParams& pp, cudaStream_t s) {
   auto kern = prep_kernel<FMT, PAT, NORM, XBF16>;
-  kern<<<row_grid(kern, pp.t_pad, pp.k), 128, 0, s>>>(pp);
-  return launched();
+  return launch_ex(kern, dim3(row_grid(kern, pp.t_pad, pp.k)), dim3(128), 0, s, 1, pp);
 }
 
 template <bool NORM, bool XBF16>
@@ -195,8 +236,7 @@ sharq_status prep_dispatch_p(const PrepParams& pp, int pat, bool norm, bool xbf1
 template <int FMT, int PAT, bool XBF16>
 sharq_status launch_prep_swiglu(const PrepParams& pp, cudaStream_t s) {
   auto kern = prep_kernel<FMT, PAT, false, XBF16, true>;
-  kern<<<row_grid(kern, pp.t_pad, pp.k), 128, 0, s>>>(pp);
-  return launched();
+  return launch_ex(kern, dim3(row_grid(kern, pp.t_pad, pp.k)), dim3(128), 0, s, 1, pp);
 }
 template <int FMT, int PAT>
 sharq_status swiglu_dispatch_x(const PrepParams& pp, bool xbf16, cudaStream_t s) {
@@ -229,8 +269,7 @@ sharq_status launch_gemm(const GemmMaps& maps, const GemmParams& gp, cudaStream_
   const int tiles = (int)(gp.t_pad / C::BM) * (int)(gp.n / C::BN);
   const int sms = sm_count();
   dim3 grid(tiles < sms ? tiles : sms);
-  gemm_kernel<KIND, SPARSE><<<grid, 448, C::kSmemBytes, s>>>(maps, gp);
-  return launched();
+  return launch_ex(gemm_kernel<KIND, SPARSE>, grid, dim3(448), C::kSmemBytes, s, 1, maps, gp);
 }
 
 sharq_status check_prepared(const sharq_prepared* a) {
@@ -273,20 +312,8 @@ sharq_status launch_pair(const GemmMaps& maps, const GemmParams& gp, cudaStream_
   }
   const int tiles = (int)(gp.t_pad / 256) * (int)(gp.n / C::BN);
   const int pairs = sm_count() / 2;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(2 * (tiles < pairs ? tiles : pairs)));
-  cfg.blockDim = dim3(448);
-  cfg.dynamicSmemBytes = C::kSmemBytes;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  SHARQ_CUDA(cudaLaunchKernelEx(&cfg, gemm_pair_kernel<KIND>, maps, gp));
-  return launched();
+  return launch_ex(gemm_pair_kernel<KIND>, dim3((unsigned)(2 * (tiles < pairs ? tiles : pairs))), dim3(448),
+                   C::kSmemBytes, s, 2, maps, gp);
 }
 
 sharq_status run_linear(const sharq_prepared* a, const sharq_weight* w, const int32_t* offsets, void* y,
@@ -354,6 +381,7 @@ sharq_status run_linear(const sharq_prepared* a, const sharq_weight* w, const in
   gp.sf_w_sparse = static_cast<const uint8_t*>(w->scales_sparse);
   gp.tensor_x = a->tensor;
   gp.tensor_w = w->tensor;
+  gp.w_codes = w->codes;
   gp.y = y;
   gp.y_bf16 = y_dt == SHARQ_BF16;
   gp.paths = paths;
@@ -591,8 +619,7 @@ sharq_status sharq_gather_prepared(const sharq_prepared* src, const int32_t* row
   gp.bbs_per_row = d816 ? k / b : k / (2 * b);
   gp.rs_per_row = k / b;
   gp.zero_meta = d816 ? 0x00FF00FFu : 0x44444444u;
-  gather_rows_kernel<<<(unsigned)((gp.t_pad + 7) / 8), 256, 0, s>>>(gp);
-  st = launched();
+  st = launch_ex(gather_rows_kernel, dim3((unsigned)((gp.t_pad + 7) / 8)), dim3(256), 0, s, 1, gp);
   if (st != SHARQ_OK) return st;
   SHARQ_CUDA(cudaMemcpyAsync(dst->tensor, src->tensor, 3 * sizeof(float), cudaMemcpyDeviceToDevice, s));
   return SHARQ_OK;
