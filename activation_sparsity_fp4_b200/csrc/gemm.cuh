@@ -71,7 +71,11 @@ struct GemmCfg {
   static constexpr int kChunksR = BK / kVecDense / 4;                  // 512-byte scale chunks per stage
   static constexpr int kChunksB = SPARSE ? BK / kVecSparse / 4 : kChunksR;
   static constexpr int kSfaR = kChunksR * 512;
-  static constexpr int kSfbD = kNRB * kChunksR * 512;
+  // the sparse kinds load only the weight's sparse-view scales: its dense view is
+  // each of them repeated (one weight scale per 2b logical K), written into
+  // tensor memory by the staging warps; the dense-backbone form loads the dense view
+  static_assert(!SPARSE || kChunksR == 2 * kChunksB, "dense view = each sparse-view scale twice");
+  static constexpr int kSfbD = SPARSE ? 0 : kNRB * kChunksR * 512;
   static constexpr int kSfaB = kChunksB * 512;
   static constexpr int kSfbS = SPARSE ? kNRB * kChunksB * 512 : 0;
   // stage layout (offsets in bytes)
@@ -256,10 +260,12 @@ __global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ Ge
             tma_load_2d_u32(sb + C::oE + bx * C::BM * 16, &maps.e, kx_e + 16 * bx, (int32_t)m0, fb);
           bulk_load_u32(sb + C::oSfaR, g_sfa_r, C::kSfaR, fb);
           bulk_load_u32(sb + C::oSfaB, g_sfa_b, C::kSfaB, fb);
+          if constexpr (!SPARSE) {
 #pragma unroll
-          for (int rb = 0; rb < C::kNRB; rb++)
-            bulk_load_u32(sb + C::oSfbD + rb * C::kChunksR * 512, g_sfb_d + rb * sd_blocks * 512, C::kChunksR * 512,
-                          fb);
+            for (int rb = 0; rb < C::kNRB; rb++)
+              bulk_load_u32(sb + C::oSfbD + rb * C::kChunksR * 512, g_sfb_d + rb * sd_blocks * 512, C::kChunksR * 512,
+                            fb);
+          }
           if constexpr (SPARSE) {
 #pragma unroll
             for (int rb = 0; rb < C::kNRB; rb++)
@@ -404,14 +410,19 @@ __global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ Ge
         // memory with TMA stores (rows at or beyond t are outside the map)
         uint32_t pk[kCols / 2];
 #pragma unroll
-        for (int c = 0; c < kCols / 32; c++) {
-          uint32_t v[32];
-          tmem_ld32(tq + (uint32_t)(32 * c), v);
+        for (int c2 = 0; c2 < kCols / 32; c2 += 2) {
+          uint32_t v[2][32];  // two loads in flight per wait
+          tmem_ld32_nowait(tq + (uint32_t)(32 * c2), v[0]);
+          tmem_ld32_nowait(tq + (uint32_t)(32 * c2 + 32), v[1]);
+          tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 16; j++) {
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[2 * j]), alpha),
-                                                      __fmul_rn(__uint_as_float(v[2 * j + 1]), alpha));
-            pk[16 * c + j] = *reinterpret_cast<uint32_t*>(&h2);
+          for (int h = 0; h < 2; h++) {
+#pragma unroll
+            for (int j = 0; j < 16; j++) {
+              __nv_bfloat162 h2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[h][2 * j]), alpha),
+                                                        __fmul_rn(__uint_as_float(v[h][2 * j + 1]), alpha));
+              pk[16 * (c2 + h) + j] = *reinterpret_cast<uint32_t*>(&h2);
+            }
           }
         }
         tc_fence_before();
@@ -481,19 +492,26 @@ __global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ Ge
 #pragma unroll
         for (int c = 0; c < C::kChunksR; c++) {
           tmem_st4(slot + C::cSfaR + 4 * c, *reinterpret_cast<const uint4*>(sb + C::oSfaR + 512 * c + 16 * lane));
+          if constexpr (!SPARSE) {
 #pragma unroll
-          for (int rb = 0; rb < C::kNRB; rb++)
-            tmem_st4(slot + C::cSfbD + 4 * C::kNRB * c + 4 * rb,
-                     *reinterpret_cast<const uint4*>(sb + C::oSfbD + rb * C::kChunksR * 512 + 512 * c + 16 * lane));
+            for (int rb = 0; rb < C::kNRB; rb++)
+              tmem_st4(slot + C::cSfbD + 4 * C::kNRB * c + 4 * rb,
+                       *reinterpret_cast<const uint4*>(sb + C::oSfbD + rb * C::kChunksR * 512 + 512 * c + 16 * lane));
+          }
         }
 #pragma unroll
         for (int c = 0; c < C::kChunksB; c++) {
           tmem_st4(slot + C::cSfaB + 4 * c, *reinterpret_cast<const uint4*>(sb + C::oSfaB + 512 * c + 16 * lane));
           if constexpr (SPARSE) {
 #pragma unroll
-            for (int rb = 0; rb < C::kNRB; rb++)
-              tmem_st4(slot + C::cSfbS + 4 * C::kNRB * c + 4 * rb,
-                       *reinterpret_cast<const uint4*>(sb + C::oSfbS + rb * C::kChunksB * 512 + 512 * c + 16 * lane));
+            for (int rb = 0; rb < C::kNRB; rb++) {
+              const uint4 v =
+                  *reinterpret_cast<const uint4*>(sb + C::oSfbS + rb * C::kChunksB * 512 + 512 * c + 16 * lane);
+              tmem_st4(slot + C::cSfbS + 4 * C::kNRB * c + 4 * rb, v);
+              // dense-view chunks 2c and 2c+1: scales (s0 s0 s1 s1) and (s2 s2 s3 s3) of each row
+              tmem_st4(slot + C::cSfbD + 4 * C::kNRB * (2 * c) + 4 * rb, dup_lo_scales(v));
+              tmem_st4(slot + C::cSfbD + 4 * C::kNRB * (2 * c + 1) + 4 * rb, dup_hi_scales(v));
+            }
           }
         }
 #pragma unroll

@@ -50,7 +50,11 @@ struct PairCfg {
   static constexpr int kXStage = BK / 2, kXStageB = BK / 4;    // TMA inner coordinate steps (bytes)
   static constexpr int kChunksR = BK / kVecDense / 4;          // 512-byte scale chunks per stage
   static constexpr int kChunksB = BK / kVecSparse / 4;
-  static constexpr int kSfaR = kChunksR * 512, kSfbD = kNRB * kChunksR * 512;
+  // the weight's dense-view scales are its sparse-view scales repeated (one weight
+  // scale per 2b logical K): only the sparse view is loaded, the staging warps
+  // write both views into tensor memory
+  static_assert(kChunksR == 2 * kChunksB, "dense view = each sparse-view scale twice");
+  static constexpr int kSfaR = kChunksR * 512, kSfbD = 0;
   static constexpr int kSfaB = kChunksB * 512, kSfbS = kNRB * kChunksB * 512;
   static constexpr int oW = 0, oR = oW + kBoxW, oB = oR + kBoxR, oE = oB + kBBytes;
   static constexpr int oSfaR = oE + kEBytes, oSfbD = oSfaR + kSfaR, oSfaB = oSfbD + kSfbD, oSfbS = oSfaB + kSfaB;
@@ -164,7 +168,6 @@ __global__ void __launch_bounds__(448, 1) gemm_pair_kernel(const __grid_constant
         const int32_t wrow = (int32_t)((int64_t)nt * C::BN + C::BNh * rank);  // this CTA's weight rows
         const uint8_t* g_sfa_r = p.sf_res + (m0 / 128) * sd_blocks * 512;
         const uint8_t* g_sfa_b = p.sf_bb + (m0 / 128) * sb_blocks * 512;
-        const uint8_t* g_sfb_d = p.sf_w_dense + (int64_t)nt * C::kNRB * sd_blocks * 512;
         const uint8_t* g_sfb_s = p.sf_w_sparse + (int64_t)nt * C::kNRB * sb_blocks * 512;
         int32_t kx = 0, kx_b = 0, kx_e = 0;
         for (int kt = 0; kt < k_tiles; kt++, g++) {
@@ -183,18 +186,14 @@ __global__ void __launch_bounds__(448, 1) gemm_pair_kernel(const __grid_constant
           bulk_load_u32(sb + C::oSfaR, g_sfa_r, C::kSfaR, sf);
           bulk_load_u32(sb + C::oSfaB, g_sfa_b, C::kSfaB, sf);
 #pragma unroll
-          for (int rb = 0; rb < C::kNRB; rb++) {
-            bulk_load_u32(sb + C::oSfbD + rb * C::kChunksR * 512, g_sfb_d + rb * sd_blocks * 512, C::kChunksR * 512,
-                          sf);
+          for (int rb = 0; rb < C::kNRB; rb++)
             bulk_load_u32(sb + C::oSfbS + rb * C::kChunksB * 512, g_sfb_s + rb * sb_blocks * 512, C::kChunksB * 512,
                           sf);
-          }
           kx += C::kXStage;
           kx_b += C::kXStageB;
           kx_e += C::kMetaStage;
           g_sfa_r += C::kSfaR;
           g_sfa_b += C::kSfaB;
-          g_sfb_d += C::kChunksR * 512;
           g_sfb_s += C::kChunksB * 512;
           issued |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (ph << stage);
@@ -292,14 +291,19 @@ __global__ void __launch_bounds__(448, 1) gemm_pair_kernel(const __grid_constant
         // accumulator so the next tile's MMAs start while the stores drain
         uint32_t pk[kCols / 2];
 #pragma unroll
-        for (int c = 0; c < kCols / 32; c++) {
-          uint32_t v[32];
-          tmem_ld32(tq + (uint32_t)(32 * c), v);
+        for (int c2 = 0; c2 < kCols / 32; c2 += 2) {
+          uint32_t v[2][32];  // two loads in flight per wait
+          tmem_ld32_nowait(tq + (uint32_t)(32 * c2), v[0]);
+          tmem_ld32_nowait(tq + (uint32_t)(32 * c2 + 32), v[1]);
+          tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 16; j++) {
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[2 * j]), alpha),
-                                                      __fmul_rn(__uint_as_float(v[2 * j + 1]), alpha));
-            pk[16 * c + j] = *reinterpret_cast<uint32_t*>(&h2);
+          for (int h = 0; h < 2; h++) {
+#pragma unroll
+            for (int j = 0; j < 16; j++) {
+              __nv_bfloat162 h2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[h][2 * j]), alpha),
+                                                        __fmul_rn(__uint_as_float(v[h][2 * j + 1]), alpha));
+              pk[16 * (c2 + h) + j] = *reinterpret_cast<uint32_t*>(&h2);
+            }
           }
         }
         tc_fence_before();
@@ -386,20 +390,19 @@ __global__ void __launch_bounds__(448, 1) gemm_pair_kernel(const __grid_constant
         const uint8_t* sb = smem + stage * C::kStageBytes;
         const uint32_t st = tq + C::BN + (uint32_t)(slot * C::kSlotCols);
 #pragma unroll
-        for (int c = 0; c < C::kChunksR; c++) {
+        for (int c = 0; c < C::kChunksR; c++)
           tmem_st4(st + C::cSfaR + 4 * c, *reinterpret_cast<const uint4*>(sb + C::oSfaR + 512 * c + 16 * lane));
-#pragma unroll
-          for (int rb = 0; rb < C::kNRB; rb++)
-            tmem_st4(st + C::cSfbD + 4 * C::kNRB * c + 4 * rb,
-                     *reinterpret_cast<const uint4*>(sb + C::oSfbD + rb * C::kChunksR * 512 + 512 * c + 16 * lane));
-        }
 #pragma unroll
         for (int c = 0; c < C::kChunksB; c++) {
           tmem_st4(st + C::cSfaB + 4 * c, *reinterpret_cast<const uint4*>(sb + C::oSfaB + 512 * c + 16 * lane));
 #pragma unroll
-          for (int rb = 0; rb < C::kNRB; rb++)
-            tmem_st4(st + C::cSfbS + 4 * C::kNRB * c + 4 * rb,
-                     *reinterpret_cast<const uint4*>(sb + C::oSfbS + rb * C::kChunksB * 512 + 512 * c + 16 * lane));
+          for (int rb = 0; rb < C::kNRB; rb++) {
+            const uint4 v = *reinterpret_cast<const uint4*>(sb + C::oSfbS + rb * C::kChunksB * 512 + 512 * c + 16 * lane);
+            tmem_st4(st + C::cSfbS + 4 * C::kNRB * c + 4 * rb, v);
+            // dense-view chunks 2c and 2c+1: scales (s0 s0 s1 s1) and (s2 s2 s3 s3) of each row
+            tmem_st4(st + C::cSfbD + 4 * C::kNRB * (2 * c) + 4 * rb, dup_lo_scales(v));
+            tmem_st4(st + C::cSfbD + 4 * C::kNRB * (2 * c + 1) + 4 * rb, dup_hi_scales(v));
+          }
         }
         tmem_st4(st + C::cE, *reinterpret_cast<const uint4*>(sb + C::oE + 16 * (32 * q + lane)));
         tmem_st_wait();

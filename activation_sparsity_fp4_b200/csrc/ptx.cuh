@@ -23,6 +23,18 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
+// A 16-byte scale-chunk row holds four rows' four scales (one 32-bit word per
+// row).  These repeat each of a word's first (lo) or last (hi) two scales:
+// (s0 s1 s2 s3) -> (s0 s0 s1 s1) or (s2 s2 s3 s3).
+__device__ __forceinline__ uint4 dup_lo_scales(uint4 v) {
+  return make_uint4(__byte_perm(v.x, 0, 0x1100), __byte_perm(v.y, 0, 0x1100), __byte_perm(v.z, 0, 0x1100),
+                    __byte_perm(v.w, 0, 0x1100));
+}
+__device__ __forceinline__ uint4 dup_hi_scales(uint4 v) {
+  return make_uint4(__byte_perm(v.x, 0, 0x3322), __byte_perm(v.y, 0, 0x3322), __byte_perm(v.z, 0, 0x3322),
+                    __byte_perm(v.w, 0, 0x3322));
+}
+
 // ------------------------------------------------- programmatic dependent launch
 // A kernel launched with programmatic stream serialization may start while the
 // kernel before it in the stream is still running.  grid_dep_wait blocks until
