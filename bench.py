@@ -367,16 +367,14 @@ def run_sharq(args):
     step_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = sum(step_ms)
 
-    # caller-given amax variant of prep (no extra read of x), for the prep roofline
-    pev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    # caller-given amax variant of prep (no extra read of x), for the prep roofline:
+    # a graph of the same call with the amax the device found, replayed like the others
     amax = float(prep.tensor[0].item())
-    for i in range(args.steps):
-        flush.fill_(1)
-        pev[i][0].record(stream)
+    g_given = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_given):
         do_prep(amax if fmt == "nvfp4" else 0.0)
-        pev[i][1].record(stream)
-    torch.cuda.synchronize()
-    prep_given_ms = statistics.mean(a.elapsed_time(b) for a, b in pev)
+    prep_given_ms = statistics.mean(replay_ms(g_given))
+    sharq.sharq_sync_status()
 
     # end to end through the public API from pinned host buffers
     eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
