@@ -110,11 +110,32 @@ struct GemmCfg {
   static constexpr uint32_t kIdesc = (kFmt << 7) | (kFmt << 10) | ((uint32_t)(BN >> 3) << 17) |
                                      ((KIND == GK_NVF4 ? 0u : 1u) << 23) | ((uint32_t)(BM >> 4) << 24);
   static constexpr uint32_t kIdescSp = kIdesc | (1u << 2);
+  static constexpr int kBandTiles = 16;  // row tiles per raster band (2048 rows)
   // 16-byte-unit offset inside a stage of the dense operand slice for logical K index kk
   __host__ __device__ static constexpr uint32_t dense_off(int box_bytes, int kk) {
     return (uint32_t)((kk / kBoxElems) * (box_bytes / 16) + (kUnpacked ? (kk % kBoxElems) / 16 : (kk % kBoxElems) / 32));
   }
 };
+
+// Raster order of the output tiles: bands of up to gm row tiles; inside a band
+// the row tile varies fastest, so the tiles in flight at one time share a few
+// activation row blocks and weight column blocks, which stay in L2 (plain row-
+// major order would sweep all activation rows once per weight column block).
+struct TileXY {
+  int mt, nt;    // row tile, column tile
+  int lo, h;     // the band: row tiles lo .. lo + h - 1
+};
+__device__ __forceinline__ TileXY tile_xy(int t, int m_tiles, int n_tiles, int gm) {
+  const int per_band = gm * n_tiles;
+  const int b = t / per_band;
+  TileXY x;
+  x.lo = b * gm;
+  x.h = m_tiles - x.lo < gm ? m_tiles - x.lo : gm;
+  const int r = t - b * per_band;
+  x.mt = x.lo + r % x.h;
+  x.nt = r / x.h;
+  return x;
+}
 
 struct GemmParams {
   int64_t t;          // rows of y to store (rows >= t are computed but not stored)
@@ -193,11 +214,11 @@ __global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ Ge
     // while the kernel before this one finishes: warm L2 with this CTA's share
     // of the weight rows of its first tile (the CTAs on one column of tiles
     // split them); the weight is not written by the preparation kernels
-    const int mt = (int)blockIdx.x % m_tiles, nt = (int)blockIdx.x / m_tiles;
-    const int per = (C::BN + m_tiles - 1) / m_tiles;
+    const TileXY x = tile_xy((int)blockIdx.x, m_tiles, n_tiles, C::kBandTiles);
+    const int per = (C::BN + x.h - 1) / x.h, i = x.mt - x.lo;
     const int64_t row_bytes = p.k / 2;
-    const uint8_t* w0 = static_cast<const uint8_t*>(p.w_codes) + ((int64_t)nt * C::BN + (int64_t)mt * per) * row_bytes;
-    for (int r = 0; r < per && mt * per + r < C::BN; r++) prefetch_l2(w0 + r * row_bytes, (uint32_t)row_bytes);
+    const uint8_t* w0 = static_cast<const uint8_t*>(p.w_codes) + ((int64_t)x.nt * C::BN + (int64_t)i * per) * row_bytes;
+    for (int r = 0; r < per && i * per + r < C::BN; r++) prefetch_l2(w0 + r * row_bytes, (uint32_t)row_bytes);
   }
   grid_dep_wait();  // the prepared activations (and scales) are complete
   const int64_t sd_per_row = p.k / C::kVecDense;                    // dense-view scales per row
@@ -230,7 +251,8 @@ __global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ Ge
       const int64_t sd_blocks = (sd_per_row + 3) / 4, sb_blocks = (sb_per_row + 3) / 4;
       const int64_t ss_blocks = (p.k / C::kVecSparse + 3) / 4;
       for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x) {
-        const int mt = tile % m_tiles, nt = tile / m_tiles;
+        const TileXY xy = tile_xy(tile, m_tiles, n_tiles, C::kBandTiles);
+        const int mt = xy.mt, nt = xy.nt;
         const int64_t m0 = (int64_t)mt * C::BM;
         const int e = tile_expert(m0);
         if (e < 0) continue;
@@ -304,7 +326,7 @@ __global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ Ge
       const uint32_t lo0 = smem_u32(smem) >> 4;
       const uint32_t empty0 = smem_u32(empty);
       for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x, it++) {
-        const int mt = tile % m_tiles;
+        const int mt = tile_xy(tile, m_tiles, n_tiles, C::kBandTiles).mt;
         if (tile_expert((int64_t)mt * C::BM) < 0) { it--; continue; }
         if (!mbar_wait(acc_empty, (it & 1) ^ 1, p.timeout_ns, abort_flag)) { *abort_flag = 1; break; }
         tc_fence_after();
@@ -394,7 +416,8 @@ __global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ Ge
     uint8_t* yb = ybuf + (warp - 2) * (32 * C::kYCols * 2);
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x, it++) {
-      const int mt = tile % m_tiles, nt = tile / m_tiles;
+      const TileXY xy = tile_xy(tile, m_tiles, n_tiles, C::kBandTiles);
+      const int mt = xy.mt, nt = xy.nt;
       const int64_t m0 = (int64_t)mt * C::BM;
       const int e = tile_expert(m0);
       if (e < 0) { it--; continue; }
@@ -483,7 +506,7 @@ __global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ Ge
     int stage = 0;
     uint32_t phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x) {
-      const int mt = tile % m_tiles;
+      const int mt = tile_xy(tile, m_tiles, n_tiles, C::kBandTiles).mt;
       if (tile_expert((int64_t)mt * C::BM) < 0) continue;
       for (int kt = 0; kt < k_tiles; kt++) {
         if (!mbar_wait(&full[stage], phase, p.timeout_ns, abort_flag)) { *abort_flag = 1; break; }

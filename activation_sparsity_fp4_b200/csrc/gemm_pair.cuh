@@ -75,6 +75,7 @@ struct PairCfg {
   static constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                                      ((KIND == GK_NVF4 ? 0u : 1u) << 23) | ((uint32_t)(256 >> 4) << 24);
   static constexpr uint32_t kIdescSp = kIdesc | (1u << 2);
+  static constexpr int kBandTiles = 8;  // row-tile pairs per raster band (2048 rows)
 };
 
 __device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
@@ -143,12 +144,12 @@ __global__ void __launch_bounds__(448, 1) gemm_pair_kernel(const __grid_constant
     // while the kernel before this one finishes: warm L2 with this CTA's share
     // of the weight rows of its first tile (the pairs on one column of tiles
     // split them); the weight is not written by the preparation kernels
-    const int mt = cluster % m_pairs, nt = cluster / m_pairs;
-    const int per = (C::BNh + m_pairs - 1) / m_pairs;
+    const TileXY x = tile_xy(cluster, m_pairs, n_tiles, C::kBandTiles);
+    const int per = (C::BNh + x.h - 1) / x.h, i = x.mt - x.lo;
     const int64_t row_bytes = p.k / 2;
     const uint8_t* w0 = static_cast<const uint8_t*>(p.w_codes) +
-                        ((int64_t)nt * C::BN + C::BNh * (int64_t)rank + (int64_t)mt * per) * row_bytes;
-    for (int r = 0; r < per && mt * per + r < C::BNh; r++) prefetch_l2(w0 + r * row_bytes, (uint32_t)row_bytes);
+                        ((int64_t)x.nt * C::BN + C::BNh * (int64_t)rank + (int64_t)i * per) * row_bytes;
+    for (int r = 0; r < per && i * per + r < C::BNh; r++) prefetch_l2(w0 + r * row_bytes, (uint32_t)row_bytes);
   }
   grid_dep_wait();  // the prepared activations (and scales) are complete
   const int64_t sd_blocks = (p.k / C::kVecDense + 3) / 4;   // 512-byte blocks per 128-row block, dense view
@@ -163,7 +164,8 @@ __global__ void __launch_bounds__(448, 1) gemm_pair_kernel(const __grid_constant
       const uint32_t smem0 = smem_u32(smem);
       const uint32_t full_leader = mapa_u32(smem_u32(full), 0);
       for (int tile = cluster; tile < num_tiles && !*abort_flag; tile += nclusters) {
-        const int mt = tile % m_pairs, nt = tile / m_pairs;
+        const TileXY xy = tile_xy(tile, m_pairs, n_tiles, C::kBandTiles);
+        const int mt = xy.mt, nt = xy.nt;
         const int64_t m0 = (int64_t)mt * 256 + 128 * (int64_t)rank;         // this CTA's activation rows
         const int32_t wrow = (int32_t)((int64_t)nt * C::BN + C::BNh * rank);  // this CTA's weight rows
         const uint8_t* g_sfa_r = p.sf_res + (m0 / 128) * sd_blocks * 512;
@@ -279,7 +281,8 @@ __global__ void __launch_bounds__(448, 1) gemm_pair_kernel(const __grid_constant
     const uint32_t acc_empty_leader = mapa_u32(smem_u32(acc_empty), 0);
     int it = 0;
     for (int tile = cluster; tile < num_tiles && !*abort_flag; tile += nclusters, it++) {
-      const int mt = tile % m_pairs, nt = tile / m_pairs;
+      const TileXY xy = tile_xy(tile, m_pairs, n_tiles, C::kBandTiles);
+      const int mt = xy.mt, nt = xy.nt;
       if (!mbar_wait(acc_full, (uint32_t)(it & 1), p.timeout_ns, abort_flag)) { abort_both(); break; }
       tc_fence_after();
       const float alpha = __fmul_rn(__ldg(p.tensor_x + 2), __ldg(p.tensor_w + 2));
