@@ -154,6 +154,11 @@ struct GemmParams {
   int y_bf16;
   int paths;          // bit 0 sparse backbone, bit 1 dense residual
   uint64_t timeout_ns;
+  // stream-K (CTA-pair kernel only; null = whole tiles): per pair a slot of
+  // partial sums (2 CTAs x 8 epilogue warps x 32 x 128 fp32) and one counter
+  // per (slot, CTA, epilogue warp), odd while a partial waits to be added
+  float* sk_part;
+  uint32_t* sk_flag;
 };
 
 struct GemmMaps {

@@ -152,6 +152,37 @@ __global__ void __launch_bounds__(448, 1) gemm_pair_kernel(const __grid_constant
     for (int r = 0; r < per && i * per + r < C::BNh; r++) prefetch_l2(w0 + r * row_bytes, (uint32_t)row_bytes);
   }
   grid_dep_wait();  // the prepared activations (and scales) are complete
+
+  // Work of this pair.  Whole tiles cluster, cluster + nclusters, ... in raster
+  // order; or, with a stream-K workspace, the contiguous run [u_lo, u_hi) of
+  // an even split of all (tile, K tile) units over the pairs, cut at tile
+  // boundaries into segments [ks, ke) of one tile.  A segment that starts inside
+  // its tile (ks > 0, only a pair's first) leaves its partial sums in this
+  // pair's workspace slot; the segment that holds the tile's K tile 0 but not
+  // its last (only a pair's last) adds the partials of the pairs after it
+  // before writing the output; every other segment is a whole tile.
+  const bool sk = p.sk_part != nullptr;
+  const int64_t units = (int64_t)num_tiles * k_tiles;
+  auto unit_lo = [&](int64_t q) -> int64_t { return q * units / nclusters; };
+  auto next_seg = [&](int64_t& st, int& tile, int& ks, int& ke) -> bool {
+    if (sk) {
+      const int64_t hi = unit_lo(cluster + 1);
+      if (st >= hi) return false;
+      tile = (int)(st / k_tiles);
+      ks = (int)(st - (int64_t)tile * k_tiles);
+      const int64_t tend = (int64_t)(tile + 1) * k_tiles;
+      ke = (int)((tend < hi ? tend : hi) - (int64_t)tile * k_tiles);
+      st = (int64_t)tile * k_tiles + ke;
+      return true;
+    }
+    if (st >= num_tiles) return false;
+    tile = (int)st;
+    ks = 0;
+    ke = k_tiles;
+    st += nclusters;
+    return true;
+  };
+  const int64_t seg0 = sk ? unit_lo(cluster) : (int64_t)cluster;
   const int64_t sd_blocks = (p.k / C::kVecDense + 3) / 4;   // 512-byte blocks per 128-row block, dense view
   const int64_t sb_blocks = (p.k / C::kVecSparse + 3) / 4;  // backbone / sparse view
   const bool run_sparse = (p.paths & 1) != 0;
@@ -163,16 +194,19 @@ __global__ void __launch_bounds__(448, 1) gemm_pair_kernel(const __grid_constant
       uint32_t g = 0, issued = 0, issued_par = 0;
       const uint32_t smem0 = smem_u32(smem);
       const uint32_t full_leader = mapa_u32(smem_u32(full), 0);
-      for (int tile = cluster; tile < num_tiles && !*abort_flag; tile += nclusters) {
+      int64_t st = seg0;
+      int tile, ks, ke;
+      while (!*abort_flag && next_seg(st, tile, ks, ke)) {
         const TileXY xy = tile_xy(tile, m_pairs, n_tiles, C::kBandTiles);
         const int mt = xy.mt, nt = xy.nt;
         const int64_t m0 = (int64_t)mt * 256 + 128 * (int64_t)rank;         // this CTA's activation rows
         const int32_t wrow = (int32_t)((int64_t)nt * C::BN + C::BNh * rank);  // this CTA's weight rows
-        const uint8_t* g_sfa_r = p.sf_res + (m0 / 128) * sd_blocks * 512;
-        const uint8_t* g_sfa_b = p.sf_bb + (m0 / 128) * sb_blocks * 512;
-        const uint8_t* g_sfb_s = p.sf_w_sparse + (int64_t)nt * C::kNRB * sb_blocks * 512;
-        int32_t kx = 0, kx_b = 0, kx_e = 0;
-        for (int kt = 0; kt < k_tiles; kt++, g++) {
+        const uint8_t* g_sfa_r = p.sf_res + (m0 / 128) * sd_blocks * 512 + (int64_t)ks * C::kSfaR;
+        const uint8_t* g_sfa_b = p.sf_bb + (m0 / 128) * sb_blocks * 512 + (int64_t)ks * C::kSfaB;
+        const uint8_t* g_sfb_s =
+            p.sf_w_sparse + (int64_t)nt * C::kNRB * sb_blocks * 512 + (int64_t)ks * C::kChunksB * 512;
+        int32_t kx = ks * C::kXStage, kx_b = ks * C::kXStageB, kx_e = ks * C::kMetaStage;
+        for (int kt = ks; kt < ke; kt++, g++) {
           const int stage = (int)(g % C::kStages);
           const uint32_t ph = (g / C::kStages) & 1u;
           if (!mbar_wait(&empty[stage], ph ^ 1u, p.timeout_ns, abort_flag)) { abort_both(); break; }
@@ -218,11 +252,13 @@ __global__ void __launch_bounds__(448, 1) gemm_pair_kernel(const __grid_constant
       const uint32_t lo0 = smem_u32(smem) >> 4;
       const uint32_t empty_own = smem_u32(empty), empty_peer = mapa_u32(empty_own, 1);
       const uint32_t accf_own = smem_u32(acc_full), accf_peer = mapa_u32(accf_own, 1);
-      for (int tile = cluster; tile < num_tiles && !*abort_flag; tile += nclusters, it++) {
+      int64_t st = seg0;
+      int tile, ks, ke;
+      for (; !*abort_flag && next_seg(st, tile, ks, ke); it++) {
         if (!mbar_wait(acc_empty, (uint32_t)(it & 1) ^ 1u, p.timeout_ns, abort_flag)) { abort_both(); break; }
         tc_fence_after();
         uint32_t accumulate = 0;
-        for (int kt = 0; kt < k_tiles; kt++, g++) {
+        for (int kt = ks; kt < ke; kt++, g++) {
           const int stage = (int)(g % C::kStages), slot = (int)(g % C::kSlots);
           if (!mbar_wait(&full[stage], (g / C::kStages) & 1u, p.timeout_ns, abort_flag)) { abort_both(); break; }
           if (!mbar_wait(&sf_ready[slot], (g / C::kSlots) & 1u, p.timeout_ns, abort_flag)) { abort_both(); break; }
@@ -279,16 +315,87 @@ __global__ void __launch_bounds__(448, 1) gemm_pair_kernel(const __grid_constant
     const int q = warp & 3, hcol = (warp - 2) >> 2;
     const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(kCols * hcol);
     const uint32_t acc_empty_leader = mapa_u32(smem_u32(acc_empty), 0);
+    const int w8 = warp - 2;  // this warp's share of a partial-sum slot
+    // partial sums of pair q's slot for this CTA and warp: 32 x 128 fp32 as
+    // float4 [column chunk c (32)][4-column group j (8)][lane]
+    auto part_of = [&](int64_t q) {
+      return reinterpret_cast<float4*>(p.sk_part) + ((q * 2 + rank) * 8 + w8) * (kCols / 4) * 32;
+    };
+    auto flag_of = [&](int64_t q) { return p.sk_flag + (q * 2 + rank) * 8 + w8; };
     int it = 0;
-    for (int tile = cluster; tile < num_tiles && !*abort_flag; tile += nclusters, it++) {
+    int64_t st = seg0;
+    int tile, ks, ke;
+    for (; !*abort_flag && next_seg(st, tile, ks, ke); it++) {
       const TileXY xy = tile_xy(tile, m_pairs, n_tiles, C::kBandTiles);
       const int mt = xy.mt, nt = xy.nt;
       if (!mbar_wait(acc_full, (uint32_t)(it & 1), p.timeout_ns, abort_flag)) { abort_both(); break; }
       tc_fence_after();
+      if (ks > 0) {
+        // stream-K, a segment that starts inside its tile: the raw sums go to
+        // this pair's slot; the pair holding the tile's K tile 0 adds them
+        float4* part = part_of(cluster);
+#pragma unroll 1
+        for (int c2 = 0; c2 < kCols / 32; c2 += 2) {
+          uint32_t v[2][32];
+          tmem_ld32_nowait(tq + (uint32_t)(32 * c2), v[0]);
+          tmem_ld32_nowait(tq + (uint32_t)(32 * c2 + 32), v[1]);
+          tmem_ld_wait();
+#pragma unroll
+          for (int h = 0; h < 2; h++)
+#pragma unroll
+            for (int j = 0; j < 8; j++)
+              __stcg(part + ((c2 + h) * 8 + j) * 32 + lane,
+                     make_float4(__uint_as_float(v[h][4 * j]), __uint_as_float(v[h][4 * j + 1]),
+                                 __uint_as_float(v[h][4 * j + 2]), __uint_as_float(v[h][4 * j + 3])));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(acc_empty_leader);
+        __threadfence();  // the partial is visible device-wide before its counter turns odd
+        __syncwarp();
+        if (lane == 0) atomicAdd(flag_of(cluster), 1u);
+        continue;
+      }
+      // pairs after this one whose first segments complete this tile (stream-K)
+      // (the host launches stream-K only with at least two units per pair, so
+      // every pair's run is non-empty and starts after the previous one's)
+      int q_end = cluster + 1;
+      if (sk && ke < k_tiles) {
+        const int64_t tend = (int64_t)(tile + 1) * k_tiles;
+        while (q_end < nclusters && unit_lo(q_end) < tend) q_end++;
+        bool ok = true;
+        if (lane == 0)
+          for (int q = cluster + 1; q < q_end && ok; q++) ok = wait_odd_acquire(flag_of(q), p.timeout_ns, abort_flag);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        __syncwarp();
+        __threadfence();
+        if (!ok) { abort_both(); break; }
+      }
       const float alpha = __fmul_rn(__ldg(p.tensor_x + 2), __ldg(p.tensor_w + 2));
       const int64_t row = (int64_t)mt * 256 + 128 * (int64_t)rank + 32 * q + lane;
       const bool store = row < p.t;
       const int64_t n0 = (int64_t)nt * C::BN + kCols * hcol;
+      // 32 columns of this warp's accumulator (+ the partial sums) as fp32
+      auto drain = [&](const uint32_t (&v)[32], int c, float (&f)[32]) {
+#pragma unroll
+        for (int i = 0; i < 32; i++) f[i] = __uint_as_float(v[i]);
+        for (int qq = cluster + 1; qq < q_end; qq++) {
+          const float4* part = part_of(qq);
+#pragma unroll
+          for (int j = 0; j < 8; j++) {
+            const float4 a = __ldcg(part + (c * 8 + j) * 32 + lane);
+            f[4 * j] = __fadd_rn(f[4 * j], a.x);
+            f[4 * j + 1] = __fadd_rn(f[4 * j + 1], a.y);
+            f[4 * j + 2] = __fadd_rn(f[4 * j + 2], a.z);
+            f[4 * j + 3] = __fadd_rn(f[4 * j + 3], a.w);
+          }
+        }
+      };
+      auto release_partials = [&]() {  // the partials added here may be rewritten by the next call
+        __syncwarp();
+        if (lane == 0)
+          for (int qq = cluster + 1; qq < q_end; qq++) atomicAdd(flag_of(qq), 1u);
+      };
       if (p.y_bf16) {
         // this warp's columns into registers as bf16, then release the
         // accumulator so the next tile's MMAs start while the stores drain
@@ -301,10 +408,11 @@ __global__ void __launch_bounds__(448, 1) gemm_pair_kernel(const __grid_constant
           tmem_ld_wait();
 #pragma unroll
           for (int h = 0; h < 2; h++) {
+            float f[32];
+            drain(v[h], c2 + h, f);
 #pragma unroll
             for (int j = 0; j < 16; j++) {
-              __nv_bfloat162 h2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[h][2 * j]), alpha),
-                                                        __fmul_rn(__uint_as_float(v[h][2 * j + 1]), alpha));
+              __nv_bfloat162 h2 = __floats2bfloat162_rn(__fmul_rn(f[2 * j], alpha), __fmul_rn(f[2 * j + 1], alpha));
               pk[16 * (c2 + h) + j] = *reinterpret_cast<uint32_t*>(&h2);
             }
           }
@@ -312,6 +420,7 @@ __global__ void __launch_bounds__(448, 1) gemm_pair_kernel(const __grid_constant
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_remote(acc_empty_leader);
+        release_partials();
         // 32 rows x 32 columns at a time through shared memory, written by a
         // TMA store (whole lines; rows at or beyond t are clipped by the map)
         (void)store;
@@ -345,32 +454,19 @@ __global__ void __launch_bounds__(448, 1) gemm_pair_kernel(const __grid_constant
 #pragma unroll
         for (int h = 0; h < 2; h++) {
           const int c = c2 + h;
-          const uint32_t(&v)[32] = vv[h];
-          if (p.y_bf16) {
-            uint32_t pk[16];
+          float f[32];
+          drain(vv[h], c, f);
+          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.y) + row * p.n + n0 + 32 * c);
 #pragma unroll
-            for (int j = 0; j < 16; j++) {
-              __nv_bfloat162 h2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[2 * j]), alpha),
-                                                        __fmul_rn(__uint_as_float(v[2 * j + 1]), alpha));
-              pk[j] = *reinterpret_cast<uint32_t*>(&h2);
-            }
-            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.y) + row * p.n + n0 + 32 * c);
-#pragma unroll
-            for (int j = 0; j < 4; j++) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-          } else {
-            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.y) + row * p.n + n0 + 32 * c);
-#pragma unroll
-            for (int j = 0; j < 8; j++)
-              dst[j] = make_float4(__fmul_rn(__uint_as_float(v[4 * j]), alpha),
-                                   __fmul_rn(__uint_as_float(v[4 * j + 1]), alpha),
-                                   __fmul_rn(__uint_as_float(v[4 * j + 2]), alpha),
-                                   __fmul_rn(__uint_as_float(v[4 * j + 3]), alpha));
-          }
+          for (int j = 0; j < 8; j++)
+            dst[j] = make_float4(__fmul_rn(f[4 * j], alpha), __fmul_rn(f[4 * j + 1], alpha),
+                                 __fmul_rn(f[4 * j + 2], alpha), __fmul_rn(f[4 * j + 3], alpha));
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(acc_empty_leader);
+      release_partials();
     }
   } else {
     // ------------------------------------------------ scale-slot staging
@@ -379,8 +475,10 @@ __global__ void __launch_bounds__(448, 1) gemm_pair_kernel(const __grid_constant
     const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16);
     const uint32_t sf_ready_leader = mapa_u32(smem_u32(sf_ready), 0);
     uint32_t g = 0;
-    for (int tile = cluster; tile < num_tiles && !*abort_flag; tile += nclusters) {
-      for (int kt = 0; kt < k_tiles; kt++, g++) {
+    int64_t st = seg0;
+    int tile, ks, ke;
+    while (!*abort_flag && next_seg(st, tile, ks, ke)) {
+      for (int kt = ks; kt < ke; kt++, g++) {
         const int stage = (int)(g % C::kStages), slot = (int)(g % C::kSlots);
         if (g >= (uint32_t)C::kSlots) {  // the slot's previous K tile has been consumed by its MMAs
           const uint32_t gp = g - C::kSlots;

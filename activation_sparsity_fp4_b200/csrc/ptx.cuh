@@ -100,6 +100,28 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
   }
 }
 
+// Wait until the 32-bit global counter is odd (load with acquire semantics at
+// GPU scope), or until timeout_ns has passed, or *abort becomes nonzero.  On a
+// timeout set the error word and return false.
+__device__ __forceinline__ bool wait_odd_acquire(const uint32_t* ctr, uint64_t timeout_ns, volatile int* abort) {
+  auto odd = [&]() {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    return (v & 1u) != 0;
+  };
+  if (odd()) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
+    if (odd()) return true;
+    if (abort && *abort) return false;
+    if (global_ns() - t0 > timeout_ns) {
+      atomicOr(&g_error_word, kErrTimeout);
+      return false;
+    }
+    __nanosleep(64);
+  }
+}
+
 // 32-bit shared-address forms for the issue loops (no address conversion per call)
 __device__ __forceinline__ void mbar_arrive_expect_tx_u32(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");

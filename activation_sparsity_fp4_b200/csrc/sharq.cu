@@ -71,6 +71,15 @@ bool pair_enabled() {
   return v;
 }
 
+// SHARQ_STREAMK=0 keeps whole tiles even when a stream-K workspace is given (for comparison).
+bool stream_k_enabled() {
+  static const bool v = [] {
+    const char* e = getenv("SHARQ_STREAMK");
+    return !(e && e[0] == '0');
+  }();
+  return v;
+}
+
 // SHARQ_PDL=0 launches every kernel with plain stream order (for comparison).
 bool pdl_enabled() {
   static const bool v = [] {
@@ -300,6 +309,34 @@ sharq_status check_weight(const sharq_weight* w) {
   return SHARQ_OK;
 }
 
+// Clusters of the CTA-pair GEMM that can be resident at once on this device (0 if unknown).
+template <int KIND>
+int pair_max_resident() {
+  static int v = -1;
+  if (v < 0) {
+    using C = PairCfg<KIND>;
+    cudaFuncSetAttribute(gemm_pair_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(sm_count() & ~1));
+    cfg.blockDim = dim3(448);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<KIND>, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+    v = n;
+  }
+  return v;
+}
+
 // CTA-pair GEMM: clusters of 2 CTAs, one per SM, persistent over 256 x 256 tiles.
 template <int KIND>
 sharq_status launch_pair(const GemmMaps& maps, const GemmParams& gp, cudaStream_t s) {
@@ -312,12 +349,27 @@ sharq_status launch_pair(const GemmMaps& maps, const GemmParams& gp, cudaStream_
   }
   const int tiles = (int)(gp.t_pad / 256) * (int)(gp.n / C::BN);
   const int pairs = sm_count() / 2;
-  return launch_ex(gemm_pair_kernel<KIND>, dim3((unsigned)(2 * (tiles < pairs ? tiles : pairs))), dim3(448),
-                   C::kSmemBytes, s, 2, maps, gp);
+  int clusters = tiles < pairs ? tiles : pairs;
+  if (gp.sk_part) {
+    // stream-K: as many pairs as can be resident at once (a pair waits for the
+    // partial sums of the pairs after it), and at least two K tiles per pair
+    const int64_t units = (int64_t)tiles * (gp.k / C::BK);
+    clusters = pair_max_resident<KIND>();
+    if (clusters > pairs) clusters = pairs;
+    if (units < 2 * (int64_t)clusters) clusters = (int)(units / 2);
+  }
+  return launch_ex(gemm_pair_kernel<KIND>, dim3((unsigned)(2 * clusters)), dim3(448), C::kSmemBytes, s, 2, maps, gp);
 }
 
+// Stream-K workspace of the CTA-pair GEMM: per pair a slot of partial sums
+// (2 CTAs x 8 epilogue warps x 32 rows x 128 fp32 columns), then one 32-bit
+// counter per (slot, CTA, epilogue warp).
+constexpr size_t kSkSlotBytes = 2 * 8 * 32 * 128 * sizeof(float);
+constexpr size_t kSkFlagBytes = 2 * 8 * sizeof(uint32_t);
+size_t sk_workspace_bytes() { return (size_t)(sm_count() / 2) * (kSkSlotBytes + kSkFlagBytes); }
+
 sharq_status run_linear(const sharq_prepared* a, const sharq_weight* w, const int32_t* offsets, void* y,
-                        sharq_dtype y_dt, int32_t paths, cudaStream_t s) {
+                        sharq_dtype y_dt, int32_t paths, cudaStream_t s, void* ws = nullptr, size_t ws_bytes = 0) {
   sharq_status st = check_prepared(a);
   if (st != SHARQ_OK) return st;
   st = check_weight(w);
@@ -386,10 +438,31 @@ sharq_status run_linear(const sharq_prepared* a, const sharq_weight* w, const in
   gp.y_bf16 = y_dt == SHARQ_BF16;
   gp.paths = paths;
   gp.timeout_ns = wait_timeout_ns();
+  gp.sk_part = nullptr;
+  gp.sk_flag = nullptr;
+  if (ws) {
+    if (ws_bytes < sk_workspace_bytes() || !aligned(ws, 16))
+      return fail(SHARQ_ERR_WORKSPACE, "stream-K workspace: %zu bytes, 16-byte aligned, needed",
+                  sk_workspace_bytes());
+  }
   if (pairs) {
     // CTA pairs: each SM loads half of every weight tile (128-row weight boxes)
     st = make_map(&maps.w, w->codes, w->k / 2, w->n, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != SHARQ_OK) return st;
+    const int64_t tiles = (t_pad / 256) * (w->n / 256);
+    const int npairs = sm_count() / 2;
+    const int resident = a->fmt == SHARQ_NVFP4 ? pair_max_resident<GK_NVF4>() : pair_max_resident<GK_MXF4>();
+    const int np = resident < npairs ? resident : npairs;
+    const int64_t units = tiles * (w->k / 256);
+    if (ws && stream_k_enabled() && np > 0 && 2 * tiles <= np && units >= 8 * (int64_t)np) {
+      // few tiles with long K loops (most pairs would idle): split the K loops
+      // of all tiles evenly over every pair (stream-K).  Measured on B200: at
+      // 256 x 4096 x 16384 it takes 44 instead of 54 us; with more tiles or
+      // shorter K the extra segment boundaries and the partial sums cost more
+      // than the balance gains (2048 x 4096 x 4096: 41 instead of 35 us)
+      gp.sk_part = static_cast<float*>(ws);
+      gp.sk_flag = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + (size_t)npairs * kSkSlotBytes);
+    }
     return a->fmt == SHARQ_NVFP4 ? launch_pair<GK_NVF4>(maps, gp, s) : launch_pair<GK_MXF4>(maps, gp, s);
   }
   if (a->fmt == SHARQ_NVFP4)
@@ -644,6 +717,16 @@ sharq_status sharq_linear(const sharq_prepared* a, const sharq_weight* w, void* 
   return run_linear(a, w, nullptr, y, y_dt, 3, reinterpret_cast<cudaStream_t>(stream));
 }
 
+sharq_status sharq_linear_workspace_size(size_t* bytes) {
+  if (!bytes) return fail(SHARQ_ERR_INVALID, "bytes is NULL");
+  *bytes = sk_workspace_bytes();
+  return SHARQ_OK;
+}
+sharq_status sharq_linear_ws(const sharq_prepared* a, const sharq_weight* w, void* y, sharq_dtype y_dt,
+                             void* workspace, size_t workspace_bytes, sharq_stream stream) {
+  if (!workspace) return fail(SHARQ_ERR_WORKSPACE, "workspace is NULL");
+  return run_linear(a, w, nullptr, y, y_dt, 3, reinterpret_cast<cudaStream_t>(stream), workspace, workspace_bytes);
+}
 sharq_status sharq_linear_paths(const sharq_prepared* a, const sharq_weight* w, void* y, sharq_dtype y_dt,
                                 int32_t paths, sharq_stream stream) {
   return run_linear(a, w, nullptr, y, y_dt, paths, reinterpret_cast<cudaStream_t>(stream));

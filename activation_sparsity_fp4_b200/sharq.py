@@ -25,7 +25,7 @@ STATUS = {0: "SHARQ_OK", 1: "SHARQ_ERR_INVALID", 2: "SHARQ_ERR_UNSUPPORTED", 3: 
 SYMBOLS = ["sharq_weight_sizes", "sharq_prepared_sizes", "sharq_quantize_weight", "sharq_prepare", "sharq_linear",
            "sharq_linear_paths", "sharq_linear_grouped", "sharq_sync_status", "sharq_selftest_wait_timeout",
            "sharq_last_error", "sharq_launch_count", "sharq_prepare_noalloc", "sharq_prepare_swiglu",
-           "sharq_gather_prepared"]
+           "sharq_gather_prepared", "sharq_linear_ws", "sharq_linear_workspace_size"]
 NOALLOC_MAX_ROWS = 65536  # SHARQ_NOALLOC_MAX_ROWS of the C header
 
 
@@ -73,6 +73,9 @@ def lib() -> ctypes.CDLL:
             "sharq_prepare_noalloc": [P, I, P, F, F, ctypes.POINTER(sharq_prepared), P],
             "sharq_prepare_swiglu": [P, P, I, F, ctypes.POINTER(sharq_prepared), P],
             "sharq_gather_prepared": [ctypes.POINTER(sharq_prepared), P, ctypes.POINTER(sharq_prepared), P],
+            "sharq_linear_ws": [ctypes.POINTER(sharq_prepared), ctypes.POINTER(sharq_weight), P, I, P,
+                                ctypes.c_size_t, P],
+            "sharq_linear_workspace_size": [ctypes.POINTER(ctypes.c_size_t)],
             "sharq_linear": [ctypes.POINTER(sharq_prepared), ctypes.POINTER(sharq_weight), P, I, P],
             "sharq_linear_paths": [ctypes.POINTER(sharq_prepared), ctypes.POINTER(sharq_weight), P, I, I32, P],
             "sharq_linear_grouped": [ctypes.POINTER(sharq_prepared), ctypes.POINTER(sharq_weight), P, P, I, P],
@@ -170,6 +173,18 @@ def sharq_gather_prepared(src: sharq_prepared, rows_ptr: int, dst: sharq_prepare
 def sharq_linear(a: sharq_prepared, w: sharq_weight, y_ptr: int, y_dt, stream=None):
     _check(lib().sharq_linear(ctypes.byref(a), ctypes.byref(w), ctypes.c_void_p(y_ptr), _dt(y_dt), _stream(stream)),
            "sharq_linear")
+
+
+def sharq_linear_ws(a: sharq_prepared, w: sharq_weight, y_ptr: int, y_dt, ws_ptr: int, ws_bytes: int, stream=None):
+    _check(lib().sharq_linear_ws(ctypes.byref(a), ctypes.byref(w), ctypes.c_void_p(y_ptr), _dt(y_dt),
+                                 ctypes.c_void_p(ws_ptr), ctypes.c_size_t(ws_bytes), _stream(stream)),
+           "sharq_linear_ws")
+
+
+def sharq_linear_workspace_size() -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().sharq_linear_workspace_size(ctypes.byref(out)), "sharq_linear_workspace_size")
+    return int(out.value)
 
 
 def sharq_linear_paths(a: sharq_prepared, w: sharq_weight, y_ptr: int, y_dt, paths: int, stream=None):
@@ -285,12 +300,24 @@ def gather_prepared(src: Prepared, rows: torch.Tensor, out: Prepared | None = No
     return out
 
 
+def linear_workspace(device="cuda") -> torch.Tensor:
+    """A zero-filled stream-K workspace for `linear(..., workspace=...)` on this device."""
+    with torch.cuda.device(torch.device(device)):
+        return torch.zeros(sharq_linear_workspace_size(), dtype=torch.uint8, device=device)
+
+
 def linear(a: Prepared, w: FP4Weight, out_dtype=torch.bfloat16, out: torch.Tensor | None = None, paths: int = 3,
-           stream=None) -> torch.Tensor:
-    """y = the sparse backbone GEMM plus the dense residual GEMM, (t, n)."""
+           stream=None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """y = the sparse backbone GEMM plus the dense residual GEMM, (t, n).  With a
+    workspace (see `linear_workspace`) the CTA-pair GEMM may split its K loops
+    over every SM pair (stream-K)."""
     if out is None:
         out = torch.empty((a.t, w.n), dtype=out_dtype, device=a.meta.device)
-    if paths == 3:
+    if workspace is not None:
+        assert paths == 3, "the stream-K form runs both paths"
+        sharq_linear_ws(a.struct, w.struct, out.data_ptr(), out.dtype, workspace.data_ptr(),
+                        workspace.numel() * workspace.element_size(), stream)
+    elif paths == 3:
         sharq_linear(a.struct, w.struct, out.data_ptr(), out.dtype, stream)
     else:
         sharq_linear_paths(a.struct, w.struct, out.data_ptr(), out.dtype, paths, stream)

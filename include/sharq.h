@@ -209,6 +209,26 @@ sharq_status sharq_prepare_noalloc(const void* x, sharq_dtype x_dt, const void* 
 sharq_status sharq_linear(const sharq_prepared* a, const sharq_weight* w, void* y, sharq_dtype y_dt,
                           sharq_stream stream);
 
+/* sharq_linear with a stream-K workspace.  When the CTA-pair GEMM runs (the 4:8
+ * pair kinds, t a multiple of 256 after padding, not grouped) and it has few
+ * 256 x 256 output tiles with long K loops (at most half as many tiles as SM
+ * pairs, at least 8 K tiles of 256 per pair), the K loops of all tiles are split
+ * evenly over every pair: a pair whose share starts inside a tile leaves
+ * its partial sums in its workspace slot, and the pair holding that tile's first
+ * K tile adds them before writing y.  Results equal sharq_linear's up to the
+ * order of the fp32 partial sums.  Otherwise it is sharq_linear.
+ * workspace: DEVICE, >= sharq_linear_workspace_size() bytes, 16-byte aligned,
+ * zero-filled before its first use; every completed call leaves its counters as
+ * it found them.  After SHARQ_ERR_TIMEOUT zero it again before reuse.  Calls that
+ * overlap in time (several streams) need separate workspaces.
+ * SHARQ_ERR_WORKSPACE: NULL, too small or misaligned (checked on the host). */
+sharq_status sharq_linear_ws(const sharq_prepared* a, const sharq_weight* w, void* y, sharq_dtype y_dt,
+                             void* workspace, size_t workspace_bytes, sharq_stream stream);
+
+/* Bytes of sharq_linear_ws's workspace on the current device (one 256 KiB slot
+ * of partial sums and 64 bytes of counters per pair of SMs). */
+sharq_status sharq_linear_workspace_size(size_t* bytes);
+
 /* Same, with a choice of paths for diagnosis: paths bit 0 = sparse backbone GEMM,
  * bit 1 = dense residual GEMM (3 = the layer). */
 sharq_status sharq_linear_paths(const sharq_prepared* a, const sharq_weight* w, void* y, sharq_dtype y_dt,

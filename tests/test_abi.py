@@ -120,3 +120,13 @@ def test_gather_prepared_rejects_mismatch_on_host(L):
     with pytest.raises(sharq.SharqError):  # no index array
         sharq.sharq_gather_prepared(src, 0, sharq.sharq_prepared(16, 16, 16, 16, 16, 16, 128, 512, 1, 1), 0)
     assert sharq.sharq_launch_count() == before
+
+
+def test_linear_ws_requires_a_workspace(L):
+    before = sharq.sharq_launch_count()
+    a = sharq.sharq_prepared(16, 16, 16, 16, 16, 16, 256, 256, 1, 1)
+    w = sharq.sharq_weight(16, 16, 16, 16, 256, 256, 1, 1)
+    with pytest.raises(sharq.SharqError) as ei:
+        sharq.sharq_linear_ws(a, w, 16, sharq.BF16, 0, 0, 0)
+    assert ei.value.status == 5 and "workspace" in str(ei.value)
+    assert sharq.sharq_launch_count() == before

@@ -1,0 +1,100 @@
+"""Stream-K form of the CTA-pair GEMM (sharq_linear_ws): K loops of all tiles
+split evenly over the SM pairs, partial sums added by the pair that holds each
+tile's first K tile.  Results match the oracle like the whole-tile form, agree
+with it up to the order of the fp32 partial sums, and leave the workspace
+counters as they found them."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from activation_sparsity_fp4_b200 import sharq, workloads
+from gpu_common import assert_close_gemm, gpu_prepare, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _w(seed, n, k, scale=0.02):
+    rng = np.random.default_rng(seed)
+    return workloads.to_bf16_values((rng.standard_normal((n, k)) * scale).astype(np.float32))
+
+
+def _x(seed, t, k):
+    rng = np.random.default_rng(seed)
+    x = (0.5 * rng.standard_t(3, size=(t, k))).astype(np.float32)
+    x[:, rng.permutation(k)[:6]] *= 60.0
+    return workloads.to_bf16_values(x)
+
+
+def _flags(ws: torch.Tensor) -> np.ndarray:
+    pairs = torch.cuda.get_device_properties(0).multi_processor_count // 2
+    slot = 2 * 8 * 32 * 128 * 4
+    return ws[pairs * slot:].cpu().numpy().view(np.uint32)
+
+
+# (t, n, k): few tiles with long K loops, where the split applies: 16 tiles of
+# 64 K tiles (each spread over ~5 pairs), and 500 ragged rows in 16 tiles
+SHAPES = [(256, 4096, 16384), (500, 2048, 16384)]
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4"])
+@pytest.mark.parametrize("shape", SHAPES)
+def test_stream_k_matches_oracle_and_whole_tiles(cuda_ok, fmt, shape):
+    """fp32 output against fp64 and against the whole-tile form; bf16 output
+    equal to the fp32 output rounded to bf16 (same split, same sums)."""
+    t, n, k = shape
+    x, w = _x(31, t, k), _w(32, n, k)
+    p = gpu_prepare(x, "bf16", fmt, "4:8pair")
+    wq = sharq.FP4Weight.quantize(to_dev(w, "bf16"), fmt)
+    ws = sharq.linear_workspace()
+    y_sk = sharq.linear(p, wq, out_dtype=torch.float32, workspace=ws)
+    y_bf = sharq.linear(p, wq, out_dtype=torch.bfloat16, workspace=ws)
+    y_wt = sharq.linear(p, wq, out_dtype=torch.float32)
+    sharq.sharq_sync_status()
+    prep = oracle.prepare(x, fmt, "4:8pair", threads=4)
+    ref = oracle.linear_ref(prep, oracle.quantize_weight(w, fmt))
+    assert_close_gemm(y_sk.cpu().numpy(), ref, f"stream-K {fmt} {shape}")
+    assert_close_gemm(y_sk.cpu().numpy(), y_wt.double().cpu().numpy(), "stream-K vs whole tiles")
+    assert torch.equal(y_bf, y_sk.to(torch.bfloat16)), "bf16 output != fp32 output rounded to bf16"
+    assert (_flags(ws) % 2 == 0).all(), "a partial-sum counter was left odd"
+
+
+def test_stream_k_repeated_calls_are_deterministic(cuda_ok):
+    """The same workspace serves call after call (counters return to even); the
+    fixed split gives the same bits every time."""
+    t, n, k = SHAPES[0]
+    x, w = _x(33, t, k), _w(34, n, k)
+    p = gpu_prepare(x, "bf16", "nvfp4", "4:8pair")
+    wq = sharq.FP4Weight.quantize(to_dev(w, "bf16"), "nvfp4")
+    ws = sharq.linear_workspace()
+    ys = [sharq.linear(p, wq, workspace=ws).clone() for _ in range(4)]
+    sharq.sharq_sync_status()
+    for y in ys[1:]:
+        assert torch.equal(y, ys[0])
+    f = _flags(ws)
+    assert (f % 2 == 0).all() and f.max() > 0  # used, and every partial consumed
+
+
+def test_stream_k_not_used_on_the_q_proj_shape(cuda_ok):
+    """128 tiles of 16 K tiles (the bench's q_proj launch) keep whole tiles: the
+    workspace changes nothing and stays untouched."""
+    cfg = workloads.q_proj()
+    p = gpu_prepare(cfg["x"], "bf16", "nvfp4", "4:8pair", gamma=cfg["gamma"])
+    wq = sharq.FP4Weight.quantize(to_dev(cfg["w"], "bf16"), "nvfp4")
+    ws = sharq.linear_workspace()
+    a, b = sharq.linear(p, wq, workspace=ws), sharq.linear(p, wq)
+    sharq.sharq_sync_status()
+    assert torch.equal(a, b)
+    assert (_flags(ws) == 0).all()
+
+
+def test_stream_k_falls_back_where_it_does_not_apply(cuda_ok):
+    """Grouped, single-CTA kinds and whole waves ignore the workspace (same bits as sharq_linear)."""
+    x, w = _x(35, 300, 1024), _w(36, 512, 1024)  # 384 padded rows: single-CTA kernel
+    p = gpu_prepare(x, "bf16", "mxfp4", "2:4")
+    wq = sharq.FP4Weight.quantize(to_dev(w, "bf16"), "mxfp4")
+    ws = sharq.linear_workspace()
+    a, b = sharq.linear(p, wq, workspace=ws), sharq.linear(p, wq)
+    sharq.sharq_sync_status()
+    assert torch.equal(a, b)
+    assert (_flags(ws) == 0).all()
