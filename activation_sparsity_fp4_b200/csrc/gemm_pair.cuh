@@ -82,7 +82,8 @@ __device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
 
-template <int KIND>
+// SK: the stream-K form (p.sk_part set); otherwise whole tiles only.
+template <int KIND, bool SK>
 __global__ void __launch_bounds__(448, 1) gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
   using C = PairCfg<KIND>;
   extern __shared__ uint8_t smem_raw[];
@@ -161,7 +162,7 @@ __global__ void __launch_bounds__(448, 1) gemm_pair_kernel(const __grid_constant
   // pair's workspace slot; the segment that holds the tile's K tile 0 but not
   // its last (only a pair's last) adds the partials of the pairs after it
   // before writing the output; every other segment is a whole tile.
-  const bool sk = p.sk_part != nullptr;
+  constexpr bool sk = SK;
   const int64_t units = (int64_t)num_tiles * k_tiles;
   auto unit_lo = [&](int64_t q) -> int64_t { return q * units / nclusters; };
   auto next_seg = [&](int64_t& st, int& tile, int& ks, int& ke) -> bool {
@@ -330,7 +331,7 @@ __global__ void __launch_bounds__(448, 1) gemm_pair_kernel(const __grid_constant
       const int mt = xy.mt, nt = xy.nt;
       if (!mbar_wait(acc_full, (uint32_t)(it & 1), p.timeout_ns, abort_flag)) { abort_both(); break; }
       tc_fence_after();
-      if (ks > 0) {
+      if (sk && ks > 0) {
         // stream-K, a segment that starts inside its tile: the raw sums go to
         // this pair's slot; the pair holding the tile's K tile 0 adds them
         float4* part = part_of(cluster);
@@ -379,7 +380,7 @@ __global__ void __launch_bounds__(448, 1) gemm_pair_kernel(const __grid_constant
       auto drain = [&](const uint32_t (&v)[32], int c, float (&f)[32]) {
 #pragma unroll
         for (int i = 0; i < 32; i++) f[i] = __uint_as_float(v[i]);
-        for (int qq = cluster + 1; qq < q_end; qq++) {
+        for (int qq = cluster + 1; SK && qq < q_end; qq++) {
           const float4* part = part_of(qq);
 #pragma unroll
           for (int j = 0; j < 8; j++) {
@@ -392,9 +393,11 @@ __global__ void __launch_bounds__(448, 1) gemm_pair_kernel(const __grid_constant
         }
       };
       auto release_partials = [&]() {  // the partials added here may be rewritten by the next call
-        __syncwarp();
-        if (lane == 0)
-          for (int qq = cluster + 1; qq < q_end; qq++) atomicAdd(flag_of(qq), 1u);
+        if (SK) {
+          __syncwarp();
+          if (lane == 0)
+            for (int qq = cluster + 1; qq < q_end; qq++) atomicAdd(flag_of(qq), 1u);
+        }
       };
       if (p.y_bf16) {
         // this warp's columns into registers as bf16, then release the

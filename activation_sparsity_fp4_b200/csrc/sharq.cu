@@ -315,7 +315,7 @@ int pair_max_resident() {
   static int v = -1;
   if (v < 0) {
     using C = PairCfg<KIND>;
-    cudaFuncSetAttribute(gemm_pair_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    cudaFuncSetAttribute(gemm_pair_kernel<KIND, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(sm_count() & ~1));
     cfg.blockDim = dim3(448);
@@ -328,7 +328,7 @@ int pair_max_resident() {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<KIND>, &cfg) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<KIND, true>, &cfg) != cudaSuccess) {
       cudaGetLastError();
       n = 0;
     }
@@ -343,7 +343,9 @@ sharq_status launch_pair(const GemmMaps& maps, const GemmParams& gp, cudaStream_
   using C = PairCfg<KIND>;
   static bool configured = false;
   if (!configured) {
-    SHARQ_CUDA(cudaFuncSetAttribute(gemm_pair_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    SHARQ_CUDA(cudaFuncSetAttribute(gemm_pair_kernel<KIND, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    C::kSmemBytes));
+    SHARQ_CUDA(cudaFuncSetAttribute(gemm_pair_kernel<KIND, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     C::kSmemBytes));
     configured = true;
   }
@@ -358,7 +360,11 @@ sharq_status launch_pair(const GemmMaps& maps, const GemmParams& gp, cudaStream_
     if (clusters > pairs) clusters = pairs;
     if (units < 2 * (int64_t)clusters) clusters = (int)(units / 2);
   }
-  return launch_ex(gemm_pair_kernel<KIND>, dim3((unsigned)(2 * clusters)), dim3(448), C::kSmemBytes, s, 2, maps, gp);
+  if (gp.sk_part)
+    return launch_ex(gemm_pair_kernel<KIND, true>, dim3((unsigned)(2 * clusters)), dim3(448), C::kSmemBytes, s, 2,
+                     maps, gp);
+  return launch_ex(gemm_pair_kernel<KIND, false>, dim3((unsigned)(2 * clusters)), dim3(448), C::kSmemBytes, s, 2,
+                   maps, gp);
 }
 
 // Stream-K workspace of the CTA-pair GEMM: per pair a slot of partial sums
