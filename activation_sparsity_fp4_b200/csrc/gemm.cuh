@@ -137,6 +137,8 @@ __device__ __forceinline__ TileXY tile_xy(int t, int m_tiles, int n_tiles, int g
   return x;
 }
 
+constexpr int kMaxSplit = 4;  // K slices per tile in the split-K form of the single-CTA kernel
+
 struct GemmParams {
   int64_t t;          // rows of y to store (rows >= t are computed but not stored)
   int64_t t_pad;      // rows of the prepared operands (multiple of 128)
@@ -159,6 +161,11 @@ struct GemmParams {
   // per (slot, CTA, epilogue warp), odd while a partial waits to be added
   float* sk_part;
   uint32_t* sk_flag;
+  // split-K (single-CTA kernel only, split >= 2): one fp32 slot [t_pad][n] of
+  // raw sums per K slice, then one counter per tile
+  float* split_acc;
+  uint32_t* split_cnt;
+  int32_t split;
 };
 
 struct GemmMaps {
@@ -166,7 +173,9 @@ struct GemmMaps {
   CUtensorMap y;  // bf16 output, 32 x 32 boxes (CTA-pair kernel only)
 };
 
-template <int KIND, bool SPARSE>
+// SPLIT: each tile's K loop is cut into p.split slices run by different CTAs
+// (few tiles, long K: the weight stream then uses every SM).
+template <int KIND, bool SPARSE, bool SPLIT>
 __global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
   using C = GemmCfg<KIND, SPARSE>;
   extern __shared__ uint8_t smem_raw[];
@@ -178,8 +187,11 @@ __global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ Ge
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain = acc_empty + 1;
   uint64_t* sf_ready = drain + 1;  // per stage: its scale slot is in tensor memory
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sf_ready + C::kStages);
+  uint64_t* ep_done = sf_ready + C::kStages;  // split-K: the 8 epilogue warps wrote their slice
+  uint64_t* ep_flag = ep_done + 1;            // split-K: split_last is set
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(ep_flag + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile uint32_t* split_last = reinterpret_cast<volatile uint32_t*>(tmem_holder + 2);  // split-K: last slice?
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -193,6 +205,8 @@ __global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ Ge
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 8);  // 8 epilogue warps
     mbar_init(drain, 1);
+    mbar_init(ep_done, 8);
+    mbar_init(ep_flag, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -226,6 +240,11 @@ __global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ Ge
     for (int r = 0; r < per && i * per + r < C::BN; r++) prefetch_l2(w0 + r * row_bytes, (uint32_t)row_bytes);
   }
   grid_dep_wait();  // the prepared activations (and scales) are complete
+  // work items: (tile, K slice) with SPLIT, else whole tiles
+  const int n_split = SPLIT ? p.split : 1;
+  const int items = num_tiles * n_split;
+  auto k_lo = [&](int item) { return (int)((int64_t)(item % n_split) * k_tiles / n_split); };
+  auto k_hi = [&](int item) { return (int)((int64_t)(item % n_split + 1) * k_tiles / n_split); };
   const int64_t sd_per_row = p.k / C::kVecDense;                    // dense-view scales per row
   const int64_t sb_per_row = SPARSE ? p.k / C::kVecSparse : sd_per_row;
   const int64_t wsd_bytes = tiled_sf_bytes(p.n, sd_per_row);
@@ -255,7 +274,8 @@ __global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ Ge
       const uint32_t smem0 = smem_u32(smem), full0 = smem_u32(full);
       const int64_t sd_blocks = (sd_per_row + 3) / 4, sb_blocks = (sb_per_row + 3) / 4;
       const int64_t ss_blocks = (p.k / C::kVecSparse + 3) / 4;
-      for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x) {
+      for (int item = blockIdx.x; item < items && !*abort_flag; item += gridDim.x) {
+        const int tile = item / n_split, k0 = k_lo(item), k1 = k_hi(item);
         const TileXY xy = tile_xy(tile, m_tiles, n_tiles, C::kBandTiles);
         const int mt = xy.mt, nt = xy.nt;
         const int64_t m0 = (int64_t)mt * C::BM;
@@ -264,12 +284,12 @@ __global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ Ge
         const int32_t wrow = (int32_t)(e * p.n + (int64_t)nt * C::BN);
         const int64_t nb = (int64_t)nt * C::kNRB;
         // scale chunks of this tile: contiguous per 128-row block, advanced per K tile
-        const uint8_t* g_sfa_r = p.sf_res + (m0 / 128) * sd_blocks * 512;
-        const uint8_t* g_sfa_b = p.sf_bb + (m0 / 128) * sb_blocks * 512;
-        const uint8_t* g_sfb_d = p.sf_w_dense + e * wsd_bytes + nb * sd_blocks * 512;
-        const uint8_t* g_sfb_s = p.sf_w_sparse + e * wss_bytes + nb * ss_blocks * 512;
-        int32_t kx = 0, kx_b = 0, kx_e = 0;
-        for (int kt = 0; kt < k_tiles; kt++) {
+        const uint8_t* g_sfa_r = p.sf_res + (m0 / 128) * sd_blocks * 512 + (int64_t)k0 * C::kSfaR;
+        const uint8_t* g_sfa_b = p.sf_bb + (m0 / 128) * sb_blocks * 512 + (int64_t)k0 * C::kSfaB;
+        const uint8_t* g_sfb_d = p.sf_w_dense + e * wsd_bytes + nb * sd_blocks * 512 + (int64_t)k0 * C::kChunksR * 512;
+        const uint8_t* g_sfb_s = p.sf_w_sparse + e * wss_bytes + nb * ss_blocks * 512 + (int64_t)k0 * C::kChunksB * 512;
+        int32_t kx = k0 * C::kXStage, kx_b = k0 * C::kXStageB, kx_e = k0 * C::kMetaStage;
+        for (int kt = k0; kt < k1; kt++) {
           if (!mbar_wait(&empty[stage], phase ^ 1, p.timeout_ns, abort_flag)) { *abort_flag = 1; break; }
           const uint32_t sb = smem0 + (uint32_t)(stage * C::kStageBytes);
           const uint32_t fb = full0 + (uint32_t)(stage * 8);
@@ -330,13 +350,14 @@ __global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ Ge
       constexpr uint32_t kLbo = 1u << 16;  // 16-byte leading offset (ignored by swizzled K-major layouts)
       const uint32_t lo0 = smem_u32(smem) >> 4;
       const uint32_t empty0 = smem_u32(empty);
-      for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x, it++) {
+      for (int item = blockIdx.x; item < items && !*abort_flag; item += gridDim.x, it++) {
+        const int tile = item / n_split, k0 = k_lo(item), k1 = k_hi(item);
         const int mt = tile_xy(tile, m_tiles, n_tiles, C::kBandTiles).mt;
         if (tile_expert((int64_t)mt * C::BM) < 0) { it--; continue; }
         if (!mbar_wait(acc_empty, (it & 1) ^ 1, p.timeout_ns, abort_flag)) { *abort_flag = 1; break; }
         tc_fence_after();
         uint32_t accumulate = 0;
-        for (int kt = 0; kt < k_tiles; kt++) {
+        for (int kt = k0; kt < k1; kt++) {
           if (!mbar_wait(&full[stage], phase, p.timeout_ns, abort_flag)) { *abort_flag = 1; break; }
           tc_fence_after();
           const uint32_t ls = lo0 + (uint32_t)(stage * (C::kStageBytes >> 4));  // stage base, 16-byte units
@@ -420,7 +441,8 @@ __global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ Ge
     const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(kCols * hcol);
     uint8_t* yb = ybuf + (warp - 2) * (32 * C::kYCols * 2);
     int it = 0;
-    for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x, it++) {
+    for (int item = blockIdx.x; item < items && !*abort_flag; item += gridDim.x, it++) {
+      const int tile = item / n_split;
       const TileXY xy = tile_xy(tile, m_tiles, n_tiles, C::kBandTiles);
       const int mt = xy.mt, nt = xy.nt;
       const int64_t m0 = (int64_t)mt * C::BM;
@@ -432,6 +454,91 @@ __global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ Ge
       const int64_t row = m0 + 32 * q + lane;
       const bool st = row < p.t;
       const int64_t n0 = (int64_t)nt * C::BN + kCols * hcol;
+      if constexpr (SPLIT) {
+        // this K slice's raw sums into its own slot of the fp32 buffer (each
+        // warp its rows); the CTA that completes the tile's last slice adds
+        // the slots in slice order (the same bits on every call) with all 256
+        // epilogue threads, coalesced along the rows, scales, writes y and
+        // resets the tile's counter for the next call
+        const int sidx = item % n_split;
+        const int64_t slot_elems = p.t_pad * p.n;
+        float4* mine = reinterpret_cast<float4*>(p.split_acc + sidx * slot_elems + row * p.n + n0);
+#pragma unroll 1
+        for (int c2 = 0; c2 < kCols / 32; c2 += 2) {
+          uint32_t v[2][32];
+          tmem_ld32_nowait(tq + (uint32_t)(32 * c2), v[0]);
+          tmem_ld32_nowait(tq + (uint32_t)(32 * c2 + 32), v[1]);
+          tmem_ld_wait();
+          if (!st) continue;
+#pragma unroll
+          for (int h = 0; h < 2; h++)
+#pragma unroll
+            for (int j = 0; j < 8; j++)
+              __stcg(mine + (c2 + h) * 8 + j,
+                     make_float4(__uint_as_float(v[h][4 * j]), __uint_as_float(v[h][4 * j + 1]),
+                                 __uint_as_float(v[h][4 * j + 2]), __uint_as_float(v[h][4 * j + 3])));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty);
+        __threadfence();  // this slice's sums are visible before the counter moves
+        __syncwarp();
+        const int et = threadIdx.x - 64;  // 0..255 over the eight epilogue warps
+        if (lane == 0) mbar_arrive(ep_done);
+        if (et == 0) {
+          if (!mbar_wait(ep_done, it & 1, p.timeout_ns, abort_flag)) *abort_flag = 1;
+          else *split_last = atomicAdd(p.split_cnt + tile, 1u) == (uint32_t)(n_split - 1) ? 1u : 0u;
+          mbar_arrive(ep_flag);
+        }
+        if (!mbar_wait(ep_flag, it & 1, p.timeout_ns, abort_flag) || *abort_flag) { *abort_flag = 1; break; }
+        const bool last = *split_last != 0u;
+        if (!last) continue;
+        __threadfence();
+        const int64_t rows = (p.t - m0) < C::BM ? (p.t - m0) : C::BM;
+        const int c4n = C::BN / 4;  // float4 groups per row of the tile
+        const int64_t tile_f4 = (m0 * p.n + (int64_t)nt * C::BN) / 4;
+        const float4* acc4 = reinterpret_cast<const float4*>(p.split_acc) + tile_f4;
+#pragma unroll 1
+        for (int64_t idx0 = 0; idx0 < rows * c4n; idx0 += 4 * 256) {
+          float4 b[kMaxSplit][4];  // four groups per thread, every slice: all loads in flight at once
+#pragma unroll
+          for (int sl = 0; sl < kMaxSplit; sl++)
+#pragma unroll
+            for (int u = 0; u < 4; u++) {
+              const int64_t idx = idx0 + u * 256 + et;
+              const int64_t off = (idx / c4n) * (p.n / 4) + idx % c4n;
+              b[sl][u] = (sl < n_split && idx < rows * c4n) ? __ldcg(acc4 + sl * (slot_elems / 4) + off)
+                                                             : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+          float4 a[4];
+#pragma unroll
+          for (int u = 0; u < 4; u++) {
+            a[u] = b[0][u];
+#pragma unroll
+            for (int sl = 1; sl < kMaxSplit; sl++)
+              if (sl < n_split)
+                a[u] = make_float4(__fadd_rn(a[u].x, b[sl][u].x), __fadd_rn(a[u].y, b[sl][u].y),
+                                   __fadd_rn(a[u].z, b[sl][u].z), __fadd_rn(a[u].w, b[sl][u].w));
+          }
+#pragma unroll
+          for (int u = 0; u < 4; u++) {
+            const int64_t idx = idx0 + u * 256 + et;
+            if (idx >= rows * c4n) continue;
+            const int64_t r = m0 + idx / c4n, c = (int64_t)nt * C::BN + 4 * (idx % c4n);
+            const float f0 = __fmul_rn(a[u].x, alpha), f1 = __fmul_rn(a[u].y, alpha);
+            const float f2 = __fmul_rn(a[u].z, alpha), f3 = __fmul_rn(a[u].w, alpha);
+            if (p.y_bf16) {
+              __nv_bfloat162 lo = __floats2bfloat162_rn(f0, f1), hi = __floats2bfloat162_rn(f2, f3);
+              *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.y) + r * p.n + c) =
+                  make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+            } else {
+              *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.y) + r * p.n + c) = make_float4(f0, f1, f2, f3);
+            }
+          }
+        }
+        if (et == 0) p.split_cnt[tile] = 0u;
+        continue;
+      }
       if (p.y_bf16) {
         // this warp's columns into registers as bf16, release the accumulator
         // so the next tile's MMAs start, then 32 x 16 tiles through shared
@@ -510,10 +617,11 @@ __global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ Ge
     const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16);
     int stage = 0;
     uint32_t phase = 0;
-    for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x) {
+    for (int item = blockIdx.x; item < items && !*abort_flag; item += gridDim.x) {
+      const int tile = item / n_split, k0 = k_lo(item), k1 = k_hi(item);
       const int mt = tile_xy(tile, m_tiles, n_tiles, C::kBandTiles).mt;
       if (tile_expert((int64_t)mt * C::BM) < 0) continue;
-      for (int kt = 0; kt < k_tiles; kt++) {
+      for (int kt = k0; kt < k1; kt++) {
         if (!mbar_wait(&full[stage], phase, p.timeout_ns, abort_flag)) { *abort_flag = 1; break; }
         const uint8_t* sb = smem + stage * C::kStageBytes;
         const uint32_t slot = tq + C::BN + (uint32_t)(stage * C::kSlotCols);

@@ -64,8 +64,9 @@ def prep_bytes_per_elem(fmt: str, pat: str, x_bytes: int = 2) -> float:
     return x_bytes + bb_codes + meta + bb_sf + 0.5 + 1 / b
 
 
-def make_workload(name: str) -> dict:
-    """Inputs and roofline terms of one bench workload (host arrays; nothing of the method here)."""
+def make_workload(name: str, tokens: int | None = None) -> dict:
+    """Inputs and roofline terms of one bench workload (host arrays; nothing of the method here).
+    tokens: row count of the q_proj / down_proj shapes (the down_proj token sweep)."""
     from activation_sparsity_fp4_b200 import workloads
     if name in ("qwen_moe_gate_up", "qwen_moe_gate_up_gather"):
         c = workloads.qwen_moe()
@@ -77,10 +78,12 @@ def make_workload(name: str) -> dict:
         if name.endswith("_gather"):
             wl.update(tokens=c["x_tok"], gather=c["gather"])
         return wl
+    kw = {"t": tokens} if tokens and name in ("q_proj", "down_proj", "down_proj_swiglu") else {}
+    desc = WORKLOADS[name].replace("2048x", f"{tokens}x") if kw else WORKLOADS[name]
     c = {"q_proj": workloads.q_proj, "down_proj": workloads.down_proj, "down_proj_swiglu": workloads.down_proj,
-         "wan": workloads.wan, "wan_816": lambda: workloads.wan(pat="8:16")}[name]()
+         "wan": workloads.wan, "wan_816": lambda: workloads.wan(pat="8:16")}[name](**kw)
     t, k = c["x"].shape
-    wl = dict(name=name, desc=WORKLOADS[name], x=c["x"], gamma=c["gamma"], eps=c["eps"], w=c["w"],
+    wl = dict(name=name, desc=desc, x=c["x"], gamma=c["gamma"], eps=c["eps"], w=c["w"],
               fmt=c["fmt"], pat=c["pat"], offsets=None, t=t, k=k, n=c["w"].shape[0], real_rows=t,
               first_group=None, gate=None, up=None)
     if name == "down_proj_swiglu":
@@ -206,19 +209,19 @@ def committed_traffic():
 _ORACLE_SETUP = {}
 
 
-def _oracle_setup(name: str):
+def _oracle_setup(name: str, tokens: int | None = None):
     """Workload and the offline weight quantization for the oracle (untimed, once)."""
-    if _ORACLE_SETUP.get("name") != name:
+    if _ORACLE_SETUP.get("name") != (name, tokens):
         import oracle
-        wl = make_workload(name)
+        wl = make_workload(name, tokens)
         w = wl["w"][0] if wl["offsets"] is not None else wl["w"]  # grouped: the first expert's weight
         wq = oracle.quantize_weight(w, wl["fmt"])
         _ORACLE_SETUP.clear()
-        _ORACLE_SETUP.update(name=name, wl=wl, wq=wq, wu=oracle.decode_weight(wq))
+        _ORACLE_SETUP.update(name=(name, tokens), wl=wl, wq=wq, wu=oracle.decode_weight(wq))
     return _ORACLE_SETUP
 
 
-def cpu_baseline(name: str = "q_proj", rows: int = 2048):
+def cpu_baseline(name: str = "q_proj", rows: int = 2048, tokens: int | None = None):
     """The oracle, as it stands, on the host cores: the tensor amax over all rows
     (NVFP4), prep of `rows` rows (grouped: rows of the first expert) and the fp64
     reference GEMM of those rows; scaled to effective TFLOP/s (2 * rows * N * K / time)."""
@@ -226,7 +229,7 @@ def cpu_baseline(name: str = "q_proj", rows: int = 2048):
 
     import oracle
 
-    st = _oracle_setup(name)
+    st = _oracle_setup(name, tokens)
     wl, wq, wu = st["wl"], st["wq"], st["wu"]
     x = wl["x"]
     r0 = wl["first_group"][0] if wl["first_group"] else 0
@@ -266,7 +269,7 @@ def run_sharq(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         pg = dist
 
-    wl = make_workload(args.workload)
+    wl = make_workload(args.workload, args.tokens)
     T, K, N, fmt, pat = wl["t"], wl["k"], wl["n"], wl["fmt"], wl["pat"]
     swiglu = wl["gate"] is not None
     gathered = wl.get("gather") is not None  # prep of the tokens, then their prepared rows gathered
@@ -281,6 +284,7 @@ def run_sharq(args):
     del w
     offsets = torch.from_numpy(wl["offsets"]).to(torch.int32).to(dev) if wl["offsets"] is not None else None
     prep = sharq.Prepared(T, K, fmt, pat, dev)
+    ws = sharq.linear_workspace(dev)  # lets few-tile shapes split their K loops over the SMs
     if gathered:
         rows_host = torch.from_numpy(wl["gather"]).to(torch.int32).pin_memory()
         rows = rows_host.to(dev)
@@ -302,7 +306,7 @@ def run_sharq(args):
 
     def do_gemm():
         if offsets is None:
-            sharq.linear(prep, wq, out=y)
+            sharq.linear(prep, wq, out=y, workspace=ws)
         else:
             sharq.linear_grouped(prep, wq, offsets, out=y)
 
@@ -392,7 +396,7 @@ def run_sharq(args):
     ptb = [sharq.Prepared(x_host.shape[0], K, fmt, pat, dev) for _ in range(n_buf)] if gathered else None
     yb = [torch.empty_like(y) for _ in range(n_buf)]
     yh = [torch.empty_like(y_host).pin_memory() for _ in range(n_buf)]
-    ws_e2e = None
+    ws_e2e = sharq.linear_workspace(dev)  # its own: the e2e steps overlap on three streams
 
     def e2e_compute(b):
         if swiglu:
@@ -403,7 +407,7 @@ def run_sharq(args):
         else:
             sharq.prepare(xb[b], fmt, pat, gamma, wl["eps"], out=pb[b], stream=s_cmp)
         if offsets is None:
-            sharq.linear(pb[b], wq, out=yb[b], stream=s_cmp)
+            sharq.linear(pb[b], wq, out=yb[b], stream=s_cmp, workspace=ws_e2e)
         else:
             sharq.linear_grouped(pb[b], wq, offsets, out=yb[b], stream=s_cmp)
 
@@ -455,6 +459,9 @@ def run_sharq(args):
         value = world * flops * args.steps / (total_ms / 1e3) / 1e12
         gemm_avg = statistics.mean(gemm_ms) / 1e3
         work, kind, work_desc = gemm_roofline(wl)
+        b_blk = 16 if fmt == "nvfp4" else 32
+        wbytes = (N * K / 2 + N * K / (2 * b_blk) * (2 if pat == "8:16" else 1)
+                  + prep_bytes_per_elem(fmt, pat, 0) * T * K + 2 * T * N)
         ratio = FP4_OVER_BF16 if kind == "fp4" else FP8_OVER_BF16
         peak = pk["bf16_tflops"] * ratio
         achieved = work / gemm_avg / 1e12
@@ -467,7 +474,8 @@ def run_sharq(args):
         clocks = clk.summary()
         grouped = offsets is not None
         kernel = {"4:8pair": "sparse", "2:4": "sparse", "8:16": "dense backbone"}[pat]
-        kname = ("gemm_pair_kernel" if (not grouped and pat == "4:8pair" and T % 256 == 0) else "gemm_kernel")
+        kname = ("gemm_pair_kernel" if (not grouped and pat == "4:8pair" and ((T + 127) // 128 * 128) % 256 == 0)
+                 else "gemm_kernel")
         kkind = "MXF8" if (fmt == "mxfp4" and pat == "2:4") else ("NVF4" if fmt == "nvfp4" else "MXF4")
         out = {
             "metric": METRIC,
@@ -487,12 +495,20 @@ def run_sharq(args):
                        "norm": "rmsnorm" if gamma is not None else "none", "y_dtype": "bf16",
                        "parallelism": f"replicas x{world}",
                        "l2": "flushed (256 MB write) before every timed step"},
-            "roofline": {"bound": "tensor", "kernel": f"{kname}<{kkind}, {kernel}>",
-                         "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
-                         "frac": round(achieved / peak, 4),
-                         "traffic": committed_traffic() if args.workload == "q_proj" else None,
-                         "peak_source": f"{src}: bf16 burst x {ratio:g} (nominal {kind.upper()}/BF16)",
-                         "work": work_desc, "avg_launch_us": round(gemm_avg * 1e6, 2)},
+            "roofline": ({"bound": "tensor", "kernel": f"{kname}<{kkind}, {kernel}>",
+                          "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
+                          "frac": round(achieved / peak, 4),
+                          "traffic": committed_traffic() if args.workload == "q_proj" and not args.tokens else None,
+                          "peak_source": f"{src}: bf16 burst x {ratio:g} (nominal {kind.upper()}/BF16)",
+                          "work": work_desc, "avg_launch_us": round(gemm_avg * 1e6, 2)}
+                         if T > 64 else
+                         # decode-size rows: the GEMM streams the weight; HBM bound
+                         {"bound": "hbm", "kernel": f"{kname}<{kkind}, {kernel}>",
+                          "achieved": round(wbytes / gemm_avg / 1e9, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                          "frac": round(wbytes / gemm_avg / 1e9 / pk["hbm_gbs"], 4), "traffic": None,
+                          "peak_source": src,
+                          "work": "weight codes N*K/2 + sparse-view scales N*K/(2b) + prepared X + y bytes",
+                          "avg_launch_us": round(gemm_avg * 1e6, 2)}),
             "prep": {"gbs_device_amax": round(prep_gbs, 1), "gbs_given_amax": round(prep_given_gbs, 1),
                      "peak_gbs": pk["hbm_gbs"], "frac_given_amax": round(prep_given_gbs / pk["hbm_gbs"], 4),
                      "frac_device_amax": round(prep_gbs / pk["hbm_gbs"], 4),
@@ -514,7 +530,7 @@ def run_sharq(args):
             out["config"]["routed_rows"] = wl["real_rows"]
             out["config"]["experts"] = int(wl["w"].shape[0])
         if not args.no_cpu_baseline and world == 1:
-            out["cpu_baseline"], _ = cpu_baseline(args.workload)
+            out["cpu_baseline"], _ = cpu_baseline(args.workload, tokens=args.tokens)
         print(json.dumps(out), flush=True)
     if pg:
         pg.barrier()
@@ -529,11 +545,11 @@ def run_reference(args):
         return
     rows = 256
     for _ in range(args.warmup):
-        cpu_baseline(args.workload, rows)
+        cpu_baseline(args.workload, rows, args.tokens)
     times = []
     base = None
     for _ in range(args.steps):
-        base, dt = cpu_baseline(args.workload, rows)
+        base, dt = cpu_baseline(args.workload, rows, args.tokens)
         times.append(dt)
     wl = _ORACLE_SETUP["wl"]
     total = sum(times)
@@ -559,6 +575,8 @@ def main():
     ap.add_argument("--impl", choices=["sharq", "reference"], default="sharq")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="q_proj")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="row count of the q_proj / down_proj shapes (down_proj token sweep: 1, 16, 64, 256)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":

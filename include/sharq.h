@@ -215,8 +215,13 @@ sharq_status sharq_linear(const sharq_prepared* a, const sharq_weight* w, void* 
  * pairs, at least 8 K tiles of 256 per pair), the K loops of all tiles are split
  * evenly over every pair: a pair whose share starts inside a tile leaves
  * its partial sums in its workspace slot, and the pair holding that tile's first
- * K tile adds them before writing y.  Results equal sharq_linear's up to the
- * order of the fp32 partial sums.  Otherwise it is sharq_linear.
+ * K tile adds them before writing y.  The single-CTA GEMM (the other shapes) with
+ * few tiles and long K loops (at most half as many tiles as SMs, >= 32 K tiles of
+ * 256, e.g. decode-size row counts of down_proj) splits each tile's K loop into
+ * up to 4 slices on different SMs; each slice writes its raw sums to its own
+ * workspace slot and the CTA that completes a tile's last slice adds the slots in
+ * slice order and writes y.  Results equal sharq_linear's up to the order of the
+ * fp32 partial sums, and repeat bit for bit.  Otherwise it is sharq_linear.
  * workspace: DEVICE, >= sharq_linear_workspace_size() bytes, 16-byte aligned,
  * zero-filled before its first use; every completed call leaves its counters as
  * it found them.  After SHARQ_ERR_TIMEOUT zero it again before reuse.  Calls that

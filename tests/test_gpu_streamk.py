@@ -98,3 +98,33 @@ def test_stream_k_falls_back_where_it_does_not_apply(cuda_ok):
     sharq.sharq_sync_status()
     assert torch.equal(a, b)
     assert (_flags(ws) == 0).all()
+
+
+# single-CTA kernel, few tiles with long K (decode-size row counts): K split
+# into slices over the SMs, slices summed in a fixed order by the last one
+SPLIT_CASES = [("mxfp4", "2:4", 1, 4096, 14336), ("mxfp4", "2:4", 16, 4096, 14336),
+               ("mxfp4", "2:4", 64, 4096, 14336), ("mxfp4", "2:4", 256, 4096, 14336),
+               ("nvfp4", "4:8pair", 16, 4096, 8192), ("nvfp4", "8:16", 100, 1024, 8192),
+               ("mxfp4", "4:8pair", 40, 2048, 8192)]
+
+
+@pytest.mark.parametrize("fmt,pat,t,n,k", SPLIT_CASES)
+def test_split_k_single_cta_matches_oracle(cuda_ok, fmt, pat, t, n, k):
+    """fp32 output against fp64 and the unsplit kernel; bf16 output equal to the
+    fp32 output rounded to bf16; a second call gives the same bits (the slice
+    sums are added in a fixed order and every counter is reset)."""
+    x, w = _x(40 + t, t, k), _w(41, n, k)
+    p = gpu_prepare(x, "bf16", fmt, pat)
+    wq = sharq.FP4Weight.quantize(to_dev(w, "bf16"), fmt)
+    ws = sharq.linear_workspace()
+    y1 = sharq.linear(p, wq, out_dtype=torch.float32, workspace=ws).clone()
+    y2 = sharq.linear(p, wq, out_dtype=torch.float32, workspace=ws).clone()
+    yb = sharq.linear(p, wq, out_dtype=torch.bfloat16, workspace=ws)
+    y0 = sharq.linear(p, wq, out_dtype=torch.float32)
+    sharq.sharq_sync_status()
+    prep = oracle.prepare(x, fmt, pat, threads=4)
+    ref = oracle.linear_ref(prep, oracle.quantize_weight(w, fmt))
+    assert_close_gemm(y1.cpu().numpy(), ref, f"split-K {fmt} {pat} t={t}")
+    assert_close_gemm(y1.cpu().numpy(), y0.double().cpu().numpy(), "split-K vs unsplit")
+    assert torch.equal(y1, y2), "split-K is not reproducible"
+    assert torch.equal(yb, y1.to(torch.bfloat16)), "bf16 output != fp32 output rounded to bf16"
