@@ -14,6 +14,7 @@
 #include "../../include/sharq.h"
 #include "gemm.cuh"
 #include "gemm_pair.cuh"
+#include "gemv.cuh"
 #include "prep.cuh"
 
 using namespace sharq;
@@ -75,6 +76,15 @@ bool pair_enabled() {
 bool stream_k_enabled() {
   static const bool v = [] {
     const char* e = getenv("SHARQ_STREAMK");
+    return !(e && e[0] == '0');
+  }();
+  return v;
+}
+
+// SHARQ_GEMV=0 runs even 1-4 row products on the tensor-core kernels (for comparison).
+bool gemv_enabled() {
+  static const bool v = [] {
+    const char* e = getenv("SHARQ_GEMV");
     return !(e && e[0] == '0');
   }();
   return v;
@@ -406,6 +416,47 @@ constexpr size_t kSkSlotBytes = 2 * 8 * 32 * 128 * sizeof(float);
 constexpr size_t kSkFlagBytes = 2 * 8 * sizeof(uint32_t);
 size_t sk_workspace_bytes() { return (size_t)(sm_count() / 2) * (kSkSlotBytes + kSkFlagBytes); }
 
+// The 1-4 row form on the CUDA cores (gemv.cuh).
+template <int FMT, int PAT>
+sharq_status launch_gemv(const GemvParams& gp, int64_t t, cudaStream_t s) {
+  constexpr int rows_per_block = kGemvWarps * kGemvRowsPerWarp;
+  const dim3 grid((unsigned)((gp.n + rows_per_block - 1) / rows_per_block)), block(kGemvWarps * 32);
+  switch (t) {
+    case 1: return launch_ex(gemv_kernel<FMT, PAT, 1>, grid, block, 0, s, 1, gp);
+    case 2: return launch_ex(gemv_kernel<FMT, PAT, 2>, grid, block, 0, s, 1, gp);
+    case 3: return launch_ex(gemv_kernel<FMT, PAT, 3>, grid, block, 0, s, 1, gp);
+    default: return launch_ex(gemv_kernel<FMT, PAT, 4>, grid, block, 0, s, 1, gp);
+  }
+}
+
+sharq_status run_gemv(const sharq_prepared* a, const sharq_weight* w, void* y, sharq_dtype y_dt, int32_t paths,
+                      cudaStream_t s) {
+  GemvParams gp;
+  gp.n = w->n;
+  gp.k = w->k;
+  gp.paths = paths;
+  gp.meta = static_cast<const uint8_t*>(a->meta);
+  gp.bb_codes = static_cast<const uint8_t*>(a->bb_codes);
+  gp.bb_scales = static_cast<const uint8_t*>(a->bb_scales);
+  gp.res_codes = static_cast<const uint8_t*>(a->res_codes);
+  gp.res_scales = static_cast<const uint8_t*>(a->res_scales);
+  gp.t_pad = round_up(a->t, 128);
+  gp.tensor_x = a->tensor;
+  gp.w_codes = static_cast<const uint8_t*>(w->codes);
+  gp.w_sf = static_cast<const uint8_t*>(w->scales_sparse);
+  gp.tensor_w = w->tensor;
+  gp.y = y;
+  gp.y_bf16 = y_dt == SHARQ_BF16;
+  const int64_t t = a->t;
+  if (a->fmt == SHARQ_NVFP4)
+    return a->pat == SHARQ_NM_8_16 ? launch_gemv<FMT_NV, PAT_816>(gp, t, s) : launch_gemv<FMT_NV, PAT_48P>(gp, t, s);
+  switch (a->pat) {
+    case SHARQ_NM_2_4: return launch_gemv<FMT_MX, PAT_24>(gp, t, s);
+    case SHARQ_NM_4_8_PAIR: return launch_gemv<FMT_MX, PAT_48P>(gp, t, s);
+    default: return launch_gemv<FMT_MX, PAT_816>(gp, t, s);
+  }
+}
+
 sharq_status run_linear(const sharq_prepared* a, const sharq_weight* w, const int32_t* offsets, void* y,
                         sharq_dtype y_dt, int32_t paths, cudaStream_t s, void* ws = nullptr, size_t ws_bytes = 0) {
   sharq_status st = check_prepared(a);
@@ -422,6 +473,7 @@ sharq_status run_linear(const sharq_prepared* a, const sharq_weight* w, const in
     return fail(SHARQ_ERR_INVALID, "a stacked weight needs sharq_linear_grouped");
   if (a->fmt == SHARQ_NVFP4 && a->pat == SHARQ_NM_2_4)
     return fail(SHARQ_ERR_UNSUPPORTED, "NVFP4 with element-wise 2:4 has no sparse tensor-core kind");
+  if (offsets == nullptr && a->t <= kGemvMaxRows && gemv_enabled()) return run_gemv(a, w, y, y_dt, paths, s);
 
   const int64_t t_pad = round_up(a->t, 128);
   const bool sparse = a->pat != SHARQ_NM_8_16;
