@@ -129,15 +129,6 @@ __device__ __forceinline__ void swiglu_unit(const void* gate, const void* up, in
   for (int i = 0; i < 32; i++) h[i] = __fmul_rn(dev_silu(a[i]), b[i]);
 }
 
-// Two E2M1 codes (low nibble = first element) -> exact fp32 values.
-__device__ __forceinline__ void e2m1x2_values(uint32_t c, float& lo, float& hi) {
-  uint32_t h2;
-  const uint16_t byte = (uint16_t)(c & 0xFF);
-  asm("{\n\t.reg .b8 t;\n\tcvt.u8.u16 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(h2) : "h"(byte));
-  lo = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFF)));
-  hi = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
-}
-
 // Eight E2M1 codes (nibbles of c, element i in nibble i) -> exact fp32 values.
 __device__ __forceinline__ void e2m1x8_values(uint32_t c, float* out) {
 #pragma unroll
@@ -546,12 +537,6 @@ __global__ void __launch_bounds__(128, 7) amax_rows_kernel(const void* x, const 
   }
 }
 
-// ------------------------------------------------------------ prep kernel
-// Byte mask of the kept pairs of a 4:8 group: byte p = 0xFF if pair p kept.
-__device__ __forceinline__ uint32_t pair_byte_mask(uint32_t kp) {
-  return ((kp & 1u) ? 0x000000FFu : 0u) | ((kp & 2u) ? 0x0000FF00u : 0u) | ((kp & 4u) ? 0x00FF0000u : 0u) |
-         ((kp & 8u) ? 0xFF000000u : 0u);
-}
 // Nibble mask of kept elements of a 2:4 quad pair (8 elements, two quads).
 __device__ __forceinline__ uint32_t nibble_mask8(uint32_t keep8) {
   uint32_t m = 0;

@@ -62,11 +62,6 @@ __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
@@ -146,24 +141,6 @@ __device__ __forceinline__ void tma_prefetch(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int32_t x, int32_t y,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-      "[%4];" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// Plain bulk copy global -> shared (16-byte aligned, size a multiple of 16).
-__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(gmem_src)), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
 // ------------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* smem_dst, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(smem_dst)),
@@ -189,14 +166,6 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
 }
 __device__ __forceinline__ void tc_commit_u32(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
-}
-// Shared -> tensor memory copies of scale factors (32 rows x 16 B, replicated to
-// the four 32-lane sub-partitions) and of sparse metadata (128 rows x 16 B).
-__device__ __forceinline__ void tc_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-__device__ __forceinline__ void tc_cp_128x128b(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 // Block-scaled MMAs, D[tmem] (+)= A[smem] * B[smem]^T with per-block scales in
@@ -252,20 +221,6 @@ __device__ __forceinline__ void mma_mxf8f6f4_sp(uint32_t d, uint64_t a, uint64_t
       : "memory");
 }
 
-// 32 lanes x 32 columns of 32-bit accumulator per warp (lane i <- TMEM lane
-// base+i), then wait for the load.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%"
-      "19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
-        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
 // The same 32-lane x 32-column load without the wait; tmem_ld_wait() completes it.
 __device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
@@ -309,31 +264,6 @@ __device__ __forceinline__ void cluster_sync_all() {
 // local arrive: no cluster-wide fence of this thread's outstanding stores).
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// mbar_wait for barriers that other CTAs of the cluster arrive on (acquire at cluster scope).
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint64_t timeout_ns,
-                                                  volatile int* abort = nullptr) {
-  if (mbar_try_wait_acq_cluster(bar, parity)) return true;
-  const uint64_t t0 = global_ns();
-  while (true) {
-    if (mbar_try_wait_acq_cluster(bar, parity)) return true;
-    if (abort && *abort) return false;
-    if (global_ns() - t0 > timeout_ns) {
-      atomicOr(&g_error_word, kErrTimeout);
-      return false;
-    }
-  }
 }
 // Tile load into this CTA's shared memory whose completion is counted on an
 // mbarrier of either CTA of the pair (a single destination CTA).
@@ -426,31 +356,6 @@ __host__ __device__ constexpr uint32_t desc_hi(uint32_t sbo, uint32_t layout) {
   return ((sbo >> 4) & 0x3FFF) | (1u << 14) | ((layout & 7u) << 29);
 }
 
-// Shared-memory matrix descriptor (K-major).  layout: 0 none, 2 128B swizzle,
-// 4 64B swizzle.  lbo/sbo in bytes.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
-  d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
-  d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
-  d |= (uint64_t)1 << 46;  // descriptor version for sm_100
-  d |= (uint64_t)(layout & 7) << 61;
-  return d;
-}
-
-// ------------------------------------------------------------- conversions
-// Two fp32 -> two E2M1 codes in one byte (lo in bits 0-3), round to nearest
-// even with saturation.
-__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
-  uint32_t out;
-  asm(
-      "{\n\t.reg .b8 t;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\t"
-      "cvt.u32.u8 %0, t;\n\t}"
-      : "=r"(out)
-      : "f"(lo), "f"(hi));
-  return out;
-}
 // Eight fp32 -> eight E2M1 codes packed in 32 bits (element i in nibble i).
 __device__ __forceinline__ uint32_t cvt_e2m1x8(const float* v) {
   uint32_t out;
@@ -464,12 +369,6 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(const float* v) {
       : "=r"(out)
       : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
   return out;
-}
-// Value of an E2M1 code (exact).
-__device__ __forceinline__ float e2m1_value(uint32_t code) {
-  const float mag = (float)((code & 4) ? ((code & 2) ? ((code & 1) ? 6 : 4) : ((code & 1) ? 3 : 2))
-                                       : ((code & 2) ? ((code & 1) ? 1.5f : 1.0f) : ((code & 1) ? 0.5f : 0.0f)));
-  return (code & 8) ? -mag : mag;
 }
 // fp32 -> E4M3 code (round to nearest even, saturate to 448).
 __device__ __forceinline__ uint32_t cvt_e4m3(float v) {

@@ -8,10 +8,13 @@ W 4096 x 4096), synthetic seeded data.  The weight is quantized once, outside
 the timed region (it is an offline step of the layer).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sharq|reference]
-                  [--workload NAME]
+                  [--workload NAME] [--tokens T]
 
 The default workload is q_proj; the others measure the remaining layer shapes
-the pages evaluate (one JSON line each, same keys).
+the pages evaluate (one JSON line each, same keys); --tokens sets the row count
+of the q_proj / down_proj shapes (the down_proj token sweep 1/16/64/256).  The
+step runs as one CUDA graph (the kernels chained by programmatic dependent
+launch); prep and GEMM are also timed alone for the roofline fields.
 
 Prints ONE JSON line (rank 0).  value = effective TFLOP/s = 2*T*N*K per step
 summed over ranks / max-over-ranks time; L2 is flushed (256 MB write) before
