@@ -477,7 +477,8 @@ def run_sharq(args):
         clocks = clk.summary()
         grouped = offsets is not None
         kernel = {"4:8pair": "sparse", "2:4": "sparse", "8:16": "dense backbone"}[pat]
-        kname = ("gemm_pair_kernel" if (not grouped and pat == "4:8pair" and ((T + 127) // 128 * 128) % 256 == 0)
+        kname = ("gemv_kernel" if (not grouped and T <= 4) else
+                 "gemm_pair_kernel" if (not grouped and pat == "4:8pair" and ((T + 127) // 128 * 128) % 256 == 0)
                  else "gemm_kernel")
         kkind = "MXF8" if (fmt == "mxfp4" and pat == "2:4") else ("NVF4" if fmt == "nvfp4" else "MXF4")
         out = {
