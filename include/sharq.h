@@ -76,7 +76,9 @@ typedef enum { SHARQ_F32 = 0, SHARQ_BF16 = 1 } sharq_dtype;
  * NVFP4) and carries two views of the same scales:
  *   codes          experts * n * k/2 bytes, row-major per expert;
  *   scales_dense   per expert, tiled scale layout, n rows, k/b scales (each 2b
- *                  scale stored twice) -- the view of the dense residual GEMM;
+ *                  scale stored twice) -- the view of the dense residual GEMM
+ *                  (the sparse-pattern GEMMs rebuild it on chip from
+ *                  scales_sparse; the 8:16 dense-backbone GEMM reads it);
  *   scales_sparse  per expert, tiled scale layout, n rows, k/(2b) scales;
  *   tensor         experts * 3 floats. */
 typedef struct {
