@@ -40,6 +40,7 @@ FP4_OVER_BF16 = 9.0 / 2.25          # nominal dense FP4 / dense BF16 ratio
 FP8_OVER_BF16 = 4.5 / 2.25          # nominal dense FP8 / dense BF16 ratio
 
 WORKLOADS = {
+    "tiny": "Tiny: X 16x256 fp32 ~N(0,1), channels 3 and 77 x40, W 256x256 ~N(0,0.02^2) fp32; no norm; MXFP4, 2:4",
     "q_proj": "Llama-3.1-8B q_proj: X 2048x4096 bf16 (0.5*t3 + 8 outlier channels x100), RMSNorm, W 4096x4096; "
               "NVFP4, 4:8 pair",
     "down_proj": "Llama-3.1-8B down_proj: X 2048x14336 bf16 = SiLU(a)*b, a,b ~N(0,1); W 4096x14336 ~N(0,0.01^2); "
@@ -75,7 +76,7 @@ def make_workload(name: str, tokens: int | None = None) -> dict:
         c = workloads.qwen_moe()
         t, k = c["x"].shape
         n = c["w_gu"].shape[1]
-        wl = dict(name=name, desc=WORKLOADS[name], x=c["x"], gamma=None, eps=1e-6, w=c["w_gu"], fmt="nvfp4",
+        wl = dict(name=name, desc=WORKLOADS[name], x=c["x"], x_dtype="bf16", gamma=None, eps=1e-6, w=c["w_gu"], fmt="nvfp4",
                   pat="4:8pair", offsets=c["offsets"], t=t, k=k, n=n, real_rows=int(c["counts"].sum()),
                   first_group=(int(c["offsets"][0]), int(c["offsets"][1])), gate=None, up=None)
         if name.endswith("_gather"):
@@ -83,10 +84,11 @@ def make_workload(name: str, tokens: int | None = None) -> dict:
         return wl
     kw = {"t": tokens} if tokens and name in ("q_proj", "down_proj", "down_proj_swiglu") else {}
     desc = WORKLOADS[name].replace("2048x", f"{tokens}x") if kw else WORKLOADS[name]
-    c = {"q_proj": workloads.q_proj, "down_proj": workloads.down_proj, "down_proj_swiglu": workloads.down_proj,
-         "wan": workloads.wan, "wan_816": lambda: workloads.wan(pat="8:16")}[name](**kw)
+    c = {"tiny": workloads.tiny, "q_proj": workloads.q_proj, "down_proj": workloads.down_proj,
+         "down_proj_swiglu": workloads.down_proj, "wan": workloads.wan,
+         "wan_816": lambda: workloads.wan(pat="8:16")}[name](**kw)
     t, k = c["x"].shape
-    wl = dict(name=name, desc=desc, x=c["x"], gamma=c["gamma"], eps=c["eps"], w=c["w"],
+    wl = dict(name=name, desc=desc, x=c["x"], x_dtype=c.get("x_dtype", "bf16"), gamma=c["gamma"], eps=c["eps"], w=c["w"],
               fmt=c["fmt"], pat=c["pat"], offsets=None, t=t, k=k, n=c["w"].shape[0], real_rows=t,
               first_group=None, gate=None, up=None)
     if name == "down_proj_swiglu":
@@ -116,6 +118,22 @@ def peaks():
 
 def dist_env():
     return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def max_over_ranks(values, dist=None, device="cpu"):
+    """Element-wise maximum of per-rank timings (one all_reduce(MAX)); the plain
+    values when there is no process group."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def replica_throughput(world: int, work_per_step: float, steps: int, ms: float) -> float:
+    """Whole-job throughput of N replicas in units of 1e12 per second: every rank
+    did work_per_step per step; ms is the max-over-ranks time of the steps."""
+    return world * work_per_step * steps / (ms / 1e3) / 1e12
 
 
 class ClockSampler:
@@ -249,6 +267,7 @@ def cpu_baseline(name: str = "q_proj", rows: int = 2048, tokens: int | None = No
     dt = time.perf_counter() - t0
     assert np.isfinite(y).all()
     value = 2.0 * rows * wl["n"] * wl["k"] / dt / 1e12
+    _ORACLE_SETUP["rows_used"] = rows
     return {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "sample": f"{rows} of {wl['t']} rows: tensor amax over all rows, prep of those rows with {cores} threads, "
                       f"fp64 numpy GEMM of those rows ({dt:.2f} s)"}, dt
@@ -277,12 +296,13 @@ def run_sharq(args):
     swiglu = wl["gate"] is not None
     gathered = wl.get("gather") is not None  # prep of the tokens, then their prepared rows gathered
     x_src = wl["gate"] if swiglu else (wl["tokens"] if gathered else wl["x"])
-    x_host = torch.from_numpy(x_src).to(torch.bfloat16).pin_memory()
+    x_dt = torch.float32 if wl.get("x_dtype") == "f32" else torch.bfloat16  # the workload's input dtype
+    x_host = torch.from_numpy(x_src).to(x_dt).pin_memory()
     x = x_host.to(dev)
     up_host = torch.from_numpy(wl["up"]).to(torch.bfloat16).pin_memory() if swiglu else None
     up = up_host.to(dev) if swiglu else None
     gamma = torch.from_numpy(wl["gamma"]).to(torch.bfloat16).to(dev) if wl["gamma"] is not None else None
-    w = torch.from_numpy(wl["w"]).to(torch.bfloat16).to(dev)
+    w = torch.from_numpy(wl["w"]).to(x_dt).to(dev)
     wq = sharq.FP4Weight.quantize(w, fmt)
     del w
     offsets = torch.from_numpy(wl["offsets"]).to(torch.int32).to(dev) if wl["offsets"] is not None else None
@@ -451,15 +471,12 @@ def run_sharq(args):
     e2e_ms = e_start.elapsed_time(e_end)
     sharq.sharq_sync_status()
 
-    times = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if pg:
-        pg.all_reduce(times, op=pg.ReduceOp.MAX)
-    total_ms, e2e_ms = times.tolist()
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], pg, dev)
 
     if rank == 0:
         pk, src = peaks()
         flops = 2.0 * wl["real_rows"] * N * K
-        value = world * flops * args.steps / (total_ms / 1e3) / 1e12
+        value = replica_throughput(world, flops, args.steps, total_ms)
         gemm_avg = statistics.mean(gemm_ms) / 1e3
         work, kind, work_desc = gemm_roofline(wl)
         b_blk = 16 if fmt == "nvfp4" else 32
@@ -468,7 +485,7 @@ def run_sharq(args):
         ratio = FP4_OVER_BF16 if kind == "fp4" else FP8_OVER_BF16
         peak = pk["bf16_tflops"] * ratio
         achieved = work / gemm_avg / 1e12
-        bpe = prep_bytes_per_elem(fmt, pat, 4 if swiglu else 2)
+        bpe = prep_bytes_per_elem(fmt, pat, 4 if (swiglu or x_dt == torch.float32) else 2)
         prep_bytes = bpe * T * K
         if gathered:  # prep of the tokens, then each routed row's prepared bytes read and written once
             prep_bytes = bpe * x_host.shape[0] * K + 2 * (bpe - 2) * T * K + 4 * T
@@ -518,10 +535,10 @@ def run_sharq(args):
                      "frac_device_amax": round(prep_gbs / pk["hbm_gbs"], 4),
                      "bytes_per_elem": bpe, "avg_us": round(statistics.mean(prep_ms) * 1e3, 2),
                      "avg_us_given_amax": round(prep_given_ms * 1e3, 2)},
-            "e2e": {"value": round(world * flops * args.steps / (e2e_ms / 1e3) / 1e12, 3), "unit": "TFLOP/s",
+            "e2e": {"value": round(replica_throughput(world, flops, args.steps, e2e_ms), 3), "unit": "TFLOP/s",
                     "mode": "public API per step (pinned host x in, y out), steps pipelined on copy-in / compute / "
                             "copy-out streams with double buffers",
-                    "h2d_bytes_per_step": int(x_host.numel() * 2 * (2 if swiglu else 1)
+                    "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size() * (2 if swiglu else 1)
                                               + (rows_host.numel() * 4 if gathered else 0)),
                     "d2h_bytes_per_step": int(y_host.numel() * 2)},
             "gpu_launches": int(launches),
@@ -556,6 +573,7 @@ def run_reference(args):
         base, dt = cpu_baseline(args.workload, rows, args.tokens)
         times.append(dt)
     wl = _ORACLE_SETUP["wl"]
+    rows = _ORACLE_SETUP["rows_used"]  # the sample (all rows of a smaller workload)
     total = sum(times)
     value = 2.0 * rows * wl["n"] * wl["k"] * args.steps / total / 1e12
     base["value"] = value
