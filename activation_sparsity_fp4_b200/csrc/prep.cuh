@@ -301,14 +301,25 @@ struct RowMap {
   int tpr;    // threads per row
   int lg;     // log2(tpr)
   int units;  // units (32 elements) per row
-  int nj;     // units per thread, <= 4
+  int nj;     // units per thread, <= 8
 };
+
+// Threads per row for a row of `units` 32-element units: the largest power of
+// two in 8..128 that divides the units with at most 8 per thread, so that no
+// thread of a row idles (5120 = 160 units: 32 threads x 5; 14336 = 448 units:
+// 64 x 7); otherwise the smallest power of two covering them in <= 4 per thread.
+__host__ __device__ __forceinline__ int rows_tpr(int64_t units) {
+  for (int c = 128; c >= 8; c >>= 1)
+    if (units % c == 0 && units / c <= 8) return c;
+  int tpr = 8;
+  while (tpr < units && tpr < 128) tpr <<= 1;
+  return tpr;
+}
 
 __device__ __forceinline__ RowMap row_map(int64_t k) {
   RowMap m;
   m.units = (int)(k / 32);
-  int tpr = 8;
-  while (tpr < m.units && tpr < 128) tpr <<= 1;
+  const int tpr = rows_tpr(m.units);
   m.tpr = tpr;
   m.lg = 31 - __clz(tpr);
   m.nj = (m.units + tpr - 1) / tpr;
@@ -325,10 +336,10 @@ __device__ __forceinline__ RowMap row_map(int64_t k) {
 template <bool XBF16>
 __device__ __forceinline__ float row_sumsq(const void* x, int64_t row_off, bool real, const RowMap& m, int t,
                                            int row_in_block, float* red /* [32 rows][4 warps][4 j] */) {
-  float s[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  float s[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
   const int wlanes = m.tpr < 32 ? m.tpr : 32;
 #pragma unroll
-  for (int j = 0; j < 4; j++) {
+  for (int j = 0; j < 8; j++) {
     if (j < m.nj) {
       const int u = t + m.tpr * j;
       float c0 = 0.0f, c1 = 0.0f;
@@ -349,22 +360,23 @@ __device__ __forceinline__ float row_sumsq(const void* x, int64_t row_off, bool 
     const int w = t >> 5, nw = m.tpr >> 5;
     if ((t & 31) == 0) {
 #pragma unroll
-      for (int j = 0; j < 4; j++) red[(row_in_block * 4 + w) * 4 + j] = s[j];
+      for (int j = 0; j < 8; j++) red[(row_in_block * 4 + w) * 8 + j] = s[j];
     }
     __syncthreads();
 #pragma unroll
-    for (int j = 0; j < 4; j++) {
-      const float w0 = red[(row_in_block * 4 + 0) * 4 + j], w1 = red[(row_in_block * 4 + 1) * 4 + j];
+    for (int j = 0; j < 8; j++) {
+      const float w0 = red[(row_in_block * 4 + 0) * 8 + j], w1 = red[(row_in_block * 4 + 1) * 8 + j];
       if (nw == 2) {
         s[j] = __fadd_rn(w0, w1);
       } else {
-        const float w2 = red[(row_in_block * 4 + 2) * 4 + j], w3 = red[(row_in_block * 4 + 3) * 4 + j];
+        const float w2 = red[(row_in_block * 4 + 2) * 8 + j], w3 = red[(row_in_block * 4 + 3) * 8 + j];
         s[j] = __fadd_rn(__fadd_rn(w0, w1), __fadd_rn(w2, w3));
       }
     }
     __syncthreads();
   }
-  return __fadd_rn(__fadd_rn(s[0], s[1]), __fadd_rn(s[2], s[3]));
+  return __fadd_rn(__fadd_rn(__fadd_rn(s[0], s[1]), __fadd_rn(s[2], s[3])),
+                   __fadd_rn(__fadd_rn(s[4], s[5]), __fadd_rn(s[6], s[7])));
 }
 
 __device__ __forceinline__ float rstd_from_sumsq(float sumsq, int64_t k, float eps) {

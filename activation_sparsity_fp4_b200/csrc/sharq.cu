@@ -208,9 +208,7 @@ unsigned row_grid(Kern kern, int64_t rows, int64_t k) {
   if (per_sm == 0) {
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 128, 0) != cudaSuccess || per_sm < 1) per_sm = 1;
   }
-  int tpr = 8;
-  while (tpr < k / 32 && tpr < 128) tpr <<= 1;
-  const int64_t rpb = 128 / tpr;
+  const int64_t rpb = 128 / rows_tpr(k / 32);
   const int64_t groups = (rows + rpb - 1) / rpb;
   const int64_t cap = (int64_t)sm_count() * per_sm;
   return (unsigned)(groups < cap ? groups : cap);
