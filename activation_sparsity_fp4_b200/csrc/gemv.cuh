@@ -179,24 +179,33 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 2) gemv_kernel(const GemvPara
   for (int j = 0; j < R; j++) nr[j] = n0 + j < p.n ? n0 + j : p.n - 1;
   const bool live = n0 < p.n;
 
-  if (lane < R && n0 + lane < p.n) prefetch_l2(p.w_codes + (n0 + lane) * (p.k / 2), (uint32_t)(p.k / 2));
-  if (threadIdx.x == 0 && (((int64_t)blockIdx.x * kGemvWarps * R) & 127) == 0) {  // scales of this 128-row block
+  if (live && lane < R && n0 + lane < p.n) prefetch_l2(p.w_codes + (n0 + lane) * (p.k / 2), (uint32_t)(p.k / 2));
+  if (live && lane == 0 && (n0 & 127) == 0) {  // the first row of a 128-row block: that block's scales
     const int64_t sblocks = (ws + 3) >> 2;
     prefetch_l2(p.w_sf + (n0 >> 7) * sblocks * 512, (uint32_t)(sblocks * 512));
   }
   grid_dep_wait();  // the prepared rows are complete
 
-  uint4 wc[kUpl][R], wn[kUpl][R];
-  uint32_t sc[kUpl][R], sn[kUpl][R];
+  // per weight row: its code row and the row part of its tiled scale offsets
+  const int64_t sblocks = (ws + 3) >> 2;
+  const uint4* wrow[R];
+  int64_t srow[R];
+#pragma unroll
+  for (int j = 0; j < R; j++) {
+    wrow[j] = reinterpret_cast<const uint4*>(p.w_codes + nr[j] * (p.k / 2));
+    srow[j] = (nr[j] >> 7) * sblocks * 512 + (nr[j] & 31) * 16 + ((nr[j] >> 5) & 3) * 4;
+  }
   auto load_w = [&](int64_t c, uint4 (&codes)[kUpl][R], uint32_t (&scl)[kUpl][R]) {
 #pragma unroll
     for (int i = 0; i < kUpl; i++) {
       const int64_t u = c * kUnits + lane + 32 * i;
+      const int64_t cs = FMT == FMT_NV ? u : u >> 1;  // sparse-view scale column
+      const int64_t scol = (cs >> 2) * 512 + (cs & 3);
 #pragma unroll
       for (int j = 0; j < R; j++) {
         if (live && u < ku) {  // the weight stream: read once, bypassing L1
-          codes[i][j] = __ldcs(reinterpret_cast<const uint4*>(p.w_codes + nr[j] * (p.k / 2)) + u);
-          scl[i][j] = __ldg(p.w_sf + tiled_sf_offset(nr[j], FMT == FMT_NV ? u : u >> 1, ws));
+          codes[i][j] = __ldcs(wrow[j] + u);
+          scl[i][j] = __ldg(p.w_sf + srow[j] + scol);
         } else {
           codes[i][j] = make_uint4(0, 0, 0, 0);
           scl[i][j] = 0;
@@ -207,25 +216,30 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 2) gemv_kernel(const GemvPara
   // decode slots of a chunk: (row, unit, quarter), quarters of a unit on neighbouring threads
   constexpr int kSlotsTotal = T * kUnits * 4;
   constexpr int kSlots = (kSlotsTotal + kGemvWarps * 32 - 1) / (kGemvWarps * 32);
-  auto slot_valid = [&](int64_t c, int sl) {
-    const int s = (int)threadIdx.x + sl * kGemvWarps * 32;
-    return s < kSlotsTotal && c * kUnits + (s % (kUnits * 4)) / 4 < ku;
-  };
+  int xrow[kSlots], xunit[kSlots], xq[kSlots];
+  bool xon[kSlots];
+#pragma unroll
+  for (int sl = 0; sl < kSlots; sl++) {
+    const int s = (int)threadIdx.x + sl * kGemvWarps * 32, rem = s % (kUnits * 4);
+    xon[sl] = s < kSlotsTotal;
+    xrow[sl] = s / (kUnits * 4);
+    xunit[sl] = rem >> 2;
+    xq[sl] = rem & 3;
+  }
   auto load_x = [&](int64_t c, GemvQuarterRaw (&raw)[kSlots]) {
 #pragma unroll
-    for (int sl = 0; sl < kSlots; sl++) {
-      const int s = (int)threadIdx.x + sl * kGemvWarps * 32, rem = s % (kUnits * 4);
-      if (slot_valid(c, sl)) gemv_load_quarter<FMT, PAT>(p, s / (kUnits * 4), c * kUnits + rem / 4, rem & 3, raw[sl]);
-    }
+    for (int sl = 0; sl < kSlots; sl++)
+      if (xon[sl] && c * kUnits + xunit[sl] < ku)
+        gemv_load_quarter<FMT, PAT>(p, xrow[sl], c * kUnits + xunit[sl], xq[sl], raw[sl]);
   };
   auto store_x = [&](int64_t c, int buf, const GemvQuarterRaw (&raw)[kSlots]) {
 #pragma unroll
     for (int sl = 0; sl < kSlots; sl++) {
-      if (!slot_valid(c, sl)) continue;
-      const int s = (int)threadIdx.x + sl * kGemvWarps * 32, rem = s % (kUnits * 4), uu = rem / 4, q = rem & 3;
+      if (!(xon[sl] && c * kUnits + xunit[sl] < ku)) continue;
+      const int uu = xunit[sl], q = xq[sl];
       float v[8];
       gemv_decode_quarter<FMT, PAT>(p, raw[sl], v);
-      float4* d = reinterpret_cast<float4*>(&xs[buf][s / (kUnits * 4)][32 * uu]);
+      float4* d = reinterpret_cast<float4*>(&xs[buf][xrow[sl]][32 * uu]);
       // 16-byte groups XOR-swizzled by the unit: lanes on different units hit different banks
       d[(2 * q) ^ (uu & 7)] = make_float4(v[0], v[1], v[2], v[3]);
       d[(2 * q + 1) ^ (uu & 7)] = make_float4(v[4], v[5], v[6], v[7]);
@@ -238,23 +252,17 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 2) gemv_kernel(const GemvPara
 #pragma unroll
     for (int r = 0; r < T; r++) acc[j][r] = 0.0f;
 
-  load_w(0, wc, sc);
-  {
-    GemvQuarterRaw raw[kSlots];
-    load_x(0, raw);
-    store_x(0, 0, raw);
-  }
-  __syncthreads();
-
-  for (int64_t c = 0; c < nchunks; c++) {
+  // one chunk: request chunk c + 1 (weights into nxt, activation bytes), products
+  // of chunk c from cur and shared-memory buffer c & 1, then decode chunk c + 1
+  auto step = [&](int64_t c, const uint4 (&cur)[kUpl][R], const uint32_t (&scur)[kUpl][R], uint4 (&nxt)[kUpl][R],
+                  uint32_t (&snxt)[kUpl][R]) {
     const int buf = (int)(c & 1);
     const bool more = c + 1 < nchunks;
     GemvQuarterRaw raw[kSlots];
     if (more) {
-      load_w(c + 1, wn, sn);
+      load_w(c + 1, nxt, snxt);
       load_x(c + 1, raw);
     }
-
     if (live) {
 #pragma unroll
       for (int i = 0; i < kUpl; i++) {
@@ -276,7 +284,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 2) gemv_kernel(const GemvPara
           }
 #pragma unroll
           for (int j = 0; j < R; j++) {
-            const uint32_t word = w == 0 ? wc[i][j].x : w == 1 ? wc[i][j].y : w == 2 ? wc[i][j].z : wc[i][j].w;
+            const uint32_t word = w == 0 ? cur[i][j].x : w == 1 ? cur[i][j].y : w == 2 ? cur[i][j].z : cur[i][j].w;
             uint64_t wv[4];
             e2m1x8_pairs(word, wv);
 #pragma unroll
@@ -287,7 +295,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 2) gemv_kernel(const GemvPara
         }
 #pragma unroll
         for (int j = 0; j < R; j++) {
-          const float wsv = scale_value<FMT>(sc[i][j]);
+          const float wsv = scale_value<FMT>(scur[i][j]);
 #pragma unroll
           for (int r = 0; r < T; r++) {
             const float even = __uint_as_float((uint32_t)part[j][r]), odd = __uint_as_float((uint32_t)(part[j][r] >> 32));
@@ -298,13 +306,20 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 2) gemv_kernel(const GemvPara
     }
     if (more) store_x(c + 1, buf ^ 1, raw);
     __syncthreads();  // chunk c + 1 decoded; chunk c's buffer free for chunk c + 2
-#pragma unroll
-    for (int i = 0; i < kUpl; i++)
-#pragma unroll
-      for (int j = 0; j < R; j++) {
-        wc[i][j] = wn[i][j];
-        sc[i][j] = sn[i][j];
-      }
+  };
+
+  uint4 wa[kUpl][R], wb[kUpl][R];  // weight codes of the current and the next chunk (ping-pong)
+  uint32_t sa[kUpl][R], sb[kUpl][R];
+  load_w(0, wa, sa);
+  {
+    GemvQuarterRaw raw[kSlots];
+    load_x(0, raw);
+    store_x(0, 0, raw);
+  }
+  __syncthreads();
+  for (int64_t c = 0; c < nchunks; c += 2) {
+    step(c, wa, sa, wb, sb);
+    if (c + 1 < nchunks) step(c + 1, wb, sb, wa, sa);
   }
   if (!live) return;
   const float alpha = __fmul_rn(__ldg(p.tensor_x + 2), __ldg(p.tensor_w + 2));
