@@ -47,6 +47,7 @@ struct PrepParams {
   float* tensor;     // [amax, g_enc, g_dec]
   float act_amax;    // > 0: given by the caller
   const float* rstd; // per-row RMSNorm factors from the amax pass, or null
+  int tpr;           // threads per row (a power of two, 8..128, set by the launcher)
 };
 
 // ------------------------------------------------------------- loading
@@ -316,10 +317,17 @@ __host__ __device__ __forceinline__ int rows_tpr(int64_t units) {
   return tpr;
 }
 
-__device__ __forceinline__ RowMap row_map(int64_t k) {
+// Few rows (all of them resident at once as one row per block) take 128 threads
+// per row whenever that leaves at most 8 units per thread: the least serial work
+// per thread.  The reductions are the same fixed tree for every power-of-two tpr.
+__host__ __device__ __forceinline__ int rows_tpr(int64_t units, int64_t rows, int64_t resident_blocks) {
+  if (rows <= resident_blocks && units >= 128 && units <= 8 * 128) return 128;
+  return rows_tpr(units);
+}
+
+__device__ __forceinline__ RowMap row_map(int64_t k, int tpr) {
   RowMap m;
   m.units = (int)(k / 32);
-  const int tpr = rows_tpr(m.units);
   m.tpr = tpr;
   m.lg = 31 - __clz(tpr);
   m.nj = (m.units + tpr - 1) / tpr;
@@ -407,12 +415,12 @@ __device__ __forceinline__ void sub2(float& a, float& b, float c, float d) {  //
 // amax_out[0] (zeroed beforehand) with one atomic per block.
 template <bool NORM, bool XBF16, bool ACT = false>
 __global__ void __launch_bounds__(128) amax_kernel(const void* x, const void* gamma, float eps, int64_t t, int64_t k,
-                                                   float* amax_out, float* rstd_out, const void* x2 = nullptr) {
+                                                   float* amax_out, float* rstd_out, const void* x2, int tpr) {
   static_assert(!(NORM && ACT), "the SwiGLU form has no RMSNorm");
   __shared__ float red[32 * 16];
   __shared__ float wmax[4];
   grid_dep_launch();
-  const RowMap m = row_map(k);
+  const RowMap m = row_map(k, tpr);
   const int rpb = 128 / m.tpr;
   const int row_in_block = threadIdx.x >> m.lg, tt = threadIdx.x & (m.tpr - 1);
   float my = 0.0f;
@@ -728,7 +736,7 @@ __global__ void __launch_bounds__(128, ACT ? 6 : 7) prep_kernel(PrepParams p) {
   __shared__ float inv_tab[128];
   __shared__ float red[32 * 16];
   const int64_t k = p.k;
-  const RowMap m = row_map(k);
+  const RowMap m = row_map(k, p.tpr);
   const int rpb = 128 / m.tpr;
   const int row_in_block = threadIdx.x >> m.lg, tt = threadIdx.x & (m.tpr - 1);
   grid_dep_wait();    // the amax pass (or whatever wrote x) has completed

@@ -202,22 +202,30 @@ sharq_status check_shape(int64_t k, int64_t n_or_t, bool is_n) {
 // ---------------------------------------------------------------- launchers
 // Blocks of 128 threads handle 128 / tpr rows at a time (tpr threads per row,
 // see RowMap); as many resident blocks as the SMs hold, striding over rows.
+struct RowLaunch {
+  unsigned grid;
+  int tpr;
+};
 template <typename Kern>
-unsigned row_grid(Kern kern, int64_t rows, int64_t k) {
+RowLaunch row_launch(Kern kern, int64_t rows, int64_t k) {
   static int per_sm = 0;
   if (per_sm == 0) {
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 128, 0) != cudaSuccess || per_sm < 1) per_sm = 1;
   }
-  const int64_t rpb = 128 / rows_tpr(k / 32);
-  const int64_t groups = (rows + rpb - 1) / rpb;
   const int64_t cap = (int64_t)sm_count() * per_sm;
-  return (unsigned)(groups < cap ? groups : cap);
+  const int tpr = rows_tpr(k / 32, rows, cap);
+  const int64_t rpb = 128 / tpr;
+  const int64_t groups = (rows + rpb - 1) / rpb;
+  return RowLaunch{(unsigned)(groups < cap ? groups : cap), tpr};
 }
 
 template <int FMT, int PAT, bool NORM, bool XBF16>
 sharq_status launch_prep(const PrepParams& pp, cudaStream_t s) {
   auto kern = prep_kernel<FMT, PAT, NORM, XBF16>;
-  return launch_ex(kern, dim3(row_grid(kern, pp.t_pad, pp.k)), dim3(128), 0, s, 1, pp);
+  const RowLaunch rl = row_launch(kern, pp.t_pad, pp.k);
+  PrepParams q = pp;
+  q.tpr = rl.tpr;
+  return launch_ex(kern, dim3(rl.grid), dim3(128), 0, s, 1, q);
 }
 
 template <bool NORM, bool XBF16>
@@ -228,7 +236,8 @@ sharq_status launch_amax(const void* x, const void* gamma, float eps, int64_t t,
     return launched();
   }
   auto kern = amax_kernel<NORM, XBF16>;
-  kern<<<row_grid(kern, t, k), 128, 0, s>>>(x, gamma, eps, t, k, out, rstd_out, nullptr);
+  const RowLaunch rl = row_launch(kern, t, k);
+  kern<<<rl.grid, 128, 0, s>>>(x, gamma, eps, t, k, out, rstd_out, nullptr, rl.tpr);
   return launched();
 }
 
@@ -253,7 +262,10 @@ sharq_status prep_dispatch_p(const PrepParams& pp, int pat, bool norm, bool xbf1
 template <int FMT, int PAT, bool XBF16>
 sharq_status launch_prep_swiglu(const PrepParams& pp, cudaStream_t s) {
   auto kern = prep_kernel<FMT, PAT, false, XBF16, true>;
-  return launch_ex(kern, dim3(row_grid(kern, pp.t_pad, pp.k)), dim3(128), 0, s, 1, pp);
+  const RowLaunch rl = row_launch(kern, pp.t_pad, pp.k);
+  PrepParams q = pp;
+  q.tpr = rl.tpr;
+  return launch_ex(kern, dim3(rl.grid), dim3(128), 0, s, 1, q);
 }
 template <int FMT, int PAT>
 sharq_status swiglu_dispatch_x(const PrepParams& pp, bool xbf16, cudaStream_t s) {
@@ -270,7 +282,8 @@ sharq_status swiglu_dispatch_p(const PrepParams& pp, int pat, bool xbf16, cudaSt
 template <bool XBF16>
 sharq_status launch_amax_swiglu(const void* gate, const void* up, int64_t t, int64_t k, float* out, cudaStream_t s) {
   auto kern = amax_kernel<false, XBF16, true>;
-  kern<<<row_grid(kern, t, k), 128, 0, s>>>(gate, nullptr, 0.0f, t, k, out, nullptr, up);
+  const RowLaunch rl = row_launch(kern, t, k);
+  kern<<<rl.grid, 128, 0, s>>>(gate, nullptr, 0.0f, t, k, out, nullptr, up, rl.tpr);
   return launched();
 }
 
