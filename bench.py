@@ -498,6 +498,8 @@ def run_sharq(args):
                  "gemm_pair_kernel" if (not grouped and pat == "4:8pair" and ((T + 127) // 128 * 128) % 256 == 0)
                  else "gemm_kernel")
         kkind = "MXF8" if (fmt == "mxfp4" and pat == "2:4") else ("NVF4" if fmt == "nvfp4" else "MXF4")
+        klabel = (f"gemv_kernel<{'MX' if fmt == 'mxfp4' else 'NV'}, {pat}, {T} rows>" if kname == "gemv_kernel"
+                  else f"{kname}<{kkind}, {kernel}>")
         out = {
             "metric": METRIC,
             "value": round(value, 2),
@@ -516,7 +518,7 @@ def run_sharq(args):
                        "norm": "rmsnorm" if gamma is not None else "none", "y_dtype": "bf16",
                        "parallelism": f"replicas x{world}",
                        "l2": "flushed (256 MB write) before every timed step"},
-            "roofline": ({"bound": "tensor", "kernel": f"{kname}<{kkind}, {kernel}>",
+            "roofline": ({"bound": "tensor", "kernel": klabel,
                           "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
                           "frac": round(achieved / peak, 4),
                           "traffic": committed_traffic() if args.workload == "q_proj" and not args.tokens else None,
@@ -524,7 +526,7 @@ def run_sharq(args):
                           "work": work_desc, "avg_launch_us": round(gemm_avg * 1e6, 2)}
                          if T > 64 else
                          # decode-size rows: the GEMM streams the weight; HBM bound
-                         {"bound": "hbm", "kernel": f"{kname}<{kkind}, {kernel}>",
+                         {"bound": "hbm", "kernel": klabel,
                           "achieved": round(wbytes / gemm_avg / 1e9, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                           "frac": round(wbytes / gemm_avg / 1e9 / pk["hbm_gbs"], 4), "traffic": None,
                           "peak_source": src,
