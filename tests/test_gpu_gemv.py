@@ -29,7 +29,7 @@ def _x(seed, t, k):
 @pytest.mark.parametrize("fmt,pat", CASES)
 @pytest.mark.parametrize("t", [1, 2, 3, 4])
 def test_gemv_matches_oracle(cuda_ok, fmt, pat, t):
-    k, n = 2304, 512  # two K chunks of 2048 and a partial one; 32 warps of 4 weight rows
+    k, n = 2304, 512  # K chunks of 2048 (1-2 rows) or 1024 (3-4 rows) and a partial one; 32 blocks of 8 warps x 2 rows
     x, w = _x(50 + t, t, k), _w(51, n, k)
     p = gpu_prepare(x, "bf16", fmt, pat)
     wq = sharq.FP4Weight.quantize(to_dev(w, "bf16"), fmt)
