@@ -4,8 +4,10 @@
 // the sparse backbone product plus the dense residual product into one output,
 // both reading the one FP4 weight.  With at most kGemvMaxRows rows the work is
 // a weight stream (N*K/2 bytes of codes) with a few multiply-adds per byte, so
-// it runs on the CUDA cores, bound by HBM: a 128-row tensor-core tile would be
-// at least 97 % padding and its K loop latency bound.
+// it runs on the CUDA cores: a 128-row tensor-core tile would be at least 97 %
+// padding and its K loop latency bound.  Each weight element costs its E2M1 ->
+// fp32 widening and half a packed FMA, so instruction issue, not HBM, is the
+// limit at one row.
 //
 // Each block decodes the rows' backbone and residual (codes, metadata and block
 // scales, without the tensor scale) one K chunk at a time into shared memory as
