@@ -59,3 +59,17 @@ def test_gemv_down_proj_decode(cuda_ok, t):
     sharq.sharq_sync_status()
     ref = oracle.linear_ref(oracle.prepare(cfg["x"], "mxfp4", "2:4"), oracle.quantize_weight(cfg["w"], "mxfp4"))
     assert_close_gemm(y.cpu().numpy(), ref, f"down_proj t={t}")
+
+
+@pytest.mark.parametrize("fmt,pat", [("nvfp4", "4:8pair"), ("mxfp4", "2:4"), ("nvfp4", "8:16")])
+@pytest.mark.parametrize("k,n", [(256, 256), (768, 512)])
+@pytest.mark.parametrize("t", [1, 3])
+def test_gemv_short_rows(cuda_ok, fmt, pat, k, n, t):
+    """Rows shorter than one K chunk: a single partial chunk, most lanes without a unit."""
+    x, w = _x(60 + t, t, k), _w(61, n, k)
+    p = gpu_prepare(x, "bf16", fmt, pat)
+    wq = sharq.FP4Weight.quantize(to_dev(w, "bf16"), fmt)
+    y = sharq.linear(p, wq, out_dtype=torch.float32)
+    sharq.sharq_sync_status()
+    ref = oracle.linear_ref(oracle.prepare(x, fmt, pat), oracle.quantize_weight(w, fmt))
+    assert_close_gemm(y.cpu().numpy(), ref, f"gemv short {fmt} {pat} k={k} t={t}")
