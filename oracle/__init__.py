@@ -71,6 +71,7 @@ def _load():
             "orc_rows_amax": (F, [P, I64, I64, P, F]),
             "orc_tensor_scale": (None, [F, P, P]),
             "orc_quant_block": (ctypes.c_uint8, [P, I, I, F, P]),
+            "orc_quant_blocks_n": (None, [P, I64, I, I, F, P, P]),
             "orc_prepare": (I, [P, I64, I64, P, F, I, I, F, P, P, P, P, P, P, P, P, P]),
             "orc_quantize_weight": (I, [P, I64, I64, I, P, P, P]),
             "orc_decode_prepared": (None, [P, P, P, P, P, I64, I64, I, I, P, P]),
@@ -173,6 +174,28 @@ def quant_block(v, fmt, g_enc: float = 1.0):
     codes = np.empty(v.size, np.uint8)
     sc = _load().orc_quant_block(_ptr(v), v.size, _fmt(fmt), g_enc, _ptr(codes))
     return int(sc), codes
+
+
+def quant_blocks(v, block: int, fmt, g_enc: float = 1.0):
+    """Consecutive blocks of ``block`` values along the last axis, each with its own
+    scale: (scale codes [..., n / block], E2M1 codes [..., n])."""
+    v = _f32(v)
+    flat = v.reshape(-1)
+    assert flat.size % block == 0
+    codes = np.empty(flat.size, np.uint8)
+    scales = np.empty(flat.size // block, np.uint8)
+    _load().orc_quant_blocks_n(_ptr(flat), flat.size // block, block, _fmt(fmt), g_enc, _ptr(codes), _ptr(scales))
+    return scales.reshape(v.shape[:-1] + (v.shape[-1] // block,)), codes.reshape(v.shape)
+
+
+def dequant_blocks(scales, codes, fmt, g_dec: float = 1.0) -> np.ndarray:
+    """fp64 values of quant_blocks' output: E2M1 * block scale (exact) * g_dec."""
+    lib = _load()
+    e2 = np.array([lib.orc_e2m1_decode(c) for c in range(16)], np.float64)
+    dec = lib.orc_e8m0_decode if _fmt(fmt) == MXFP4 else lib.orc_e4m3_decode
+    sv = np.array([dec(c) for c in range(256)], np.float64)
+    block = codes.shape[-1] // scales.shape[-1]
+    return e2[codes] * np.repeat(sv[scales], block, axis=-1) * (1.0 if _fmt(fmt) == MXFP4 else float(g_dec))
 
 
 def meta_bytes_per_row(k: int, pat) -> int:

@@ -281,9 +281,11 @@ void orc_tensor_scale(float amax, float* g_enc, float* g_dec) {
  * Quantize n values that share one scale.  Writes n E2M1 codes, returns the
  * scale code.  MXFP4 (OCP MX rule): e = floor(log2 amax) - 2 clamped to
  * [-127, 127] (amax = 0 gives -127), code = e + 127, element = E2M1(v * 2^-e).
- * NVFP4: s = amax * c with the per-tensor constant c = g_enc / 6 (the two
- * scalings folded into one rounding per block), S = E4M3(s); if S is 0 every
- * code is +0, else element = E2M1(v * (g_enc / S)).                          */
+ * NVFP4: s = (amax / 6) * g_enc, each step rounded once: amax / 6 is the
+ * block's decode scale (the largest E2M1 magnitude, 6, lands on the block
+ * amax), and multiplying by g_enc expresses it in units of the tensor's decode
+ * scale g_dec = 1 / g_enc, the form its E4M3 code stores.  S = E4M3(s); if S
+ * is 0 every code is +0, else element = E2M1(v * (g_enc / S)).               */
 uint8_t orc_quant_block(const float* v, int n, int fmt, float g_enc, uint8_t* codes) {
   float amax = 0.0f;
   for (int i = 0; i < n; i++) amax = fmaxf(amax, fabsf(v[i]));
@@ -295,8 +297,7 @@ uint8_t orc_quant_block(const float* v, int n, int fmt, float g_enc, uint8_t* co
     for (int i = 0; i < n; i++) codes[i] = orc_e2m1_encode(v[i] * mul);
     return (uint8_t)(e + 127);
   }
-  const float c6 = g_enc / 6.0f;
-  float s32 = amax * c6;
+  float s32 = (amax / 6.0f) * g_enc;
   uint8_t sc = orc_e4m3_encode(s32);
   float sv = orc_e4m3_decode(sc);
   if (sv == 0.0f) {
@@ -542,6 +543,12 @@ void orc_e2m1_encode_n(const float* v, int64_t n, uint8_t* out) {
 }
 void orc_e4m3_encode_n(const float* v, int64_t n, uint8_t* out) {
   for (int64_t i = 0; i < n; i++) out[i] = orc_e4m3_encode(v[i]);
+}
+/* Consecutive blocks of bs values, each quantized by orc_quant_block (codes one
+ * per byte, one scale code per block). */
+void orc_quant_blocks_n(const float* v, int64_t nblocks, int bs, int fmt, float g_enc, uint8_t* codes,
+                        uint8_t* scales) {
+  for (int64_t i = 0; i < nblocks; i++) scales[i] = orc_quant_block(v + i * bs, bs, fmt, g_enc, codes + i * bs);
 }
 void orc_floor_log2_n(const float* v, int64_t n, int32_t* out) {
   for (int64_t i = 0; i < n; i++) out[i] = orc_floor_log2(v[i]);

@@ -76,8 +76,8 @@ def _window_scale_codes(h, fmt, b, g_enc):
                 e = (math.frexp(amax)[1] - 1 - 2) if amax > 0 else -127
                 out[r, w] = max(-127, min(127, e)) + 127
             else:
-                c6 = np.float32(np.float32(g_enc) / np.float32(6.0))
-                out[r, w] = oracle.e4m3_encode([np.float32(np.float32(amax) * c6)])[0]
+                d = np.float32(np.float32(amax) / np.float32(6.0))
+                out[r, w] = oracle.e4m3_encode([np.float32(d * np.float32(g_enc))])[0]
     return out
 
 
