@@ -246,19 +246,34 @@ __device__ __forceinline__ float pow2f(int e) {  // exact 2^e for e in [-127, 12
   return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(0x00400000u);
 }
 
+// amax / 6 rounded to nearest (the block's decode scale before the tensor
+// scale: the largest E2M1 magnitude, 6, is mapped onto the block amax).  For
+// amax >= 2^-125 one product with RN(1/6) is corrected by its remainder, which
+// a fused multiply-add gives exactly (Markstein's correction step for division
+// by a constant whose reciprocal is rounded to nearest); checked against IEEE
+// division for every fp32 value in that range.  Below it the quotient is
+// subnormal and the remainder inexact, so those (rare) inputs divide directly.
+__device__ __forceinline__ float div6_rn(float a) {
+  if (a < 0x1p-125f) return __fdiv_rn(a, 6.0f);
+  constexpr float kSixth = 1.0f / 6.0f;  // RN(1/6)
+  const float q0 = __fmul_rn(a, kSixth);
+  return __fmaf_rn(__fmaf_rn(-q0, 6.0f, a), kSixth, q0);
+}
+
 // Block scale: returns the scale code, the multiplier that maps values onto the
 // E2M1 grid (0 means "all codes +0") and the decoded scale (times g_dec for
 // the dequantized value: deq = (e2m1 * sv) * g_dec for NVFP4, e2m1 * sv for MX).
-// NVFP4: s = amax * c6 with c6 = g_enc / 6, S = E4M3(s), mul = g_enc / S (exact table).
+// NVFP4: s = (amax / 6) * g_enc, each step rounded once, S = E4M3(s),
+// mul = g_enc / S (exact table).
 template <int FMT>
-__device__ __forceinline__ uint32_t block_scale(float amax, float c6, const float* inv_tab, float& mul, float& sv) {
+__device__ __forceinline__ uint32_t block_scale(float amax, float g_enc, const float* inv_tab, float& mul, float& sv) {
   if constexpr (FMT == FMT_MX) {
     const int e = mx_exponent(amax);
     mul = pow2f(-e);
     sv = pow2f(e);
     return (uint32_t)(e + 127);
   } else {
-    const uint32_t sc = cvt_e4m3(__fmul_rn(amax, c6));
+    const uint32_t sc = cvt_e4m3(__fmul_rn(div6_rn(amax), g_enc));
     sv = e4m3_value(sc);
     mul = inv_tab[sc];  // 0 for code 0
     return sc;
@@ -597,7 +612,7 @@ __device__ __forceinline__ void sub_deq8(float* h, uint32_t c, float sv, float g
 // words) and scales.  The backbone is quantized in its expanded form (codes
 // of dropped positions masked to +0), so R = h - deq needs no selects.
 template <int FMT, int PAT>
-__device__ __forceinline__ void quantize_unit(float (&h)[32], float c6, float g_dec, const float* inv_tab,
+__device__ __forceinline__ void quantize_unit(float (&h)[32], float g_enc, float g_dec, const float* inv_tab,
                                               uint32_t& meta, uint32_t (&bc)[4], uint32_t& bsc, uint32_t (&rc)[4],
                                               uint32_t& rsc0, uint32_t& rsc1) {
   uint32_t keepw[4];  // nibble mask of kept elements, per 8 elements
@@ -640,7 +655,7 @@ __device__ __forceinline__ void quantize_unit(float (&h)[32], float c6, float g_
   // the group maximum is always kept, so the backbone block amax is the window amax
   if constexpr (FMT == FMT_MX) bamax = fmaxf(bamax, __shfl_xor_sync(0xffffffffu, bamax, 1));
   float bmul, bsv;
-  bsc = block_scale<FMT>(bamax, c6, inv_tab, bmul, bsv);
+  bsc = block_scale<FMT>(bamax, g_enc, inv_tab, bmul, bsv);
 
   // backbone codes in expanded form; dropped positions -> +0
   uint32_t cw[4];
@@ -695,8 +710,8 @@ __device__ __forceinline__ void quantize_unit(float (&h)[32], float c6, float g_
 #pragma unroll
     for (int i = 16; i < 32; i++) a1 = fmaxf(a1, fabsf(h[i]));
     float m0, m1, sv0, sv1;
-    rsc0 = block_scale<FMT>(a0, c6, inv_tab, m0, sv0);
-    rsc1 = block_scale<FMT>(a1, c6, inv_tab, m1, sv1);
+    rsc0 = block_scale<FMT>(a0, g_enc, inv_tab, m0, sv0);
+    rsc1 = block_scale<FMT>(a1, g_enc, inv_tab, m1, sv1);
 #pragma unroll
     for (int w = 0; w < 4; w++) {
       const float mm = w < 2 ? m0 : m1;
@@ -714,7 +729,7 @@ __device__ __forceinline__ void quantize_unit(float (&h)[32], float c6, float g_
 #pragma unroll
     for (int i = 0; i < 32; i++) a0 = fmaxf(a0, fabsf(h[i]));
     float m0, sv0;
-    rsc0 = block_scale<FMT>(a0, c6, inv_tab, m0, sv0);
+    rsc0 = block_scale<FMT>(a0, g_enc, inv_tab, m0, sv0);
     rsc1 = 0;
 #pragma unroll
     for (int w = 0; w < 4; w++) {
@@ -742,11 +757,10 @@ __global__ void __launch_bounds__(128, ACT ? 6 : 7) prep_kernel(PrepParams p) {
   grid_dep_wait();    // the amax pass (or whatever wrote x) has completed
   grid_dep_launch();  // the GEMM may be scheduled; it waits for this grid in turn
 
-  float g_enc = 1.0f, g_dec = 1.0f, c6 = 1.0f;
+  float g_enc = 1.0f, g_dec = 1.0f;
   if constexpr (FMT == FMT_NV) {
     const float amax = p.act_amax > 0.0f ? p.act_amax : *reinterpret_cast<volatile const float*>(p.tensor);
     tensor_scales(amax, g_enc, g_dec);
-    c6 = __fdiv_rn(g_enc, 6.0f);
     fill_inv_table(inv_tab, g_enc);
     __syncthreads();
     if (blockIdx.x == 0 && threadIdx.x == 0) {
@@ -795,7 +809,7 @@ __global__ void __launch_bounds__(128, ACT ? 6 : 7) prep_kernel(PrepParams p) {
         for (int i = 0; i < 32; i++) h[i] = 0.0f;
       }
       uint32_t meta, bc[4], bsc, rc[4], rsc0, rsc1;
-      quantize_unit<FMT, PAT>(h, c6, g_dec, inv_tab, meta, bc, bsc, rc, rsc0, rsc1);
+      quantize_unit<FMT, PAT>(h, g_enc, g_dec, inv_tab, meta, bc, bsc, rc, rsc0, rsc1);
       if (!active || !in_pad) continue;
 
       if constexpr (PAT == PAT_48P) {
@@ -918,7 +932,7 @@ __global__ void __launch_bounds__(256) weight_kernel(WeightParams p) {
     sc = (uint32_t)(e + 127);
     mul = pow2f(-e);
   } else {
-    sc = cvt_e4m3(__fmul_rn(amax, __fdiv_rn(g_enc, 6.0f)));
+    sc = cvt_e4m3(__fmul_rn(__fdiv_rn(amax, 6.0f), g_enc));
     const float sv = e4m3_value(sc);
     mul = sv == 0.0f ? 0.0f : __fdiv_rn(g_enc, sv);
   }
