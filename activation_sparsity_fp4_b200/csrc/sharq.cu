@@ -302,6 +302,22 @@ sharq_status launch_gemm(const GemmMaps& maps, const GemmParams& gp, cudaStream_
   return launch_ex(gemm_kernel<KIND, SPARSE, SPLIT>, grid, dim3(448), C::kSmemBytes, s, 1, maps, gp);
 }
 
+// Workspace of sharq_linear_ws.  Every counter sits in a fixed region at the
+// start, so that no call's partial sums can land on another call's counters
+// whatever the shapes of the calls that share the workspace:
+//   [0, npairs * kSkFlagBytes)        stream-K counters (CTA-pair GEMM): one per
+//                                     (pair, CTA, epilogue warp);
+//   [.., + sms * 4)                   split-K counters (single-CTA GEMM): one per
+//                                     tile (split-K runs at most sms / 2 tiles);
+//   [ws_data_offset(), end)           partial sums: a stream-K slot of
+//                                     kSkSlotBytes per pair, or the split-K
+//                                     slices (one fp32 [t_pad][n] slot each).
+constexpr size_t kSkSlotBytes = 2 * 8 * 32 * 128 * sizeof(float);
+constexpr size_t kSkFlagBytes = 2 * 8 * sizeof(uint32_t);
+size_t ws_split_cnt_offset() { return (size_t)(sm_count() / 2) * kSkFlagBytes; }
+size_t ws_data_offset() { return (size_t)round_up((int64_t)(ws_split_cnt_offset() + sm_count() * sizeof(uint32_t)), 256); }
+size_t sk_workspace_bytes() { return ws_data_offset() + (size_t)(sm_count() / 2) * kSkSlotBytes; }
+
 // Split-K of the single-CTA GEMM for few tiles with long K loops: slices per
 // tile so that the work items fill the SMs, each slice at least 4 K tiles, at
 // most kMaxSplit slices.
@@ -318,8 +334,8 @@ int split_for(const GemmParams& gp, size_t ws_bytes) {
   int64_t split = sms / tiles;
   if (split > k_tiles / 4) split = k_tiles / 4;
   if (split > kMaxSplit) split = kMaxSplit;
-  const size_t slot = (size_t)gp.t_pad * gp.n * sizeof(float), cnt = (size_t)tiles * sizeof(uint32_t);
-  while (split >= 2 && (size_t)split * slot + cnt > ws_bytes) split--;  // one slot per slice must fit
+  const size_t slot = (size_t)gp.t_pad * gp.n * sizeof(float);
+  while (split >= 2 && ws_data_offset() + (size_t)split * slot > ws_bytes) split--;  // one slot per slice must fit
   return split >= 2 ? (int)split : 0;
 }
 
@@ -328,9 +344,8 @@ sharq_status launch_gemm_ws(const GemmMaps& maps, GemmParams gp, cudaStream_t s,
   const int split = ws ? split_for<KIND, SPARSE>(gp, ws_bytes) : 0;
   if (split < 2) return launch_gemm<KIND, SPARSE>(maps, gp, s);
   gp.split = split;
-  gp.split_acc = static_cast<float*>(ws);
-  gp.split_cnt =
-      reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + (size_t)split * gp.t_pad * gp.n * sizeof(float));
+  gp.split_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + ws_data_offset());
+  gp.split_cnt = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + ws_split_cnt_offset());
   return launch_gemm<KIND, SPARSE, true>(maps, gp, s);
 }
 
@@ -419,13 +434,6 @@ sharq_status launch_pair(const GemmMaps& maps, const GemmParams& gp, cudaStream_
   return launch_ex(gemm_pair_kernel<KIND, false>, dim3((unsigned)(2 * clusters)), dim3(448), C::kSmemBytes, s, 2,
                    maps, gp);
 }
-
-// Stream-K workspace of the CTA-pair GEMM: per pair a slot of partial sums
-// (2 CTAs x 8 epilogue warps x 32 rows x 128 fp32 columns), then one 32-bit
-// counter per (slot, CTA, epilogue warp).
-constexpr size_t kSkSlotBytes = 2 * 8 * 32 * 128 * sizeof(float);
-constexpr size_t kSkFlagBytes = 2 * 8 * sizeof(uint32_t);
-size_t sk_workspace_bytes() { return (size_t)(sm_count() / 2) * (kSkSlotBytes + kSkFlagBytes); }
 
 // The 1-4 row form on the CUDA cores (gemv.cuh).
 template <int FMT, int PAT>
@@ -564,8 +572,8 @@ sharq_status run_linear(const sharq_prepared* a, const sharq_weight* w, const in
       // 256 x 4096 x 16384 it takes 44 instead of 54 us; with more tiles or
       // shorter K the extra segment boundaries and the partial sums cost more
       // than the balance gains (2048 x 4096 x 4096: 41 instead of 35 us)
-      gp.sk_part = static_cast<float*>(ws);
-      gp.sk_flag = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + (size_t)npairs * kSkSlotBytes);
+      gp.sk_part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + ws_data_offset());
+      gp.sk_flag = reinterpret_cast<uint32_t*>(ws);
     }
     return a->fmt == SHARQ_NVFP4 ? launch_pair<GK_NVF4>(maps, gp, s) : launch_pair<GK_MXF4>(maps, gp, s);
   }
@@ -592,22 +600,59 @@ namespace {
 constexpr int kNoAllocMaxDevices = 64;
 std::mutex g_noalloc_mu;
 float* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+unsigned long long g_noalloc_ctx[kNoAllocMaxDevices] = {};  // id of the context the address belongs to
+
+// Unique id of the calling thread's current CUDA context (cuCtxGetId, through
+// the runtime's driver entry points); 0 if it cannot be read.  A device reset
+// destroys the primary context, and the one created after it has a new id.
+unsigned long long current_ctx_id() {
+  typedef CUresult (*GetCurrentFn)(CUcontext*);
+  typedef CUresult (*GetIdFn)(CUcontext, unsigned long long*);
+  static GetCurrentFn get_current = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<GetCurrentFn>(p);
+  }();
+  static GetIdFn get_id = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<GetIdFn>(p);
+  }();
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 // Device address of the current device's copy of g_noalloc_rstd, looked up
-// once per device (with that device current) and cached.  The first lookup
-// may load the module on that device, which is why the first call on a device
-// has to come before any stream capture.
+// with that device current and cached together with the id of the context it
+// belongs to.  The lookup runs on the first call on a device and again after
+// the device's context was replaced (cudaDeviceReset, or a context rebuilt
+// after an error: the module is loaded afresh and the old address is gone).
+// A lookup may load the module on that device, which is why the first call
+// on a device (and the first one after a reset) has to come before any
+// stream capture.
 sharq_status noalloc_scratch(float** out) {
   int dev = -1;
   SHARQ_CUDA(cudaGetDevice(&dev));
   if (dev < 0 || dev >= kNoAllocMaxDevices)
     return fail(SHARQ_ERR_INVALID, "device %d is beyond the %d devices the static scratch tracks", dev,
                 kNoAllocMaxDevices);
+  // before the device's first runtime call there is no current context (id 0):
+  // the lookup below creates it, and its id is read afterwards
+  const unsigned long long ctx = current_ctx_id();
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  if (!g_noalloc_ptr[dev] || ctx == 0 || ctx != g_noalloc_ctx[dev]) {
     void* p = nullptr;
     SHARQ_CUDA(cudaGetSymbolAddress(&p, g_noalloc_rstd));
     g_noalloc_ptr[dev] = static_cast<float*>(p);
+    g_noalloc_ctx[dev] = current_ctx_id();
   }
   *out = g_noalloc_ptr[dev];
   return SHARQ_OK;

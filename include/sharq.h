@@ -192,7 +192,10 @@ sharq_status sharq_gather_prepared(const sharq_prepared* src, const int32_t* row
  *     use sharq_prepare with a workspace for larger t.
  *   - The first call on a device looks up the scratch's address with that device
  *     current (this may load the library's module there); make it before any
- *     stream capture.  Later calls do no set-up.
+ *     stream capture.  Later calls do no set-up, unless the device's context was
+ *     replaced in between (cudaDeviceReset, or a context rebuilt after an error):
+ *     the call then notices the new context and looks the address up again, so
+ *     the first call after a reset also has to come before any stream capture.
  *   - Nothing in the scratch needs to start at zero (every row read was written by
  *     the same call); the amax accumulator, out->tensor[0], is zeroed on the stream
  *     as in sharq_prepare.
@@ -235,8 +238,12 @@ sharq_status sharq_linear(const sharq_prepared* a, const sharq_weight* w, void* 
 sharq_status sharq_linear_ws(const sharq_prepared* a, const sharq_weight* w, void* y, sharq_dtype y_dt,
                              void* workspace, size_t workspace_bytes, sharq_stream stream);
 
-/* Bytes of sharq_linear_ws's workspace on the current device (one 256 KiB slot
- * of partial sums and 64 bytes of counters per pair of SMs). */
+/* Bytes of sharq_linear_ws's workspace on the current device.  Layout: a fixed
+ * counter region first (64 bytes of stream-K counters per pair of SMs, then one
+ * 32-bit split-K counter per SM), then the partial sums from a 256-byte boundary
+ * on (one 256 KiB stream-K slot per pair of SMs; split-K slices use the same
+ * bytes).  No call's partial sums overlap any counter, so one workspace may
+ * serve calls of every shape in turn. */
 sharq_status sharq_linear_workspace_size(size_t* bytes);
 
 /* Same, with a choice of paths for diagnosis: paths bit 0 = sparse backbone GEMM,

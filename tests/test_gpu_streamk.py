@@ -26,10 +26,16 @@ def _x(seed, t, k):
     return workloads.to_bf16_values(x)
 
 
+def _counters(ws: torch.Tensor) -> tuple[np.ndarray, np.ndarray]:
+    """The workspace's fixed counter region: stream-K counters (16 per SM pair)
+    at the start, then one split-K counter per SM."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    words = ws[: (sms // 2) * 64 + sms * 4].cpu().numpy().view(np.uint32)
+    return words[: (sms // 2) * 16], words[(sms // 2) * 16:]
+
+
 def _flags(ws: torch.Tensor) -> np.ndarray:
-    pairs = torch.cuda.get_device_properties(0).multi_processor_count // 2
-    slot = 2 * 8 * 32 * 128 * 4
-    return ws[pairs * slot:].cpu().numpy().view(np.uint32)
+    return _counters(ws)[0]
 
 
 # (t, n, k): few tiles with long K loops, where the split applies: 16 tiles of
@@ -128,3 +134,38 @@ def test_split_k_single_cta_matches_oracle(cuda_ok, fmt, pat, t, n, k):
     assert_close_gemm(y1.cpu().numpy(), y0.double().cpu().numpy(), "split-K vs unsplit")
     assert torch.equal(y1, y2), "split-K is not reproducible"
     assert torch.equal(yb, y1.to(torch.bfloat16)), "bf16 output != fp32 output rounded to bf16"
+
+
+def test_one_workspace_serves_every_shape_in_turn(cuda_ok):
+    """One workspace kept per device for prefill and decode sizes: split-K at 256
+    rows, then 16 rows, then 256 rows again (MXFP4 2:4, k = 14336), then a
+    stream-K shape and split-K once more.  The partial sums of one call never
+    land on the counters of another (they sit in a fixed region before every
+    data slot), so every output matches the unsplit kernel, a repeated shape
+    gives the same bits, and every counter is back at zero."""
+    n, k = 4096, 14336
+    w = _w(50, n, k)
+    wq = sharq.FP4Weight.quantize(to_dev(w, "bf16"), "mxfp4")
+    preps = {t: gpu_prepare(_x(51 + t, t, k), "bf16", "mxfp4", "2:4") for t in (256, 16)}
+    xs, ws_ = _x(53, 256, 16384), _w(54, 4096, 16384)
+    psk = gpu_prepare(xs, "bf16", "nvfp4", "4:8pair")
+    wsk = sharq.FP4Weight.quantize(to_dev(ws_, "bf16"), "nvfp4")
+    ws = sharq.linear_workspace()
+    outs = []
+    for t in (256, 16, 256):
+        outs.append((t, sharq.linear(preps[t], wq, out_dtype=torch.float32, workspace=ws).clone()))
+    y_sk = sharq.linear(psk, wsk, out_dtype=torch.float32, workspace=ws).clone()
+    outs.append((16, sharq.linear(preps[16], wq, out_dtype=torch.float32, workspace=ws).clone()))
+    sharq.sharq_sync_status()
+    for t, y in outs:
+        y0 = sharq.linear(preps[t], wq, out_dtype=torch.float32)
+        sharq.sharq_sync_status()
+        assert_close_gemm(y.cpu().numpy(), y0.double().cpu().numpy(), f"reused workspace, t={t}")
+    assert torch.equal(outs[0][1], outs[2][1]), "t=256 after t=16 changed bits"
+    assert torch.equal(outs[1][1], outs[3][1]), "t=16 after the stream-K call changed bits"
+    y0 = sharq.linear(psk, wsk, out_dtype=torch.float32)
+    sharq.sharq_sync_status()
+    assert_close_gemm(y_sk.cpu().numpy(), y0.double().cpu().numpy(), "stream-K on a reused workspace")
+    flags, split_cnt = _counters(ws)
+    assert (flags % 2 == 0).all() and flags.max() > 0, "stream-K counters not back to even"
+    assert (split_cnt == 0).all(), "a split-K counter was left set"
