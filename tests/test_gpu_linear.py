@@ -228,6 +228,7 @@ def test_linear_wan_full_size_sampled_rows(cuda_ok, pat):
     p, _, y = _run_linear(cfg["x"], cfg["w"], "nvfp4", pat, gamma=cfg["gamma"], out_dtype=torch.float32)
     rows = np.sort(np.random.default_rng(12).choice(32768, 24, replace=False))
     amax = float(p.tensor[0].item())
+    assert np.float32(amax) == np.float32(oracle.rows_amax(cfg["x"], cfg["gamma"])), "device amax differs"
     prep = oracle.prepare(cfg["x"][rows], "nvfp4", pat, gamma=cfg["gamma"], act_amax=amax)
     wq = oracle.quantize_weight(cfg["w"], "nvfp4")
     assert_close_gemm(y[rows], oracle.linear_ref(prep, wq), f"wan {pat} sampled rows")
@@ -249,6 +250,9 @@ def test_linear_grouped_qwen_moe(cuda_ok, which):
     sharq.sharq_sync_status()
     y = y.cpu().numpy()
     amax = float(p.tensor[0].item())
+    # the device-computed tensor amax over all routed rows must be the oracle's
+    # before it is handed to the oracle for the sampled rows
+    assert np.float32(amax) == np.float32(oracle.rows_amax(x)), "MoE device amax differs from the oracle"
     rng = np.random.default_rng(13)
     experts = [0, 5, 64, 127] + list(rng.choice(128, 4, replace=False))
     for e in experts:
@@ -268,6 +272,7 @@ def test_linear_q_proj_full_size_sampled_rows(cuda_ok):
     p, wq_gpu, y = _run_linear(cfg["x"], cfg["w"], "nvfp4", "4:8pair", gamma=cfg["gamma"])
     rows = np.sort(np.random.default_rng(8).choice(2048, 64, replace=False))
     amax = float(p.tensor[0].item())
+    assert np.float32(amax) == np.float32(oracle.rows_amax(cfg["x"], cfg["gamma"])), "device amax differs"
     prep = oracle.prepare(cfg["x"][rows], "nvfp4", "4:8pair", gamma=cfg["gamma"], act_amax=amax)
     wq = oracle.quantize_weight(cfg["w"], "nvfp4")
     assert_close_gemm(y[rows], oracle.linear_ref(prep, wq), "q_proj sampled rows")
