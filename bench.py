@@ -8,18 +8,27 @@ W 4096 x 4096), synthetic seeded data.  The weight is quantized once, outside
 the timed region (it is an offline step of the layer).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sharq|reference]
-                  [--workload NAME] [--tokens T]
+                  [--workload NAME] [--tokens T] [--extra all|none]
 
-The default workload is q_proj; the others measure the remaining layer shapes
-the pages evaluate (one JSON line each, same keys); --tokens sets the row count
-of the q_proj / down_proj shapes (the down_proj token sweep 1/16/64/256).  The
-step runs as one CUDA graph (the kernels chained by programmatic dependent
-launch); prep and GEMM are also timed alone for the roofline fields.
+The headline line measures --workload (default q_proj) and, with --extra all
+(the default), carries a "workloads" object with the same measurements for
+every other layer shape the pages evaluate: Tiny, down_proj at 2048 rows and
+the 1/16/64/256-row sweep, Wan2.2 (4:8 pair and 8:16), and the Qwen3-30B-A3B
+MoE gate/up (tokens prepared once, prepared rows gathered) and down
+projections.  --tokens sets the row count of the q_proj / down_proj shapes.
+
+Timing.  Each workload holds R sets of inputs, weights and outputs whose
+total is at least three times the 126 MB L2 (R = 1 once one set is that
+large); consecutive steps use consecutive sets, so every step reads data that
+has left L2.  The K timed steps run back to back as ONE CUDA graph (kernels
+chained by programmatic dependent launch) between two CUDA events; prep and
+GEMM are then timed alone the same way (a graph of back-to-back launches over
+the sets), which gives each kernel's average launch duration for the roofline
+fields.
 
 Prints ONE JSON line (rank 0).  value = effective TFLOP/s = 2*T*N*K per step
-summed over ranks / max-over-ranks time; L2 is flushed (256 MB write) before
-every timed step, outside the step's CUDA events.  Multi-GPU runs are
-independent replicas (the layer has no exchange step): weak scaling.
+summed over ranks / max-over-ranks time.  Multi-GPU runs are independent
+replicas (the layer has no exchange step): weak scaling.
 """
 from __future__ import annotations
 
@@ -55,7 +64,17 @@ WORKLOADS = {
                         "padded to 128 rows), hidden 2048; per expert W 1536x2048; NVFP4, 4:8 pair, no norm; grouped",
     "qwen_moe_gate_up_gather": "Qwen3-30B-A3B MoE gate/up as qwen_moe_gate_up, but each of the 4096 tokens prepared "
                                "once and its prepared row gathered into the 32768 routed rows; grouped",
+    "qwen_moe_down": "Qwen3-30B-A3B MoE down: 32768 routed rows (expert order, each expert padded to 128 rows) x 768 "
+                     "bf16 0.5*t3; per expert W 2048x768; NVFP4, 4:8 pair, no norm; grouped",
 }
+
+# the shapes the headline line also reports (name, rows or None)
+EXTRA = [("tiny", None), ("down_proj", None), ("down_proj", 1), ("down_proj", 16), ("down_proj", 64),
+         ("down_proj", 256), ("wan", None), ("wan_816", None), ("qwen_moe_gate_up_gather", None),
+         ("qwen_moe_down", None)]
+
+L2_BYTES = 126 * 1024 * 1024
+ROTATE_BYTES = 3 * L2_BYTES  # the rotating sets of a workload cover at least this much
 
 
 def prep_bytes_per_elem(fmt: str, pat: str, x_bytes: int = 2) -> float:
@@ -68,15 +87,29 @@ def prep_bytes_per_elem(fmt: str, pat: str, x_bytes: int = 2) -> float:
     return x_bytes + bb_codes + meta + bb_sf + 0.5 + 1 / b
 
 
+_CONFIG_CACHE = {}
+
+
+def _config(fn, **kw) -> dict:
+    """Seeded inputs of a config generator, built once per process (the MoE config
+    serves two workloads)."""
+    key = (fn.__name__, tuple(sorted(kw.items())))
+    if key not in _CONFIG_CACHE:
+        _CONFIG_CACHE[key] = fn(**kw)
+    return _CONFIG_CACHE[key]
+
+
 def make_workload(name: str, tokens: int | None = None) -> dict:
     """Inputs and roofline terms of one bench workload (host arrays; nothing of the method here).
     tokens: row count of the q_proj / down_proj shapes (the down_proj token sweep)."""
     from activation_sparsity_fp4_b200 import workloads
-    if name in ("qwen_moe_gate_up", "qwen_moe_gate_up_gather"):
-        c = workloads.qwen_moe()
-        t, k = c["x"].shape
-        n = c["w_gu"].shape[1]
-        wl = dict(name=name, desc=WORKLOADS[name], x=c["x"], x_dtype="bf16", gamma=None, eps=1e-6, w=c["w_gu"], fmt="nvfp4",
+    if name.startswith("qwen_moe"):
+        c = _config(workloads.qwen_moe)
+        down = name == "qwen_moe_down"
+        x, w = (c["x_down"], c["w_d"]) if down else (c["x"], c["w_gu"])
+        t, k = x.shape
+        n = w.shape[1]
+        wl = dict(name=name, desc=WORKLOADS[name], x=x, x_dtype="bf16", gamma=None, eps=1e-6, w=w, fmt="nvfp4",
                   pat="4:8pair", offsets=c["offsets"], t=t, k=k, n=n, real_rows=int(c["counts"].sum()),
                   first_group=(int(c["offsets"][0]), int(c["offsets"][1])), gate=None, up=None)
         if name.endswith("_gather"):
@@ -84,9 +117,11 @@ def make_workload(name: str, tokens: int | None = None) -> dict:
         return wl
     kw = {"t": tokens} if tokens and name in ("q_proj", "down_proj", "down_proj_swiglu") else {}
     desc = WORKLOADS[name].replace("2048x", f"{tokens}x") if kw else WORKLOADS[name]
-    c = {"tiny": workloads.tiny, "q_proj": workloads.q_proj, "down_proj": workloads.down_proj,
-         "down_proj_swiglu": workloads.down_proj, "wan": workloads.wan,
-         "wan_816": lambda: workloads.wan(pat="8:16")}[name](**kw)
+    gen = {"tiny": workloads.tiny, "q_proj": workloads.q_proj, "down_proj": workloads.down_proj,
+           "down_proj_swiglu": workloads.down_proj, "wan": workloads.wan, "wan_816": workloads.wan}[name]
+    if name == "wan_816":
+        kw = {"pat": "8:16"}
+    c = _config(gen, **kw)
     t, k = c["x"].shape
     wl = dict(name=name, desc=desc, x=c["x"], x_dtype=c.get("x_dtype", "bf16"), gamma=c["gamma"], eps=c["eps"], w=c["w"],
               fmt=c["fmt"], pat=c["pat"], offsets=None, t=t, k=k, n=c["w"].shape[0], real_rows=t,
@@ -274,11 +309,255 @@ def cpu_baseline(name: str = "q_proj", rows: int = 2048, tokens: int | None = No
 
 
 # --------------------------------------------------------------------- GPU
-def run_sharq(args):
-    import numpy as np
+class LayerSets:
+    """Device state of one workload: R sets of inputs, quantized weight, prepared
+    activations and outputs, used in turn by consecutive steps so that together
+    they cover at least ROTATE_BYTES (a step never finds its data in L2)."""
+
+    def __init__(self, wl: dict, dev, max_sets: int = 16):
+        import torch
+
+        from activation_sparsity_fp4_b200 import sharq
+        self.wl = wl
+        T, K, N, fmt, pat = wl["t"], wl["k"], wl["n"], wl["fmt"], wl["pat"]
+        self.swiglu = wl["gate"] is not None
+        self.gathered = wl.get("gather") is not None
+        x_src = wl["gate"] if self.swiglu else (wl["tokens"] if self.gathered else wl["x"])
+        self.x_dt = torch.float32 if wl.get("x_dtype") == "f32" else torch.bfloat16
+        self.x_host = torch.from_numpy(x_src).to(self.x_dt).pin_memory()
+        self.up_host = torch.from_numpy(wl["up"]).to(torch.bfloat16).pin_memory() if self.swiglu else None
+        self.gamma = torch.from_numpy(wl["gamma"]).to(torch.bfloat16).to(dev) if wl["gamma"] is not None else None
+        self.offsets = torch.from_numpy(wl["offsets"]).to(torch.int32).to(dev) if wl["offsets"] is not None else None
+        self.rows_host = torch.from_numpy(wl["gather"]).to(torch.int32).pin_memory() if self.gathered else None
+        self.rows = self.rows_host.to(dev) if self.gathered else None
+        w = torch.from_numpy(wl["w"]).to(self.x_dt).to(dev)
+        experts = int(wl["w"].shape[0]) if wl["offsets"] is not None else 1
+        b = 16 if fmt == "nvfp4" else 32
+        tp = (T + 127) // 128 * 128
+        self.set_bytes = (self.x_host.numel() * self.x_host.element_size() * (2 if self.swiglu else 1)
+                          + experts * (N * K // 2 + 2 * N * K // b) + tp * K + T * N * 2)
+        self.R = max(1, min(max_sets, -(-ROTATE_BYTES // self.set_bytes)))
+        self.x, self.up, self.prep, self.prep_tok, self.y, self.wq, self.ws = [], [], [], [], [], [], []
+        for i in range(self.R):
+            self.x.append(self.x_host.to(dev))
+            self.up.append(self.up_host.to(dev) if self.swiglu else None)
+            self.prep.append(sharq.Prepared(T, K, fmt, pat, dev))
+            self.prep_tok.append(sharq.Prepared(self.x_host.shape[0], K, fmt, pat, dev) if self.gathered else None)
+            self.y.append(torch.zeros((T, N), dtype=torch.bfloat16, device=dev))
+            self.wq.append(sharq.FP4Weight.quantize(w, fmt))  # the same codes in every set
+            self.ws.append(sharq.linear_workspace(dev))  # lets few-tile shapes split their K loops
+        del w
+
+    def do_prep(self, i: int, act_amax: float = 0.0, stream=None):
+        from activation_sparsity_fp4_b200 import sharq
+        wl = self.wl
+        if self.swiglu:
+            sharq.prepare_swiglu(self.x[i], self.up[i], wl["fmt"], wl["pat"], act_amax=act_amax, out=self.prep[i],
+                                 stream=stream)
+        elif self.gathered:
+            sharq.prepare(self.x[i], wl["fmt"], wl["pat"], self.gamma, wl["eps"], act_amax=act_amax,
+                          out=self.prep_tok[i], stream=stream)
+            sharq.gather_prepared(self.prep_tok[i], self.rows, out=self.prep[i], stream=stream)
+        else:
+            sharq.prepare(self.x[i], wl["fmt"], wl["pat"], self.gamma, wl["eps"], act_amax=act_amax,
+                          out=self.prep[i], stream=stream)
+
+    def do_gemm(self, i: int, stream=None):
+        from activation_sparsity_fp4_b200 import sharq
+        if self.offsets is None:
+            sharq.linear(self.prep[i], self.wq[i], out=self.y[i], workspace=self.ws[i], stream=stream)
+        else:
+            sharq.linear_grouped(self.prep[i], self.wq[i], self.offsets, out=self.y[i], stream=stream)
+
+    def step(self, i: int):
+        self.do_prep(i)
+        self.do_gemm(i)
+
+
+def graph_of(fn, count: int, R: int):
+    """One CUDA graph of `count` back-to-back calls fn(i % R)."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(count):
+            fn(i % R)
+    return g
+
+
+def timed_replay_ms(g, stream) -> float:
+    import torch
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(stream)
+    g.replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b)
+
+
+def measure(name: str, tokens, steps: int, warmup: int, e2e_steps: int, dev, pg, world: int) -> dict:
+    """Timings of one workload (max over ranks) and its JSON fields."""
     import torch
 
     from activation_sparsity_fp4_b200 import sharq
+
+    wl = make_workload(name, tokens)
+    T, K, N, fmt, pat = wl["t"], wl["k"], wl["n"], wl["fmt"], wl["pat"]
+    L = LayerSets(wl, dev)
+    R = L.R
+    stream = torch.cuda.current_stream()
+    sharq.sharq_sync_status()
+    for i in range(warmup):
+        L.step(i % R)
+    sharq.sharq_sync_status()
+
+    # the K steps as ONE graph, back to back over the rotating sets; launches counted at capture
+    sharq.sharq_launch_count(reset=True)
+    g_steps = graph_of(L.step, steps, R)
+    launches = sharq.sharq_launch_count()
+    g_warm = graph_of(L.step, warmup, R)
+    m = R * max(1, -(-16 // R))  # kernel-alone graphs: >= 16 launches, whole rounds of the sets
+    g_prep = graph_of(L.do_prep, m, R)
+    g_gemm = graph_of(L.do_gemm, m, R)
+    g_warm.replay()
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        total_ms = timed_replay_ms(g_steps, stream)
+        if pg:
+            pg.barrier()
+        prep_ms = timed_replay_ms(g_prep, stream) / m
+        gemm_ms = timed_replay_ms(g_gemm, stream) / m
+    sharq.sharq_sync_status()
+    # caller-given amax variant of prep (no extra read of x), for the prep roofline
+    amax = float(L.prep[0].tensor[0].item())
+    g_given = graph_of(lambda i: L.do_prep(i, amax if fmt == "nvfp4" else 0.0), m, R)
+    given_ms = timed_replay_ms(g_given, stream) / m
+    sharq.sharq_sync_status()
+    del g_steps, g_warm, g_prep, g_gemm, g_given
+
+    # end to end through the public API from pinned host buffers: every step copies
+    # its input in, runs prep + GEMM and copies y out; the steps run as a pipeline on
+    # three streams (input copies, compute, output copies) with two sets of device
+    # buffers (sets 0 and 1 when there are two), so step i+1's input copy and step
+    # i-1's output copy overlap step i's compute.  Timed from the first input copy to
+    # the last output copy (device events).
+    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    nb = min(R, 2)
+    y_host = [torch.empty((T, N), dtype=torch.bfloat16).pin_memory() for _ in range(nb)]
+    ev_in = [torch.cuda.Event() for _ in range(nb)]
+    ev_cmp = [torch.cuda.Event() for _ in range(nb)]
+    ev_out = [torch.cuda.Event() for _ in range(nb)]
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    for i in range(warmup + e2e_steps):
+        b = i % nb
+        if i == warmup:
+            torch.cuda.synchronize()
+            e_start.record(s_in)
+        with torch.cuda.stream(s_in):
+            if i >= nb:
+                s_in.wait_event(ev_cmp[b])  # the compute that read these inputs is done
+            L.x[b].copy_(L.x_host, non_blocking=True)
+            if L.swiglu:
+                L.up[b].copy_(L.up_host, non_blocking=True)
+            if L.gathered:
+                L.rows.copy_(L.rows_host, non_blocking=True)
+            ev_in[b].record(s_in)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(ev_in[b])
+            if i >= nb:
+                s_cmp.wait_event(ev_out[b])  # y of this buffer has been copied out
+            L.do_prep(b, stream=s_cmp)
+            L.do_gemm(b, stream=s_cmp)
+            ev_cmp[b].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_cmp[b])
+            y_host[b].copy_(L.y[b], non_blocking=True)
+            ev_out[b].record(s_out)
+    s_out.wait_stream(s_in)
+    s_out.wait_stream(s_cmp)
+    e_end.record(s_out)
+    torch.cuda.synchronize()
+    e2e_ms = e_start.elapsed_time(e_end)
+    sharq.sharq_sync_status()
+
+    total_ms, e2e_ms, prep_ms, given_ms, gemm_ms = max_over_ranks([total_ms, e2e_ms, prep_ms, given_ms, gemm_ms],
+                                                                   pg, dev)
+    pk, src = peaks()
+    flops = 2.0 * wl["real_rows"] * N * K
+    value = replica_throughput(world, flops, steps, total_ms)
+    gemm_s = gemm_ms / 1e3
+    work, kind, work_desc = gemm_roofline(wl)
+    b_blk = 16 if fmt == "nvfp4" else 32
+    wbytes = (N * K / 2 + N * K / (2 * b_blk) * (2 if pat == "8:16" else 1)
+              + prep_bytes_per_elem(fmt, pat, 0) * T * K + 2 * T * N)
+    ratio = FP4_OVER_BF16 if kind == "fp4" else FP8_OVER_BF16
+    peak = pk["bf16_tflops"] * ratio
+    achieved = work / gemm_s / 1e12
+    bpe = prep_bytes_per_elem(fmt, pat, 4 if (L.swiglu or L.x_dt == torch.float32) else 2)
+    prep_bytes = bpe * T * K
+    if L.gathered:  # prep of the tokens, then each routed row's prepared bytes read and written once
+        prep_bytes = bpe * L.x_host.shape[0] * K + 2 * (bpe - 2) * T * K + 4 * T
+    prep_gbs = prep_bytes / (prep_ms / 1e3) / 1e9
+    given_gbs = prep_bytes / (given_ms / 1e3) / 1e9
+    grouped = wl["offsets"] is not None
+    kernel = {"4:8pair": "sparse", "2:4": "sparse", "8:16": "dense backbone"}[pat]
+    kname = ("gemv_kernel" if (not grouped and T <= 4) else
+             "gemm_pair_kernel" if (not grouped and pat == "4:8pair" and ((T + 127) // 128 * 128) % 256 == 0)
+             else "gemm_kernel")
+    kkind = "MXF8" if (fmt == "mxfp4" and pat == "2:4") else ("NVF4" if fmt == "nvfp4" else "MXF4")
+    klabel = (f"gemv_kernel<{'MX' if fmt == 'mxfp4' else 'NV'}, {pat}, {T} rows>" if kname == "gemv_kernel"
+              else f"{kname}<{kkind}, {kernel}>")
+    set_mb = L.set_bytes / 2 ** 20
+    res = {
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "ms_per_step": round(total_ms / steps, 5),
+        "steps": steps,
+        "config": {"workload": wl["desc"], "t": T, "k": K, "n": N, "fmt": fmt, "pattern": pat,
+                   "norm": "rmsnorm" if wl["gamma"] is not None else "none", "y_dtype": "bf16",
+                   "l2": (f"{R} rotating sets of inputs, weight and outputs ({set_mb:.0f} MiB each, "
+                          f"{R * set_mb:.0f} MiB in all, L2 126 MB), steps back to back; each set is touched "
+                          f"once every {R} steps")},
+        "roofline": ({"bound": "tensor", "kernel": klabel,
+                      "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
+                      "frac": round(achieved / peak, 4), "traffic": None,
+                      "peak_source": f"{src}: bf16 burst x {ratio:g} (nominal {kind.upper()}/BF16)",
+                      "work": work_desc, "avg_launch_us": round(gemm_s * 1e6, 2)}
+                     if T > 64 else
+                     # decode-size rows: the GEMM streams the weight; HBM bound
+                     {"bound": "hbm", "kernel": klabel,
+                      "achieved": round(wbytes / gemm_s / 1e9, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                      "frac": round(wbytes / gemm_s / 1e9 / pk["hbm_gbs"], 4), "traffic": None,
+                      "peak_source": src,
+                      "work": "weight codes N*K/2 + sparse-view scales N*K/(2b) + prepared X + y bytes",
+                      "avg_launch_us": round(gemm_s * 1e6, 2)}),
+        "prep": {"gbs_device_amax": round(prep_gbs, 1), "gbs_given_amax": round(given_gbs, 1),
+                 "peak_gbs": pk["hbm_gbs"], "frac_given_amax": round(given_gbs / pk["hbm_gbs"], 4),
+                 "frac_device_amax": round(prep_gbs / pk["hbm_gbs"], 4),
+                 "bytes_per_elem": bpe, "avg_us": round(prep_ms * 1e3, 2), "avg_us_given_amax": round(given_ms * 1e3, 2)},
+        "e2e": {"value": round(replica_throughput(world, flops, e2e_steps, e2e_ms), 3), "unit": "TFLOP/s",
+                "steps": e2e_steps,
+                "mode": "public API per step (pinned host x in, y out), steps pipelined on copy-in / compute / "
+                        "copy-out streams with double buffers",
+                "h2d_bytes_per_step": int(L.x_host.numel() * L.x_host.element_size() * (2 if L.swiglu else 1)
+                                          + (L.rows_host.numel() * 4 if L.gathered else 0)),
+                "d2h_bytes_per_step": int(T * N * 2)},
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+    }
+    if grouped:
+        res["config"]["routed_rows"] = wl["real_rows"]
+        res["config"]["experts"] = int(wl["w"].shape[0])
+    del L
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_sharq(args):
+    import torch
 
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
@@ -291,267 +570,46 @@ def run_sharq(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         pg = dist
 
-    wl = make_workload(args.workload, args.tokens)
-    T, K, N, fmt, pat = wl["t"], wl["k"], wl["n"], wl["fmt"], wl["pat"]
-    swiglu = wl["gate"] is not None
-    gathered = wl.get("gather") is not None  # prep of the tokens, then their prepared rows gathered
-    x_src = wl["gate"] if swiglu else (wl["tokens"] if gathered else wl["x"])
-    x_dt = torch.float32 if wl.get("x_dtype") == "f32" else torch.bfloat16  # the workload's input dtype
-    x_host = torch.from_numpy(x_src).to(x_dt).pin_memory()
-    x = x_host.to(dev)
-    up_host = torch.from_numpy(wl["up"]).to(torch.bfloat16).pin_memory() if swiglu else None
-    up = up_host.to(dev) if swiglu else None
-    gamma = torch.from_numpy(wl["gamma"]).to(torch.bfloat16).to(dev) if wl["gamma"] is not None else None
-    w = torch.from_numpy(wl["w"]).to(x_dt).to(dev)
-    wq = sharq.FP4Weight.quantize(w, fmt)
-    del w
-    offsets = torch.from_numpy(wl["offsets"]).to(torch.int32).to(dev) if wl["offsets"] is not None else None
-    prep = sharq.Prepared(T, K, fmt, pat, dev)
-    ws = sharq.linear_workspace(dev)  # lets few-tile shapes split their K loops over the SMs
-    if gathered:
-        rows_host = torch.from_numpy(wl["gather"]).to(torch.int32).pin_memory()
-        rows = rows_host.to(dev)
-        prep_tok = sharq.Prepared(x_host.shape[0], K, fmt, pat, dev)
-    y = torch.zeros((T, N), dtype=torch.bfloat16, device=dev)
-    y_host = torch.empty((T, N), dtype=torch.bfloat16).pin_memory()
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream()
-    sharq.sharq_sync_status()
-
-    def do_prep(act_amax=0.0):
-        if swiglu:
-            sharq.prepare_swiglu(x, up, fmt, pat, act_amax=act_amax, out=prep)
-        elif gathered:
-            sharq.prepare(x, fmt, pat, gamma, wl["eps"], act_amax=act_amax, out=prep_tok)
-            sharq.gather_prepared(prep_tok, rows, out=prep)
-        else:
-            sharq.prepare(x, fmt, pat, gamma, wl["eps"], act_amax=act_amax, out=prep)
-
-    def do_gemm():
-        if offsets is None:
-            sharq.linear(prep, wq, out=y, workspace=ws)
-        else:
-            sharq.linear_grouped(prep, wq, offsets, out=y)
-
-    def step():
-        do_prep()
-        do_gemm()
-
-    for _ in range(args.warmup):
-        flush.fill_(1)
-        step()
-    sharq.sharq_sync_status()
-
-    # the step as ONE CUDA graph (amax, prep, GEMM): no host launch overhead, and
-    # the kernels keep their programmatic-launch overlap (each is scheduled while
-    # the one before it finishes).  Nothing is recorded between prep and GEMM
-    # inside the timed steps, since an event node there would serialise them;
-    # prep and GEMM are timed on their own right after, as graphs of the same
-    # calls replayed on the same inputs with the same L2 flush.
-    g_step, g_prep, g_gemm = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    sharq.sharq_launch_count(reset=True)
-    with torch.cuda.graph(g_step):
-        step()
-    launches_per_step = sharq.sharq_launch_count()
-    with torch.cuda.graph(g_prep):
-        do_prep()
-    with torch.cuda.graph(g_gemm):
-        do_gemm()
-    for _ in range(args.warmup):
-        flush.fill_(1)
-        g_step.replay()
-    torch.cuda.synchronize()
-
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-    if pg:
-        pg.barrier()
-    torch.cuda.synchronize()
-    def replay_ms(g):
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-        for a, b in evs:
-            flush.fill_(1)
-            a.record(stream)
-            g.replay()
-            b.record(stream)
-        torch.cuda.synchronize()
-        return [a.elapsed_time(b) for a, b in evs]
-
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        for i in range(args.steps):
-            flush.fill_(1)
-            ev[i][0].record(stream)
-            g_step.replay()
-            ev[i][1].record(stream)
-        torch.cuda.synchronize()
-        if pg:
-            pg.barrier()
-        # the two kernels of the step alone, same inputs and flush (the GEMM's
-        # launch duration for the roofline; prep for its GB/s)
-        prep_ms = replay_ms(g_prep)
-        gemm_ms = replay_ms(g_gemm)
-    launches = launches_per_step * args.steps
-    sharq.sharq_sync_status()
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = sum(step_ms)
-
-    # caller-given amax variant of prep (no extra read of x), for the prep roofline:
-    # a graph of the same call with the amax the device found, replayed like the others
-    amax = float(prep.tensor[0].item())
-    g_given = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_given):
-        do_prep(amax if fmt == "nvfp4" else 0.0)
-    prep_given_ms = statistics.mean(replay_ms(g_given))
-    sharq.sharq_sync_status()
-
-    # end to end through the public API from pinned host buffers: every step
-    # copies its input in, runs prep + GEMM and copies y out; the steps run as a
-    # pipeline on three streams (input copies, compute, output copies) with two
-    # sets of device buffers, so step i+1's input copy and step i-1's output copy
-    # overlap step i's compute.  The compute stream also writes the 256 MB L2
-    # flush before every step.  Timed from the first input copy to the last
-    # output copy (device events).
-    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
-    n_buf = 2
-    xb = [torch.empty_like(x) for _ in range(n_buf)]
-    upb = [torch.empty_like(up) for _ in range(n_buf)] if swiglu else None
-    rowsb = [torch.empty_like(rows) for _ in range(n_buf)] if gathered else None
-    pb = [sharq.Prepared(T, K, fmt, pat, dev) for _ in range(n_buf)]
-    ptb = [sharq.Prepared(x_host.shape[0], K, fmt, pat, dev) for _ in range(n_buf)] if gathered else None
-    yb = [torch.empty_like(y) for _ in range(n_buf)]
-    yh = [torch.empty_like(y_host).pin_memory() for _ in range(n_buf)]
-    ws_e2e = sharq.linear_workspace(dev)  # its own: the e2e steps overlap on three streams
-
-    def e2e_compute(b):
-        if swiglu:
-            sharq.prepare_swiglu(xb[b], upb[b], fmt, pat, out=pb[b], stream=s_cmp)
-        elif gathered:
-            sharq.prepare(xb[b], fmt, pat, gamma, wl["eps"], out=ptb[b], stream=s_cmp)
-            sharq.gather_prepared(ptb[b], rowsb[b], out=pb[b], stream=s_cmp)
-        else:
-            sharq.prepare(xb[b], fmt, pat, gamma, wl["eps"], out=pb[b], stream=s_cmp)
-        if offsets is None:
-            sharq.linear(pb[b], wq, out=yb[b], stream=s_cmp, workspace=ws_e2e)
-        else:
-            sharq.linear_grouped(pb[b], wq, offsets, out=yb[b], stream=s_cmp)
-
-    ev_in = [torch.cuda.Event() for _ in range(n_buf)]
-    ev_cmp = [torch.cuda.Event() for _ in range(n_buf)]
-    ev_out = [torch.cuda.Event() for _ in range(n_buf)]
-    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    for i in range(args.warmup + args.steps):
-        b = i % n_buf
-        if i == args.warmup:
-            torch.cuda.synchronize()
-            e_start.record(s_in)
-        with torch.cuda.stream(s_in):
-            if i >= n_buf:
-                s_in.wait_event(ev_cmp[b])  # the compute that read these inputs is done
-            xb[b].copy_(x_host, non_blocking=True)
-            if swiglu:
-                upb[b].copy_(up_host, non_blocking=True)
-            if gathered:
-                rowsb[b].copy_(rows_host, non_blocking=True)
-            ev_in[b].record(s_in)
-        with torch.cuda.stream(s_cmp):
-            s_cmp.wait_event(ev_in[b])
-            if i >= n_buf:
-                s_cmp.wait_event(ev_out[b])  # y of this buffer has been copied out
-            flush.fill_(1)
-            e2e_compute(b)
-            ev_cmp[b].record(s_cmp)
-        with torch.cuda.stream(s_out):
-            s_out.wait_event(ev_cmp[b])
-            yh[b].copy_(yb[b], non_blocking=True)
-            ev_out[b].record(s_out)
-    s_out.wait_stream(s_in)
-    s_out.wait_stream(s_cmp)
-    e_end.record(s_out)
-    torch.cuda.synchronize()
-    e2e_ms = e_start.elapsed_time(e_end)
-    sharq.sharq_sync_status()
-
-    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], pg, dev)
+    head = measure(args.workload, args.tokens, args.steps, args.warmup, args.steps, dev, pg, world)
+    extras = {}
+    if args.extra == "all" and args.workload == "q_proj" and not args.tokens:
+        for name, tokens in EXTRA:
+            key = name if tokens is None else f"{name}_t{tokens}"
+            big = name.startswith(("wan", "qwen"))
+            extras[key] = measure(name, tokens, min(args.steps, 10 if big else 20), 3,
+                                  min(args.steps, 4 if big else 10), dev, pg, world)
 
     if rank == 0:
-        pk, src = peaks()
-        flops = 2.0 * wl["real_rows"] * N * K
-        value = replica_throughput(world, flops, args.steps, total_ms)
-        gemm_avg = statistics.mean(gemm_ms) / 1e3
-        work, kind, work_desc = gemm_roofline(wl)
-        b_blk = 16 if fmt == "nvfp4" else 32
-        wbytes = (N * K / 2 + N * K / (2 * b_blk) * (2 if pat == "8:16" else 1)
-                  + prep_bytes_per_elem(fmt, pat, 0) * T * K + 2 * T * N)
-        ratio = FP4_OVER_BF16 if kind == "fp4" else FP8_OVER_BF16
-        peak = pk["bf16_tflops"] * ratio
-        achieved = work / gemm_avg / 1e12
-        bpe = prep_bytes_per_elem(fmt, pat, 4 if (swiglu or x_dt == torch.float32) else 2)
-        prep_bytes = bpe * T * K
-        if gathered:  # prep of the tokens, then each routed row's prepared bytes read and written once
-            prep_bytes = bpe * x_host.shape[0] * K + 2 * (bpe - 2) * T * K + 4 * T
-        prep_gbs = prep_bytes / (statistics.mean(prep_ms) / 1e3) / 1e9
-        prep_given_gbs = prep_bytes / (prep_given_ms / 1e3) / 1e9
-        clocks = clk.summary()
-        grouped = offsets is not None
-        kernel = {"4:8pair": "sparse", "2:4": "sparse", "8:16": "dense backbone"}[pat]
-        kname = ("gemv_kernel" if (not grouped and T <= 4) else
-                 "gemm_pair_kernel" if (not grouped and pat == "4:8pair" and ((T + 127) // 128 * 128) % 256 == 0)
-                 else "gemm_kernel")
-        kkind = "MXF8" if (fmt == "mxfp4" and pat == "2:4") else ("NVF4" if fmt == "nvfp4" else "MXF4")
-        klabel = (f"gemv_kernel<{'MX' if fmt == 'mxfp4' else 'NV'}, {pat}, {T} rows>" if kname == "gemv_kernel"
-                  else f"{kname}<{kkind}, {kernel}>")
+        wl = make_workload(args.workload, args.tokens)
+        fmt = wl["fmt"]
+        traffic = committed_traffic() if args.workload == "q_proj" and not args.tokens else None
+        head["roofline"]["traffic"] = traffic
         out = {
             "metric": METRIC,
-            "value": round(value, 2),
+            "value": head["value"],
             "unit": "TFLOP/s",
             "n_gpus": world,
             "steps": args.steps,
             "warmup": args.warmup,
-            "ms_per_step": round(total_ms / args.steps, 5),
+            "ms_per_step": head["ms_per_step"],
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
             "dtype": (f"{fmt} (e2m1 x {'e4m3 block-16' if fmt == 'nvfp4' else 'e8m0 block-32'} scales, "
                       "fp32 accumulate)"),
             "data": f"synthetic (seeded, shaped like the pages' {args.workload} layer)",
-            "config": {"workload": wl["desc"], "t": T, "k": K, "n": N, "fmt": fmt, "pattern": pat,
-                       "norm": "rmsnorm" if gamma is not None else "none", "y_dtype": "bf16",
-                       "parallelism": f"replicas x{world}",
-                       "l2": "flushed (256 MB write) before every timed step"},
-            "roofline": ({"bound": "tensor", "kernel": klabel,
-                          "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
-                          "frac": round(achieved / peak, 4),
-                          "traffic": committed_traffic() if args.workload == "q_proj" and not args.tokens else None,
-                          "peak_source": f"{src}: bf16 burst x {ratio:g} (nominal {kind.upper()}/BF16)",
-                          "work": work_desc, "avg_launch_us": round(gemm_avg * 1e6, 2)}
-                         if T > 64 else
-                         # decode-size rows: the GEMM streams the weight; HBM bound
-                         {"bound": "hbm", "kernel": klabel,
-                          "achieved": round(wbytes / gemm_avg / 1e9, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-                          "frac": round(wbytes / gemm_avg / 1e9 / pk["hbm_gbs"], 4), "traffic": None,
-                          "peak_source": src,
-                          "work": "weight codes N*K/2 + sparse-view scales N*K/(2b) + prepared X + y bytes",
-                          "avg_launch_us": round(gemm_avg * 1e6, 2)}),
-            "prep": {"gbs_device_amax": round(prep_gbs, 1), "gbs_given_amax": round(prep_given_gbs, 1),
-                     "peak_gbs": pk["hbm_gbs"], "frac_given_amax": round(prep_given_gbs / pk["hbm_gbs"], 4),
-                     "frac_device_amax": round(prep_gbs / pk["hbm_gbs"], 4),
-                     "bytes_per_elem": bpe, "avg_us": round(statistics.mean(prep_ms) * 1e3, 2),
-                     "avg_us_given_amax": round(prep_given_ms * 1e3, 2)},
-            "e2e": {"value": round(replica_throughput(world, flops, args.steps, e2e_ms), 3), "unit": "TFLOP/s",
-                    "mode": "public API per step (pinned host x in, y out), steps pipelined on copy-in / compute / "
-                            "copy-out streams with double buffers",
-                    "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size() * (2 if swiglu else 1)
-                                              + (rows_host.numel() * 4 if gathered else 0)),
-                    "d2h_bytes_per_step": int(y_host.numel() * 2)},
-            "gpu_launches": int(launches),
-            "launch_mode": ("one CUDA graph per step (amax, prep, GEMM with programmatic dependent launch); "
-                            "prep and GEMM timed alone as graphs of the same calls right after the timed steps; "
-                            "e2e uses direct API calls"),
-            "clocks": clocks,
+            "config": dict(head["config"], parallelism=f"replicas x{world}"),
+            "roofline": head["roofline"],
+            "prep": head["prep"],
+            "e2e": head["e2e"],
+            "gpu_launches": head["gpu_launches"],
+            "launch_mode": ("the K steps as one CUDA graph (amax, prep, GEMM per step, chained by programmatic "
+                            "dependent launch) over rotating sets; prep and GEMM timed alone as graphs of "
+                            "back-to-back launches over the same sets; e2e uses direct API calls"),
+            "clocks": head["clocks"],
         }
-        if grouped:
-            out["config"]["routed_rows"] = wl["real_rows"]
-            out["config"]["experts"] = int(wl["w"].shape[0])
+        if extras:
+            out["workloads"] = extras
         if not args.no_cpu_baseline and world == 1:
             out["cpu_baseline"], _ = cpu_baseline(args.workload, tokens=args.tokens)
         print(json.dumps(out), flush=True)
@@ -601,6 +659,8 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="q_proj")
     ap.add_argument("--tokens", type=int, default=None,
                     help="row count of the q_proj / down_proj shapes (down_proj token sweep: 1, 16, 64, 256)")
+    ap.add_argument("--extra", choices=["all", "none"], default="all",
+                    help="with the default q_proj headline: also measure every other layer shape ('workloads')")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
