@@ -31,9 +31,10 @@ _BUILD_DIR = os.path.join(_HERE, "_build")
 _LIB_PATH = os.path.join(_BUILD_DIR, "liboracle.so")
 
 MXFP4, NVFP4 = 0, 1
-NM_2_4, NM_4_8_PAIR, NM_8_16 = 0, 1, 2
+NM_2_4, NM_4_8_PAIR, NM_8_16, NM_8_16_PAIR = 0, 1, 2, 3
 FORMATS = {"mxfp4": MXFP4, "nvfp4": NVFP4}
-PATTERNS = {"2:4": NM_2_4, "4:8pair": NM_4_8_PAIR, "8:16": NM_8_16}
+# "8:16pair": the 8:16 selection re-packed into the 4:8 pair layout
+PATTERNS = {"2:4": NM_2_4, "4:8pair": NM_4_8_PAIR, "8:16": NM_8_16, "8:16pair": NM_8_16_PAIR}
 
 _lock = threading.Lock()
 _lib = None

@@ -36,6 +36,7 @@
 #define ORC_NM_2_4 0
 #define ORC_NM_4_8_PAIR 1
 #define ORC_NM_8_16 2
+#define ORC_NM_8_16_PAIR 3 /* 8:16 selection re-packed into the 4:8 pair layout */
 
 /* ------------------------------------------------------------------ E2M1 --
  * 4-bit float: sign | 2-bit exponent | 1-bit mantissa.  Magnitudes of codes
@@ -198,10 +199,38 @@ void orc_swiglu(const float* gate, const float* up, int64_t n, float* h) {
  * Top-N by magnitude per group of M consecutive K elements; ties go to the
  * lower index.  For the 4:8 pair pattern the unit is an adjacent pair (2p,
  * 2p+1) scored by the larger magnitude of the two, and the top 2 of 4 pairs
- * are kept (ties to the lower pair).                                          */
+ * are kept (ties to the lower pair).
+ * 8:16 re-packed into the 4:8 pair layout (the 8:16 selection run on the
+ * sparse tensor cores, whose pattern is the 4:8 pair; what does not fit goes
+ * to the residual): the top 8 of each group of 16 are found as for 8:16; then
+ * in each aligned half of 8, pair p is ranked by (how many of those 8 it
+ * holds, its larger magnitude, lower index first) and the top 2 of 4 are kept. */
 static int pattern_m(int pat) { return pat == ORC_NM_2_4 ? 4 : (pat == ORC_NM_4_8_PAIR ? 8 : 16); }
 
+static void mask_row_nm(const float* h, int64_t k, int m, int n, uint8_t* keep);
+
 void orc_mask_row(const float* h, int64_t k, int pat, uint8_t* keep) {
+  if (pat == ORC_NM_8_16_PAIR) {
+    uint8_t* k16 = (uint8_t*)malloc((size_t)k);
+    mask_row_nm(h, k, 16, 8, k16);
+    for (int64_t g = 0; g < k; g += 8) {
+      int cnt[4];
+      float score[4];
+      for (int p = 0; p < 4; p++) {
+        cnt[p] = k16[g + 2 * p] + k16[g + 2 * p + 1];
+        score[p] = fmaxf(fabsf(h[g + 2 * p]), fabsf(h[g + 2 * p + 1]));
+      }
+      for (int p = 0; p < 4; p++) {
+        int beat = 0;
+        for (int q = 0; q < 4; q++)
+          if (cnt[q] > cnt[p] || (cnt[q] == cnt[p] && (score[q] > score[p] || (score[q] == score[p] && q < p))))
+            beat++;
+        keep[g + 2 * p] = keep[g + 2 * p + 1] = (uint8_t)(beat < 2);
+      }
+    }
+    free(k16);
+    return;
+  }
   if (pat == ORC_NM_4_8_PAIR) {
     for (int64_t g = 0; g < k; g += 8) {
       float score[4];
@@ -215,7 +244,11 @@ void orc_mask_row(const float* h, int64_t k, int pat, uint8_t* keep) {
     }
     return;
   }
-  int m = pattern_m(pat), n = m / 2;
+  int m = pattern_m(pat);
+  mask_row_nm(h, k, m, m / 2, keep);
+}
+
+static void mask_row_nm(const float* h, int64_t k, int m, int n, uint8_t* keep) {
   for (int64_t g = 0; g < k; g += m) {
     for (int i = 0; i < m; i++) {
       float ai = fabsf(h[g + i]);
@@ -235,7 +268,7 @@ void orc_mask_row(const float* h, int64_t k, int pat, uint8_t* keep) {
  *   8:16     -- per group of 16, a 16-bit little-endian mask, bit j = kept.
  * Nibble g of a row sits in byte g/2, low nibble first.                       */
 int64_t orc_meta_bytes_per_row(int64_t k, int pat) {
-  return pat == ORC_NM_4_8_PAIR ? k / 16 : k / 8;
+  return (pat == ORC_NM_4_8_PAIR || pat == ORC_NM_8_16_PAIR) ? k / 16 : k / 8;
 }
 
 void orc_meta_row(const uint8_t* keep, int64_t k, int pat, uint8_t* meta) {
@@ -250,7 +283,7 @@ void orc_meta_row(const uint8_t* keep, int64_t k, int pat, uint8_t* meta) {
     }
     return;
   }
-  int unit = (pat == ORC_NM_4_8_PAIR) ? 2 : 1;
+  int unit = (pat == ORC_NM_4_8_PAIR || pat == ORC_NM_8_16_PAIR) ? 2 : 1;
   int grp = 4 * unit;
   for (int64_t g = 0; g < k / grp; g++) {
     int idx[2], n = 0;
@@ -357,7 +390,7 @@ int orc_prepare(const float* x, int64_t t, int64_t k, const float* gamma, float 
                 uint8_t* res_scales, float* tensor, float* h_out, float* bdeq, float* rdeq) {
   if (k <= 0 || k % 256 != 0 || t < 0) return -1;
   if (fmt != ORC_MXFP4 && fmt != ORC_NVFP4) return -1;
-  if (pat < 0 || pat > 2) return -1;
+  if (pat < 0 || pat > 3) return -1;
   int b = fmt_block(fmt);
   float* h = (float*)malloc(sizeof(float) * (size_t)(t * k > 0 ? t * k : 1));
   for (int64_t r = 0; r < t; r++) {
@@ -494,7 +527,7 @@ void orc_decode_prepared(const uint8_t* meta, const uint8_t* bb_codes, const uin
         for (int j = 0; j < 16; j++) keep[16 * g + j] = (uint8_t)((mask >> j) & 1);
       }
     } else {
-      int unit = (pat == ORC_NM_4_8_PAIR) ? 2 : 1, grp = 4 * unit;
+      int unit = (pat == ORC_NM_4_8_PAIR || pat == ORC_NM_8_16_PAIR) ? 2 : 1, grp = 4 * unit;
       for (int64_t g = 0; g < k / grp; g++) {
         uint8_t nib = (uint8_t)((mr[g / 2] >> (4 * (g % 2))) & 15);
         int i0 = nib & 3, i1 = (nib >> 2) & 3;

@@ -71,7 +71,7 @@ def test_8_16_random_and_adversarial_ties():
         np.testing.assert_array_equal(k, _sort_keep(list(np.float32(g)), 8))
 
 
-@pytest.mark.parametrize("pat,m", [("2:4", 4), ("4:8pair", 8), ("8:16", 16)])
+@pytest.mark.parametrize("pat,m", [("2:4", 4), ("4:8pair", 8), ("8:16", 16), ("8:16pair", 16)])
 def test_exactly_half_kept_and_pruning_ratio(pat, m):
     # Huawei problem 137-2, "模块六": pruning ratio R = pruned / total; every
     # pattern keeps N = M/2, so R is exactly 50% (the problem's target).
@@ -154,3 +154,68 @@ def test_metadata_encodes_the_mask(pat):
     keep = oracle.mask(x, pat)
     for r in range(8):
         np.testing.assert_array_equal(_decode_meta_ref(prep["meta"][r], 512, pat), keep[r])
+
+
+# ------------------------------------------------ 8:16 re-packed (4:8 pair layout)
+def _sort_keep_repacked(group16):
+    """The re-packed rule by sorting: top 8 of the 16 (ties to the lower index),
+    then per half the 2 pairs ranked by (count of those 8 they hold, larger
+    magnitude, lower index first)."""
+    k16 = _sort_keep(group16, 8)
+    keep = np.zeros(16, np.uint8)
+    for half in range(2):
+        base = 8 * half
+        key = []
+        for p in range(4):
+            a, b = base + 2 * p, base + 2 * p + 1
+            key.append((-(int(k16[a]) + int(k16[b])), -max(abs(group16[a]), abs(group16[b])), p))
+        for _, _, p in sorted(key)[:2]:
+            keep[base + 2 * p] = keep[base + 2 * p + 1] = 1
+    return keep
+
+
+def test_8_16_pair_against_sorting_with_ties():
+    rng = np.random.default_rng(16)
+    groups = [rng.integers(-3, 4, 16).astype(np.float64) for _ in range(3000)]
+    groups += [np.full(16, 1.0), np.zeros(16), np.where(np.arange(16) % 2 == 0, 5.0, -5.0)]
+    groups += [rng.standard_normal(16) for _ in range(500)]
+    x, ng = _rows_of_groups(groups, 16)
+    keep = oracle.mask(x, "8:16pair").reshape(-1, 16)[:ng]
+    for g, k in zip(groups, keep):
+        np.testing.assert_array_equal(k, _sort_keep_repacked(list(np.float32(g))), err_msg=str(g))
+
+
+def test_8_16_pair_is_a_4_8_pair_mask():
+    rng = np.random.default_rng(17)
+    x = rng.standard_t(3, size=(32, 1024)).astype(np.float32)
+    x[:, ::5] = 0.0
+    keep = oracle.mask(x, "8:16pair").reshape(32, -1, 4, 2)
+    assert np.all(keep[..., 0] == keep[..., 1])           # whole pairs
+    assert np.all(keep[..., 0].sum(axis=-1) == 2)         # two of four per group of 8
+
+
+def test_8_16_pair_equals_8_16_where_the_selection_fits():
+    """When the top 8 of every 16 already sit in two whole pairs of each half,
+    the re-packed mask IS the 8:16 mask (nothing overflows into the residual)."""
+    rng = np.random.default_rng(18)
+    x = (rng.random((16, 512)).astype(np.float32) * 0.5).reshape(16, -1, 2, 4, 2)  # small everywhere
+    for r in range(16):
+        for g in range(x.shape[1]):
+            for h in range(2):
+                p0, p1 = rng.choice(4, 2, replace=False)
+                x[r, g, h, [p0, p1], :] = rng.uniform(1.0, 8.0, (2, 2)) * rng.choice([-1, 1], (2, 2))
+    x = x.reshape(16, 512)
+    np.testing.assert_array_equal(oracle.mask(x, "8:16pair"), oracle.mask(x, "8:16"))
+
+
+def test_8_16_pair_metadata_is_the_4_8_pair_encoding():
+    rng = np.random.default_rng(19)
+    x = rng.standard_normal((4, 256)).astype(np.float32)
+    prep = oracle.prepare(x, "mxfp4", "8:16pair")
+    keep = oracle.mask(x, "8:16pair")
+    assert prep["meta"].shape == (4, 256 // 16) and prep["bb_codes"].shape == (4, 256 // 4)
+    for r in range(4):
+        for g in range(256 // 8):
+            nib = (prep["meta"][r, g // 2] >> (4 * (g % 2))) & 15
+            kept = [p for p in range(4) if keep[r, 8 * g + 2 * p]]
+            assert nib == (kept[0] | (kept[1] << 2))

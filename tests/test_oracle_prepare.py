@@ -19,6 +19,10 @@ from activation_sparsity_fp4_b200 import workloads
 
 FMTS = ["mxfp4", "nvfp4"]
 PATS = ["2:4", "4:8pair", "8:16"]
+# with the re-packed 8:16 pattern; it can drop a group's maximum into the residual
+# (a half whose two best-covered pairs are not the one holding it), so the
+# backbone-scale invariant below is not asked of it
+PATS_ALL = PATS + ["8:16pair"]
 
 
 def _rows(seed, t=24, k=512, outliers=True):
@@ -92,7 +96,7 @@ def test_backbone_scale_is_window_amax_scale(fmt, pat):
 
 
 @pytest.mark.parametrize("fmt", FMTS)
-@pytest.mark.parametrize("pat", PATS)
+@pytest.mark.parametrize("pat", PATS_ALL)
 def test_residual_never_exceeds_input(fmt, pat):
     x = _rows(21)
     prep = oracle.prepare(x, fmt, pat, want_float=True)
@@ -106,7 +110,7 @@ def test_residual_never_exceeds_input(fmt, pat):
 
 
 @pytest.mark.parametrize("fmt", FMTS)
-@pytest.mark.parametrize("pat", PATS)
+@pytest.mark.parametrize("pat", PATS_ALL)
 def test_decomposition_error_bound(fmt, pat):
     """|h - deq(B) - deq(R)| = |R - deq(R)| <= max(s/4, |R|/4) per element, s = the
     residual block's decoded scale (times g_dec for NVFP4): the E2M1 rounding bound
@@ -139,12 +143,12 @@ def _representable_sparse_rows(fmt, pat, t=8, k=512, seed=23):
     quantization is exact and the residual must vanish."""
     rng = np.random.default_rng(seed)
     b = oracle.block_size(fmt)
-    m = {"2:4": 4, "4:8pair": 8, "8:16": 16}[pat]
+    m = {"2:4": 4, "4:8pair": 8, "8:16": 16, "8:16pair": 8}[pat]
     grid = np.array([0.5, 1.0, 1.5, 2.0, 3.0, 4.0])
     x = np.zeros((t, k), np.float32)
     for r in range(t):
         for g0 in range(0, k, m):
-            if pat == "4:8pair":
+            if pat in ("4:8pair", "8:16pair"):  # two whole pairs of every 8: what the re-pack keeps whole
                 pairs = np.sort(rng.choice(4, 2, replace=False))
                 pos = np.concatenate([[2 * p, 2 * p + 1] for p in pairs])
             else:
@@ -160,7 +164,7 @@ def _representable_sparse_rows(fmt, pat, t=8, k=512, seed=23):
     return x
 
 
-@pytest.mark.parametrize("pat", PATS)
+@pytest.mark.parametrize("pat", PATS_ALL)
 def test_zero_residual_on_representable_sparse_input_mxfp4(pat):
     x = _representable_sparse_rows("mxfp4", pat)
     prep = oracle.prepare(x, "mxfp4", pat, want_float=True)
@@ -169,7 +173,7 @@ def test_zero_residual_on_representable_sparse_input_mxfp4(pat):
     assert np.all(prep["rdeq"] == 0)
 
 
-@pytest.mark.parametrize("pat", PATS)
+@pytest.mark.parametrize("pat", PATS_ALL)
 def test_zero_residual_on_representable_sparse_input_nvfp4(pat):
     x = _representable_sparse_rows("nvfp4", pat, seed=24)
     prep = oracle.prepare(x, "nvfp4", pat, act_amax=2688.0 / 16.0, want_float=True)
