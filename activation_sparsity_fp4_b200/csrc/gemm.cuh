@@ -103,7 +103,8 @@ struct GemmCfg {
   static_assert(BN + kStages * kSlotCols <= kTmemCols, "tensor memory budget");
   static constexpr int kYCols = 16;                // bf16 output staged 32 rows x 16 columns at a time
   static constexpr int kYBuf = 8 * 32 * kYCols * 2;  // one chunk per epilogue warp
-  static constexpr int kSmemBytes = kStages * kStageBytes + kYBuf + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int kGatherIdx = BM * 4;  // gathered form: the tile's source row indices
+  static constexpr int kSmemBytes = kStages * kStageBytes + kYBuf + 1024 /*align*/ + 256 /*barriers*/ + kGatherIdx;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   // instruction descriptor (block-scaled kinds): E2M1 x E2M1, K-major, M=128, N=BN
   static constexpr uint32_t kFmt = kUnpacked ? 5u : 1u;
@@ -166,6 +167,15 @@ struct GemmParams {
   float* split_acc;
   uint32_t* split_cnt;
   int32_t split;
+  // gathered activation rows (single-CTA kernel, GATHER): row r of the routed
+  // operand is row gather_rows[r] of the token-prepared buffers below (an index
+  // < 0 or >= gather_src_t stands for an all-zero input row); sf_res / sf_bb
+  // then point at the tokens' scales (tiled, gather_src_tpad rows)
+  const int32_t* gather_rows;
+  int64_t gather_src_t, gather_src_tpad;
+  const uint8_t* g_res_codes;
+  const uint8_t* g_bb_codes;
+  const uint8_t* g_meta;
 };
 
 struct GemmMaps {
@@ -175,9 +185,18 @@ struct GemmMaps {
 
 // SPLIT: each tile's K loop is cut into p.split slices run by different CTAs
 // (few tiles, long K: the weight stream then uses every SM).
-template <int KIND, bool SPARSE, bool SPLIT>
+// GATHER (NVFP4 4:8 pair, grouped): the activation rows of a tile are read by
+// index from the token-prepared buffers (a mixture-of-experts layer prepares
+// each token once; its routed copies are never written out).  The producer
+// warp copies each row's residual, backbone and metadata bytes and its scale
+// words with cp.async into the stage, placing them where a tensor load with
+// the same swizzle would, and writes the all-zero row's encoding for padding
+// rows; a stage is handed to the MMA once its copies have landed and been made
+// visible to the tensor cores (fence.proxy.async), kGatherLag stages behind.
+template <int KIND, bool SPARSE, bool SPLIT, bool GATHER = false>
 __global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
   using C = GemmCfg<KIND, SPARSE>;
+  static_assert(!GATHER || (KIND == GK_NVF4 && SPARSE && !SPLIT), "gathered rows: NVFP4 4:8 pair, whole tiles");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ybuf = smem + C::kStages * C::kStageBytes;
@@ -192,13 +211,15 @@ __global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ Ge
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(ep_flag + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile uint32_t* split_last = reinterpret_cast<volatile uint32_t*>(tmem_holder + 2);  // split-K: last slice?
+  int32_t* gidx = reinterpret_cast<int32_t*>(smem_raw + C::kSmemBytes - C::kGatherIdx);  // gathered: source rows
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; s++) {
-      mbar_init(&full[s], 1);
+      // gathered form: the weight's tensor loads and, later, the landed row copies
+      mbar_init(&full[s], GATHER ? 2 : 1);
       mbar_init(&empty[s], 1);
       mbar_init(&sf_ready[s], 4);
     }
@@ -216,9 +237,11 @@ __global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ Ge
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch(&maps.w);
-    tma_prefetch(&maps.r);
-    tma_prefetch(&maps.b);
-    if (C::kEBoxes > 0) tma_prefetch(&maps.e);
+    if (!GATHER) {
+      tma_prefetch(&maps.r);
+      tma_prefetch(&maps.b);
+      if (C::kEBoxes > 0) tma_prefetch(&maps.e);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -265,7 +288,129 @@ __global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ Ge
     return lo;
   };
 
-  if (warp == 0) {
+  if (warp == 0 && GATHER) {
+    // ------------------------------------------- producer, gathered rows
+    // all 32 lanes copy the tile's rows; lane 0 also issues the weight loads
+    constexpr int kLag = C::kStages - 1;  // stages in flight before the oldest is handed over
+    const uint32_t smem0 = smem_u32(smem), full0 = smem_u32(full);
+    const int64_t sd_blocks = (sd_per_row + 3) / 4, sb_blocks = (sb_per_row + 3) / 4;
+    const int64_t ss_blocks = (p.k / C::kVecSparse + 3) / 4;
+    const int64_t rc_row = p.k / 2, bc_row = p.k / 4, me_row = p.k / 16;
+    const uint32_t gidx_s = smem_u32(gidx);
+    uint32_t g = 0;  // stages issued so far
+    uint32_t issued = 0, issued_par = 0;  // per stage: ever issued / parity of the last batch
+    auto hand_over = [&](uint32_t gg) {  // the copies of stage gg have landed in every lane
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&full[gg % C::kStages]);
+    };
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int item = blockIdx.x; item < items && !*abort_flag; item += gridDim.x) {
+      const int tile = item / n_split, k0 = k_lo(item), k1 = k_hi(item);
+      const TileXY xy = tile_xy(tile, m_tiles, n_tiles, C::kBandTiles);
+      const int mt = xy.mt, nt = xy.nt;
+      const int64_t m0 = (int64_t)mt * C::BM;
+      const int e = tile_expert(m0);
+      if (e < 0) continue;
+      const int32_t wrow = (int32_t)(e * p.n + (int64_t)nt * C::BN);
+      const int64_t nb = (int64_t)nt * C::kNRB;
+      const uint8_t* g_sfb_s = p.sf_w_sparse + e * wss_bytes + nb * ss_blocks * 512 + (int64_t)k0 * C::kChunksB * 512;
+      int32_t kx = k0 * C::kXStage;
+      // source rows of this tile (the copies in flight took their addresses at issue)
+      __syncwarp();
+      for (int i = lane; i < C::BM; i += 32) {
+        const int64_t r = m0 + i;
+        int32_t src = r < p.t ? __ldg(p.gather_rows + r) : -1;
+        if (src >= p.gather_src_t) src = -1;
+        gidx[i] = src;
+      }
+      __syncwarp();
+      for (int kt = k0; kt < k1; kt++) {
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait(&empty[stage], phase ^ 1, p.timeout_ns, abort_flag);
+        if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) { *abort_flag = 1; break; }
+        const uint32_t sb = smem0 + (uint32_t)(stage * C::kStageBytes);
+        if (lane == 0) {
+          const uint32_t fb = full0 + (uint32_t)(stage * 8);
+          mbar_arrive_expect_tx_u32(fb, (uint32_t)(C::kWBytes + C::kSfbS));
+          tma_load_2d_u32(sb + C::oW, &maps.w, kx, wrow, fb);
+#pragma unroll
+          for (int rb = 0; rb < C::kNRB; rb++)
+            bulk_load_u32(sb + C::oSfbS + rb * C::kChunksB * 512, g_sfb_s + rb * ss_blocks * 512, C::kChunksB * 512, fb);
+        }
+        // residual codes: 128 bytes of a row per stage, eight 16-byte pieces placed
+        // as the 128-byte swizzle does (piece c of row r at (c ^ (r % 8)) * 16)
+#pragma unroll 4
+        for (int j = 0; j < C::BM / 4; j++) {
+          const int r = 4 * j + (lane >> 3), c = lane & 7;
+          int32_t src;
+          asm volatile("ld.shared.s32 %0, [%1];" : "=r"(src) : "r"(gidx_s + 4 * r));
+          const uint32_t dst = sb + C::oR + (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
+          if (src >= 0) cp_async16(dst, p.g_res_codes + src * rc_row + (int64_t)kt * 128 + c * 16);
+          else st_shared_v4(dst, 0u, 0u, 0u, 0u);
+        }
+        // backbone codes: 64 bytes of a row, 64-byte swizzle (piece c at (c ^ ((r / 2) % 4)) * 16)
+#pragma unroll 4
+        for (int j = 0; j < C::BM / 8; j++) {
+          const int r = 8 * j + (lane >> 2), c = lane & 3;
+          int32_t src;
+          asm volatile("ld.shared.s32 %0, [%1];" : "=r"(src) : "r"(gidx_s + 4 * r));
+          const uint32_t dst = sb + C::oB + (uint32_t)(r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
+          if (src >= 0) cp_async16(dst, p.g_bb_codes + src * bc_row + (int64_t)kt * 64 + c * 16);
+          else st_shared_v4(dst, 0u, 0u, 0u, 0u);
+        }
+        // metadata (16 bytes a row) and the row's scale words (4 scales of each
+        // 512-byte chunk, at the row's place in the tiled layout)
+#pragma unroll
+        for (int j = 0; j < C::BM / 32; j++) {
+          const int r = 32 * j + lane;
+          int32_t src;
+          asm volatile("ld.shared.s32 %0, [%1];" : "=r"(src) : "r"(gidx_s + 4 * r));
+          const uint32_t dst_e = sb + C::oE + (uint32_t)(r * 16);
+          const uint32_t rpos = (uint32_t)((r & 31) * 16 + ((r >> 5) & 3) * 4);
+          if (src >= 0) {
+            cp_async16(dst_e, p.g_meta + src * me_row + (int64_t)kt * 16);
+            const uint8_t* sr = p.sf_res + ((int64_t)(src >> 7) * sd_blocks + (int64_t)kt * C::kChunksR) * 512 +
+                                (src & 31) * 16 + ((src >> 5) & 3) * 4;
+            const uint8_t* sbb = p.sf_bb + ((int64_t)(src >> 7) * sb_blocks + (int64_t)kt * C::kChunksB) * 512 +
+                                 (src & 31) * 16 + ((src >> 5) & 3) * 4;
+#pragma unroll
+            for (int c = 0; c < C::kChunksR; c++) cp_async4(sb + C::oSfaR + c * 512 + rpos, sr + c * 512);
+#pragma unroll
+            for (int c = 0; c < C::kChunksB; c++) cp_async4(sb + C::oSfaB + c * 512 + rpos, sbb + c * 512);
+          } else {
+            // an all-zero input row: each group of 8 keeps pairs 0 and 1 (nibble 4), codes and scales 0
+            st_shared_v4(dst_e, 0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
+#pragma unroll
+            for (int c = 0; c < C::kChunksR; c++) st_shared_u32(sb + C::oSfaR + c * 512 + rpos, 0u);
+#pragma unroll
+            for (int c = 0; c < C::kChunksB; c++) st_shared_u32(sb + C::oSfaB + c * 512 + rpos, 0u);
+          }
+        }
+        cp_async_commit();
+        if (g >= (uint32_t)kLag) {
+          cp_async_wait_group<kLag>();
+          hand_over(g - kLag);
+        }
+        g++;
+        kx += C::kXStage;
+        g_sfb_s += C::kChunksB * 512;
+        issued |= 1u << stage;
+        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+        if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+      }
+    }
+    // the last stages: every copy lands before they are handed over (also on abort,
+    // so that no copy is still in flight when the block exits)
+    cp_async_wait_group<0>();
+    for (uint32_t gg = g > (uint32_t)kLag ? g - kLag : 0; gg < g; gg++) hand_over(gg);
+    if (*abort_flag && lane == 0) {
+      // let the weight loads already issued land before the block can exit
+      for (int i = 0; i < C::kStages; i++)
+        if ((issued >> i) & 1u) (void)mbar_wait(&full[i], (issued_par >> i) & 1u, 1000000000ull, nullptr, true);
+    }
+  } else if (warp == 0) {
     // ------------------------------------------------------------- producer
     if (lane == 0) {
       int stage = 0;

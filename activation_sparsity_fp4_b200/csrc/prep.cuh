@@ -22,7 +22,10 @@
 namespace sharq {
 
 enum { FMT_MX = 0, FMT_NV = 1 };
-enum { PAT_24 = 0, PAT_48P = 1, PAT_816 = 2 };
+enum { PAT_24 = 0, PAT_48P = 1, PAT_816 = 2, PAT_816P = 3 };
+// Patterns stored in the 4:8 pair layout (metadata, compressed backbone, scales):
+// the 4:8 pair itself and the 8:16 selection re-packed into it.
+__host__ __device__ constexpr bool pair_layout(int pat) { return pat == PAT_48P || pat == PAT_816P; }
 
 // Byte offset of (row r, scale s) in the tiled scale layout with S scales per row.
 __host__ __device__ __forceinline__ int64_t tiled_sf_offset(int64_t r, int64_t s, int64_t S) {
@@ -265,19 +268,32 @@ __device__ __forceinline__ float div6_rn(float a) {
 // the dequantized value: deq = (e2m1 * sv) * g_dec for NVFP4, e2m1 * sv for MX).
 // NVFP4: s = (amax / 6) * g_enc, each step rounded once, S = E4M3(s),
 // mul = g_enc / S (exact table).
+// NVFP4 also returns the decoded scale as an f16 value in both halves of sh
+// (E4M3 values are exact in f16).
 template <int FMT>
-__device__ __forceinline__ uint32_t block_scale(float amax, float g_enc, const float* inv_tab, float& mul, float& sv) {
+__device__ __forceinline__ uint32_t block_scale(float amax, float g_enc, const float* inv_tab, float& mul, float& sv,
+                                                uint32_t& sh) {
   if constexpr (FMT == FMT_MX) {
     const int e = mx_exponent(amax);
     mul = pow2f(-e);
     sv = pow2f(e);
+    sh = 0;
     return (uint32_t)(e + 127);
   } else {
     const uint32_t sc = cvt_e4m3(__fmul_rn(div6_rn(amax), g_enc));
-    sv = e4m3_value(sc);
+    uint32_t h2;
+    const uint16_t in = (uint16_t)(sc | (sc << 8));
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+    sh = h2;
+    sv = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFF)));
     mul = inv_tab[sc];  // 0 for code 0
     return sc;
   }
+}
+template <int FMT>
+__device__ __forceinline__ uint32_t block_scale(float amax, float g_enc, const float* inv_tab, float& mul, float& sv) {
+  uint32_t sh;
+  return block_scale<FMT>(amax, g_enc, inv_tab, mul, sv, sh);
 }
 
 // Quantize 8 values: returns 8 codes (nibbles); mul = 0 gives +0 codes.
@@ -421,6 +437,13 @@ __device__ __forceinline__ void mul2(float& a, float& b, float c, float d) {  //
 __device__ __forceinline__ void sub2(float& a, float& b, float c, float d) {  // (a, b) -= (c, d)
   uint64_t r;
   asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pk2(a, b)), "l"(pk2(c, d)));
+  a = __uint_as_float((uint32_t)r);
+  b = __uint_as_float((uint32_t)(r >> 32));
+}
+
+__device__ __forceinline__ void fma2(float& a, float& b, float c, float d, float e, float f) {  // (a,b)*(c,d)+(e,f)
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(pk2(a, b)), "l"(pk2(c, d)), "l"(pk2(e, f)));
   a = __uint_as_float((uint32_t)r);
   b = __uint_as_float((uint32_t)(r >> 32));
 }
@@ -584,25 +607,43 @@ __device__ __forceinline__ uint32_t compact_pairs(uint32_t w, uint32_t p0, uint3
   return __byte_perm(w, 0u, p0 | (p1 << 4) | 0x4400u);  // bytes p0, p1 -> positions 0, 1; zeros above
 }
 
-// Residual of 8 values against their backbone codes: h -= (e2m1(c_i) * sv) * g
-// (g = 1 for MX).  e2m1 * sv is exact (2-bit times 4-bit significands), so
-// the packed multiply is safe; the NVFP4 product with g rounds, and the
-// compiler contracts a packed multiply followed by a packed subtract into one
-// fused multiply-add even with explicit rounding, which skips that rounding:
-// that step stays on scalar __fmul_rn / __fsub_rn, which are never contracted.
+// Residual of 8 values against their backbone codes, in place: h_i -= deq_i
+// with deq = (e2m1(c_i) * S) * g (NVFP4) or e2m1(c_i) * 2^e (MXFP4).
+//   NVFP4: e2m1 * S is exact (2-bit times 4-bit significands): one mixed
+//   f16 x f16 -> f32 fused multiply-add with a -0 addend forms it from the f16
+//   E2M1 pair and the f16 scale; times g is then one packed round-to-nearest
+//   multiply, and h - deq one packed fused multiply-add with -1 (deq * -1 is
+//   exact, so it rounds once, like the subtraction).  No multiply is followed
+//   by a plain subtract that could be contracted into one rounding.
+//   MXFP4: the product with 2^e is exact, so h - e2m1 * 2^e is one packed fused
+//   multiply-add.
 template <int FMT>
-__device__ __forceinline__ void sub_deq8(float* h, uint32_t c, float sv, float g) {
-  float d[8];
-  e2m1x8_values(c, d);
+__device__ __forceinline__ void sub_deq8(float* h, uint32_t c, uint32_t sh, float sv, float g) {
+  uint32_t e2[4];
+  asm("{\n\t.reg .b8 t0, t1, t2, t3;\n\tmov.b32 {t0, t1, t2, t3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, t0;\n\tcvt.rn.f16x2.e2m1x2 %1, t1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, t2;\n\tcvt.rn.f16x2.e2m1x2 %3, t3;\n\t}"
+      : "=r"(e2[0]), "=r"(e2[1]), "=r"(e2[2]), "=r"(e2[3])
+      : "r"(c));
 #pragma unroll
-  for (int i = 0; i < 8; i += 2) {
-    mul2(d[i], d[i + 1], sv, sv);
+  for (int b = 0; b < 4; b++) {
+    float d0, d1;
     if constexpr (FMT == FMT_NV) {
-      h[i] = __fsub_rn(h[i], __fmul_rn(d[i], g));
-      h[i + 1] = __fsub_rn(h[i + 1], __fmul_rn(d[i + 1], g));
+      asm("{\n\t.reg .f16 a0, a1, s0, s1;\n\tmov.b32 {a0, a1}, %2;\n\tmov.b32 {s0, s1}, %3;\n\t"
+          "fma.rn.f32.f16 %0, a0, s0, %4;\n\tfma.rn.f32.f16 %1, a1, s0, %4;\n\t}"
+          : "=f"(d0), "=f"(d1)
+          : "r"(e2[b]), "r"(sh), "f"(-0.0f));
+      mul2(d0, d1, g, g);
+      fma2(d0, d1, -1.0f, -1.0f, h[2 * b], h[2 * b + 1]);
     } else {
-      sub2(h[i], h[i + 1], d[i], d[i + 1]);
+      asm("{\n\t.reg .f16 a0, a1, one;\n\tmov.b32 {a0, a1}, %2;\n\tmov.b16 one, 0x3C00;\n\t"
+          "fma.rn.f32.f16 %0, a0, one, %3;\n\tfma.rn.f32.f16 %1, a1, one, %3;\n\t}"
+          : "=f"(d0), "=f"(d1)
+          : "r"(e2[b]), "f"(-0.0f));
+      fma2(d0, d1, -sv, -sv, h[2 * b], h[2 * b + 1]);
     }
+    h[2 * b] = d0;
+    h[2 * b + 1] = d1;
   }
 }
 
@@ -627,6 +668,40 @@ __device__ __forceinline__ void quantize_unit(float (&h)[32], float g_enc, float
       bamax = fmaxf(bamax, fmaxf(fmaxf(s0, s1), fmaxf(s2, s3)));
       uint32_t kk[4];
       top2of4_masks(s0, s1, s2, s3, kk);
+      meta |= kept_nibble(kk) << (4 * g);
+      keepw[g] = (kk[0] & 0x000000FFu) | (kk[1] & 0x0000FF00u) | (kk[2] & 0x00FF0000u) | (kk[3] & 0xFF000000u);
+    }
+  } else if constexpr (PAT == PAT_816P) {
+    // the top 8 of each group of 16, then in each group of 8 the two pairs that
+    // hold most of them, ranked by (count, larger magnitude, lower index): keys
+    // count << 32 | bits of the magnitude (non-negative floats order as their bits)
+    uint32_t m16;
+    const uint32_t keep16 = unit_mask<PAT_816>(h, m16);
+#pragma unroll
+    for (int g = 0; g < 4; g++) {
+      const float* hg = h + 8 * g;
+      float sp[4];
+      uint64_t key[4];
+#pragma unroll
+      for (int q = 0; q < 4; q++) {
+        sp[q] = fmaxf(fabsf(hg[2 * q]), fabsf(hg[2 * q + 1]));
+        const uint32_t cnt = __popc((keep16 >> (8 * g + 2 * q)) & 3u);
+        key[q] = ((uint64_t)cnt << 32) | __float_as_uint(sp[q]);
+      }
+      // pair p is kept iff it wins at least two of its three comparisons
+      // (against a lower pair on a strictly larger key, a higher pair on >=)
+      uint32_t kk[4];
+#pragma unroll
+      for (int q = 0; q < 4; q++) {
+        int wins = 0;
+#pragma unroll
+        for (int o = 0; o < 4; o++)
+          if (o != q) wins += (o < q) ? (key[q] > key[o]) : (key[q] >= key[o]);
+        kk[q] = wins >= 2 ? 0xFFFFFFFFu : 0u;
+      }
+      // the backbone block amax is over the kept values (the group maximum may be dropped)
+#pragma unroll
+      for (int q = 0; q < 4; q++) bamax = fmaxf(bamax, __uint_as_float(__float_as_uint(sp[q]) & kk[q]));
       meta |= kept_nibble(kk) << (4 * g);
       keepw[g] = (kk[0] & 0x000000FFu) | (kk[1] & 0x0000FF00u) | (kk[2] & 0x00FF0000u) | (kk[3] & 0xFF000000u);
     }
@@ -655,7 +730,8 @@ __device__ __forceinline__ void quantize_unit(float (&h)[32], float g_enc, float
   // the group maximum is always kept, so the backbone block amax is the window amax
   if constexpr (FMT == FMT_MX) bamax = fmaxf(bamax, __shfl_xor_sync(0xffffffffu, bamax, 1));
   float bmul, bsv;
-  bsc = block_scale<FMT>(bamax, g_enc, inv_tab, bmul, bsv);
+  uint32_t bsh;
+  bsc = block_scale<FMT>(bamax, g_enc, inv_tab, bmul, bsv, bsh);
 
   // backbone codes in expanded form; dropped positions -> +0
   uint32_t cw[4];
@@ -672,9 +748,9 @@ __device__ __forceinline__ void quantize_unit(float (&h)[32], float g_enc, float
   }
   // residual R = h - deq(backbone) (deq = +0 where dropped: R = h exactly)
 #pragma unroll
-  for (int g = 0; g < 4; g++) sub_deq8<FMT>(h + 8 * g, cw[g], bsv, g_dec);
+  for (int g = 0; g < 4; g++) sub_deq8<FMT>(h + 8 * g, cw[g], bsh, bsv, g_dec);
   // compaction of the kept codes (K order) for storage
-  if constexpr (PAT == PAT_48P) {
+  if constexpr (pair_layout(PAT)) {
     uint32_t half[4];
 #pragma unroll
     for (int g = 0; g < 4; g++) {
@@ -756,7 +832,6 @@ __global__ void __launch_bounds__(128, ACT ? 6 : 7) prep_kernel(PrepParams p) {
   const int row_in_block = threadIdx.x >> m.lg, tt = threadIdx.x & (m.tpr - 1);
   grid_dep_wait();    // the amax pass (or whatever wrote x) has completed
   grid_dep_launch();  // the GEMM may be scheduled; it waits for this grid in turn
-
   float g_enc = 1.0f, g_dec = 1.0f;
   if constexpr (FMT == FMT_NV) {
     const float amax = p.act_amax > 0.0f ? p.act_amax : *reinterpret_cast<volatile const float*>(p.tensor);
@@ -812,7 +887,7 @@ __global__ void __launch_bounds__(128, ACT ? 6 : 7) prep_kernel(PrepParams p) {
       quantize_unit<FMT, PAT>(h, g_enc, g_dec, inv_tab, meta, bc, bsc, rc, rsc0, rsc1);
       if (!active || !in_pad) continue;
 
-      if constexpr (PAT == PAT_48P) {
+      if constexpr (pair_layout(PAT)) {
         *reinterpret_cast<uint16_t*>(p.meta + r * (k / 16) + 2 * u) = (uint16_t)meta;
       } else {
         *reinterpret_cast<uint32_t*>(p.meta + r * (k / 8) + 4 * u) = meta;

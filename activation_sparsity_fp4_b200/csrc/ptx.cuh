@@ -137,6 +137,27 @@ __device__ __forceinline__ void bulk_load_u32(uint32_t smem_dst, const void* gme
                "l"(reinterpret_cast<uint64_t>(gmem_src)), "r"(bytes), "r"(bar)
                : "memory");
 }
+// 16- and 4-byte copies global -> shared (cp.async, generic proxy), grouped per
+// commit; the L1 serves the 16-byte pieces of one row from one line.
+__device__ __forceinline__ void cp_async16(uint32_t smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(smem_dst), "l"(reinterpret_cast<uint64_t>(gmem_src))
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_dst), "l"(reinterpret_cast<uint64_t>(gmem_src))
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t smem_dst, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(smem_dst), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+__device__ __forceinline__ void st_shared_u32(uint32_t smem_dst, uint32_t v) {
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(smem_dst), "r"(v) : "memory");
+}
 __device__ __forceinline__ void tma_prefetch(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

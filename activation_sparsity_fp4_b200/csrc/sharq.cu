@@ -53,7 +53,9 @@ int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 
 int fmt_block(sharq_format f) { return f == SHARQ_NVFP4 ? 16 : 32; }
 
-int64_t meta_row_bytes(int64_t k, sharq_pattern p) { return p == SHARQ_NM_4_8_PAIR ? k / 16 : k / 8; }
+int64_t meta_row_bytes(int64_t k, sharq_pattern p) {
+  return (p == SHARQ_NM_4_8_PAIR || p == SHARQ_NM_8_16_PAIR) ? k / 16 : k / 8;
+}
 
 uint64_t wait_timeout_ns() {
   static uint64_t v = [] {
@@ -222,8 +224,8 @@ RowLaunch row_launch(Kern kern, int64_t rows, int64_t k) {
 template <int FMT, int PAT, bool NORM, bool XBF16>
 sharq_status launch_prep(const PrepParams& pp, cudaStream_t s) {
   auto kern = prep_kernel<FMT, PAT, NORM, XBF16>;
-  const RowLaunch rl = row_launch(kern, pp.t_pad, pp.k);
   PrepParams q = pp;
+  const RowLaunch rl = row_launch(kern, pp.t_pad, pp.k);
   q.tpr = rl.tpr;
   return launch_ex(kern, dim3(rl.grid), dim3(128), 0, s, 1, q);
 }
@@ -254,6 +256,7 @@ sharq_status prep_dispatch_p(const PrepParams& pp, int pat, bool norm, bool xbf1
   switch (pat) {
     case PAT_24: return prep_dispatch_n<FMT, PAT_24>(pp, norm, xbf16, s);
     case PAT_48P: return prep_dispatch_n<FMT, PAT_48P>(pp, norm, xbf16, s);
+    case PAT_816P: return prep_dispatch_n<FMT, PAT_816P>(pp, norm, xbf16, s);
     default: return prep_dispatch_n<FMT, PAT_816>(pp, norm, xbf16, s);
   }
 }
@@ -276,6 +279,7 @@ sharq_status swiglu_dispatch_p(const PrepParams& pp, int pat, bool xbf16, cudaSt
   switch (pat) {
     case PAT_24: return swiglu_dispatch_x<FMT, PAT_24>(pp, xbf16, s);
     case PAT_48P: return swiglu_dispatch_x<FMT, PAT_48P>(pp, xbf16, s);
+    case PAT_816P: return swiglu_dispatch_x<FMT, PAT_816P>(pp, xbf16, s);
     default: return swiglu_dispatch_x<FMT, PAT_816>(pp, xbf16, s);
   }
 }
@@ -287,19 +291,19 @@ sharq_status launch_amax_swiglu(const void* gate, const void* up, int64_t t, int
   return launched();
 }
 
-template <int KIND, bool SPARSE, bool SPLIT = false>
+template <int KIND, bool SPARSE, bool SPLIT = false, bool GATHER = false>
 sharq_status launch_gemm(const GemmMaps& maps, const GemmParams& gp, cudaStream_t s) {
   using C = GemmCfg<KIND, SPARSE>;
   static bool configured = false;
   if (!configured) {
-    SHARQ_CUDA(cudaFuncSetAttribute(gemm_kernel<KIND, SPARSE, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    C::kSmemBytes));
+    SHARQ_CUDA(cudaFuncSetAttribute(gemm_kernel<KIND, SPARSE, SPLIT, GATHER>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes));
     configured = true;
   }
   const int items = (int)(gp.t_pad / C::BM) * (int)(gp.n / C::BN) * (SPLIT ? gp.split : 1);
   const int sms = sm_count();
   dim3 grid(items < sms ? items : sms);
-  return launch_ex(gemm_kernel<KIND, SPARSE, SPLIT>, grid, dim3(448), C::kSmemBytes, s, 1, maps, gp);
+  return launch_ex(gemm_kernel<KIND, SPARSE, SPLIT, GATHER>, grid, dim3(448), C::kSmemBytes, s, 1, maps, gp);
 }
 
 // Workspace of sharq_linear_ws.  Every counter sits in a fixed region at the
@@ -354,7 +358,7 @@ sharq_status check_prepared(const sharq_prepared* a) {
   sharq_status st = check_shape(a->k, a->t, false);
   if (st != SHARQ_OK) return st;
   if (a->fmt != SHARQ_MXFP4 && a->fmt != SHARQ_NVFP4) return fail(SHARQ_ERR_INVALID, "bad format %d", (int)a->fmt);
-  if (a->pat < SHARQ_NM_2_4 || a->pat > SHARQ_NM_8_16) return fail(SHARQ_ERR_INVALID, "bad pattern %d", (int)a->pat);
+  if (a->pat < SHARQ_NM_2_4 || a->pat > SHARQ_NM_8_16_PAIR) return fail(SHARQ_ERR_INVALID, "bad pattern %d", (int)a->pat);
   const void* ptrs[6] = {a->meta, a->bb_codes, a->bb_scales, a->res_codes, a->res_scales, a->tensor};
   for (int i = 0; i < 6; i++) {
     if (!ptrs[i]) return fail(SHARQ_ERR_INVALID, "prepared buffer %d is NULL", i);
@@ -405,7 +409,7 @@ int pair_max_resident() {
   return v;
 }
 
-// CTA-pair GEMM: clusters of 2 CTAs, one per SM, persistent over 256 x 256 tiles.
+// CTA-pair GEMM: clusters of 2 CTAs, one per SM, persistent over 256 x BN tiles.
 template <int KIND>
 sharq_status launch_pair(const GemmMaps& maps, const GemmParams& gp, cudaStream_t s) {
   using C = PairCfg<KIND>;
@@ -471,7 +475,8 @@ sharq_status run_gemv(const sharq_prepared* a, const sharq_weight* w, void* y, s
     return a->pat == SHARQ_NM_8_16 ? launch_gemv<FMT_NV, PAT_816>(gp, t, s) : launch_gemv<FMT_NV, PAT_48P>(gp, t, s);
   switch (a->pat) {
     case SHARQ_NM_2_4: return launch_gemv<FMT_MX, PAT_24>(gp, t, s);
-    case SHARQ_NM_4_8_PAIR: return launch_gemv<FMT_MX, PAT_48P>(gp, t, s);
+    case SHARQ_NM_4_8_PAIR:
+    case SHARQ_NM_8_16_PAIR: return launch_gemv<FMT_MX, PAT_48P>(gp, t, s);  // the 4:8 pair layout
     default: return launch_gemv<FMT_MX, PAT_816>(gp, t, s);
   }
 }
@@ -552,16 +557,21 @@ sharq_status run_linear(const sharq_prepared* a, const sharq_weight* w, const in
   gp.split_acc = nullptr;
   gp.split_cnt = nullptr;
   gp.split = 0;
+  gp.gather_rows = nullptr;
+  gp.gather_src_t = gp.gather_src_tpad = 0;
+  gp.g_res_codes = gp.g_bb_codes = gp.g_meta = nullptr;
   if (ws) {
     if (ws_bytes < sk_workspace_bytes() || !aligned(ws, 16))
       return fail(SHARQ_ERR_WORKSPACE, "stream-K workspace: %zu bytes, 16-byte aligned, needed",
                   sk_workspace_bytes());
   }
   if (pairs) {
-    // CTA pairs: each SM loads half of every weight tile (128-row weight boxes)
-    st = make_map(&maps.w, w->codes, w->k / 2, w->n, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    // CTA pairs: each SM loads half of every weight tile (boxes of BNh weight rows)
+    constexpr int kPairBN = PairCfg<GK_NVF4>::BN, kPairBNh = PairCfg<GK_NVF4>::BNh;
+    static_assert(kPairBN == PairCfg<GK_MXF4>::BN && kPairBNh == PairCfg<GK_MXF4>::BNh, "one pair tile shape");
+    st = make_map(&maps.w, w->codes, w->k / 2, w->n, 128, kPairBNh, CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != SHARQ_OK) return st;
-    const int64_t tiles = (t_pad / 256) * (w->n / 256);
+    const int64_t tiles = (t_pad / 256) * (w->n / kPairBN);
     const int npairs = sm_count() / 2;
     const int resident = a->fmt == SHARQ_NVFP4 ? pair_max_resident<GK_NVF4>() : pair_max_resident<GK_MXF4>();
     const int np = resident < npairs ? resident : npairs;
@@ -681,7 +691,7 @@ sharq_status sharq_prepared_sizes(int64_t t, int64_t k, sharq_format fmt, sharq_
   sharq_status st = check_shape(k, t, false);
   if (st != SHARQ_OK) return st;
   if (fmt != SHARQ_MXFP4 && fmt != SHARQ_NVFP4) return fail(SHARQ_ERR_INVALID, "bad format %d", (int)fmt);
-  if (pat < SHARQ_NM_2_4 || pat > SHARQ_NM_8_16) return fail(SHARQ_ERR_INVALID, "bad pattern %d", (int)pat);
+  if (pat < SHARQ_NM_2_4 || pat > SHARQ_NM_8_16_PAIR) return fail(SHARQ_ERR_INVALID, "bad pattern %d", (int)pat);
   const int64_t tp = round_up(t, 128);
   const int b = fmt_block(fmt);
   if (meta_bytes) *meta_bytes = (size_t)(tp * meta_row_bytes(k, pat));
@@ -888,6 +898,62 @@ sharq_status sharq_linear_grouped(const sharq_prepared* a, const sharq_weight* w
   if (!group_offsets) return fail(SHARQ_ERR_INVALID, "group_offsets is NULL");
   if (a && a->t % 128 != 0) return fail(SHARQ_ERR_INVALID, "grouped rows must be a multiple of 128");
   return run_linear(a, w, group_offsets, y, y_dt, 3, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sharq_status sharq_linear_grouped_gather(const sharq_prepared* tokens, const int32_t* rows, int64_t routed_rows,
+                                         const sharq_weight* w, const int32_t* group_offsets, void* y,
+                                         sharq_dtype y_dt, sharq_stream stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  sharq_status st = check_prepared(tokens);
+  if (st != SHARQ_OK) return st;
+  st = check_weight(w);
+  if (st != SHARQ_OK) return st;
+  if (tokens->fmt != SHARQ_NVFP4 || tokens->pat != SHARQ_NM_4_8_PAIR)
+    return fail(SHARQ_ERR_UNSUPPORTED, "gathered rows: NVFP4 with the 4:8 pair pattern only");
+  if (w->fmt != tokens->fmt) return fail(SHARQ_ERR_INVALID, "format mismatch between activations and weight");
+  if (tokens->k != w->k) return fail(SHARQ_ERR_INVALID, "k mismatch: activations %lld, weight %lld",
+                                     (long long)tokens->k, (long long)w->k);
+  if (routed_rows <= 0 || routed_rows % 128 != 0)
+    return fail(SHARQ_ERR_INVALID, "routed_rows=%lld must be a positive multiple of 128", (long long)routed_rows);
+  if (!rows || !aligned(rows, 4)) return fail(SHARQ_ERR_INVALID, "rows must be a device int32 array");
+  if (!group_offsets) return fail(SHARQ_ERR_INVALID, "group_offsets is NULL");
+  if (!y || !aligned(y, 16)) return fail(SHARQ_ERR_INVALID, "y must be a 16-byte aligned device pointer");
+  if (y_dt != SHARQ_F32 && y_dt != SHARQ_BF16) return fail(SHARQ_ERR_INVALID, "bad y dtype %d", (int)y_dt);
+  using C = GemmCfg<GK_NVF4, true>;
+  GemmMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  st = make_map(&maps.w, w->codes, w->k / 2, w->n * w->experts, 128, C::BN, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != SHARQ_OK) return st;
+  if (y_dt == SHARQ_BF16) {
+    st = make_map(&maps.y, y, w->n * 2, routed_rows, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != SHARQ_OK) return st;
+  }
+  GemmParams gp;
+  memset(&gp, 0, sizeof(gp));
+  gp.t = routed_rows;
+  gp.t_pad = routed_rows;
+  gp.n = w->n;
+  gp.k = w->k;
+  gp.experts = w->experts;
+  gp.group_offsets = group_offsets;
+  gp.sf_res = static_cast<const uint8_t*>(tokens->res_scales);
+  gp.sf_bb = static_cast<const uint8_t*>(tokens->bb_scales);
+  gp.sf_w_dense = static_cast<const uint8_t*>(w->scales_dense);
+  gp.sf_w_sparse = static_cast<const uint8_t*>(w->scales_sparse);
+  gp.tensor_x = tokens->tensor;
+  gp.tensor_w = w->tensor;
+  gp.w_codes = w->codes;
+  gp.y = y;
+  gp.y_bf16 = y_dt == SHARQ_BF16;
+  gp.paths = 3;
+  gp.timeout_ns = wait_timeout_ns();
+  gp.gather_rows = rows;
+  gp.gather_src_t = tokens->t;
+  gp.gather_src_tpad = round_up(tokens->t, 128);
+  gp.g_res_codes = static_cast<const uint8_t*>(tokens->res_codes);
+  gp.g_bb_codes = static_cast<const uint8_t*>(tokens->bb_codes);
+  gp.g_meta = static_cast<const uint8_t*>(tokens->meta);
+  return launch_gemm<GK_NVF4, true, false, true>(maps, gp, s);
 }
 
 sharq_status sharq_sync_status(sharq_stream stream) {

@@ -16,16 +16,17 @@ import torch
 from . import build_ext
 
 MXFP4, NVFP4 = 0, 1
-NM_2_4, NM_4_8_PAIR, NM_8_16 = 0, 1, 2
+NM_2_4, NM_4_8_PAIR, NM_8_16, NM_8_16_PAIR = 0, 1, 2, 3
 F32, BF16 = 0, 1
 FORMATS = {"mxfp4": MXFP4, "nvfp4": NVFP4}
-PATTERNS = {"2:4": NM_2_4, "4:8pair": NM_4_8_PAIR, "8:16": NM_8_16}
+PATTERNS = {"2:4": NM_2_4, "4:8pair": NM_4_8_PAIR, "8:16": NM_8_16, "8:16pair": NM_8_16_PAIR}
 STATUS = {0: "SHARQ_OK", 1: "SHARQ_ERR_INVALID", 2: "SHARQ_ERR_UNSUPPORTED", 3: "SHARQ_ERR_CUDA",
           4: "SHARQ_ERR_TIMEOUT", 5: "SHARQ_ERR_WORKSPACE"}
 SYMBOLS = ["sharq_weight_sizes", "sharq_prepared_sizes", "sharq_quantize_weight", "sharq_prepare", "sharq_linear",
            "sharq_linear_paths", "sharq_linear_grouped", "sharq_sync_status", "sharq_selftest_wait_timeout",
            "sharq_last_error", "sharq_launch_count", "sharq_prepare_noalloc", "sharq_prepare_swiglu",
-           "sharq_gather_prepared", "sharq_linear_ws", "sharq_linear_workspace_size"]
+           "sharq_gather_prepared", "sharq_linear_ws", "sharq_linear_workspace_size",
+           "sharq_linear_grouped_gather"]
 NOALLOC_MAX_ROWS = 65536  # SHARQ_NOALLOC_MAX_ROWS of the C header
 
 
@@ -79,6 +80,8 @@ def lib() -> ctypes.CDLL:
             "sharq_linear": [ctypes.POINTER(sharq_prepared), ctypes.POINTER(sharq_weight), P, I, P],
             "sharq_linear_paths": [ctypes.POINTER(sharq_prepared), ctypes.POINTER(sharq_weight), P, I, I32, P],
             "sharq_linear_grouped": [ctypes.POINTER(sharq_prepared), ctypes.POINTER(sharq_weight), P, P, I, P],
+            "sharq_linear_grouped_gather": [ctypes.POINTER(sharq_prepared), P, I64, ctypes.POINTER(sharq_weight), P,
+                                            P, I, P],
             "sharq_sync_status": [P],
             "sharq_selftest_wait_timeout": [ctypes.c_uint64, P],
         }
@@ -195,6 +198,13 @@ def sharq_linear_paths(a: sharq_prepared, w: sharq_weight, y_ptr: int, y_dt, pat
 def sharq_linear_grouped(a: sharq_prepared, w: sharq_weight, offsets_ptr: int, y_ptr: int, y_dt, stream=None):
     _check(lib().sharq_linear_grouped(ctypes.byref(a), ctypes.byref(w), ctypes.c_void_p(offsets_ptr),
                                       ctypes.c_void_p(y_ptr), _dt(y_dt), _stream(stream)), "sharq_linear_grouped")
+
+
+def sharq_linear_grouped_gather(tokens: sharq_prepared, rows_ptr: int, routed_rows: int, w: sharq_weight,
+                                offsets_ptr: int, y_ptr: int, y_dt, stream=None):
+    _check(lib().sharq_linear_grouped_gather(ctypes.byref(tokens), ctypes.c_void_p(rows_ptr), int(routed_rows),
+                                             ctypes.byref(w), ctypes.c_void_p(offsets_ptr), ctypes.c_void_p(y_ptr),
+                                             _dt(y_dt), _stream(stream)), "sharq_linear_grouped_gather")
 
 
 def sharq_sync_status(stream=None):
@@ -330,4 +340,17 @@ def linear_grouped(a: Prepared, w: FP4Weight, offsets: torch.Tensor, out_dtype=t
         out = torch.zeros((a.t, w.n), dtype=out_dtype, device=a.meta.device)
     offsets = offsets.to(torch.int32).contiguous()
     sharq_linear_grouped(a.struct, w.struct, offsets.data_ptr(), out.data_ptr(), out.dtype, stream)
+    return out
+
+
+def linear_grouped_gather(tokens: Prepared, rows: torch.Tensor, w: FP4Weight, offsets: torch.Tensor,
+                          out_dtype=torch.bfloat16, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Grouped linear over routed rows read by index from the token-prepared buffers
+    (rows[r] = token of routed row r, < 0 for a padding row)."""
+    rows = rows.to(torch.int32).contiguous()
+    if out is None:
+        out = torch.zeros((rows.numel(), w.n), dtype=out_dtype, device=tokens.meta.device)
+    offsets = offsets.to(torch.int32).contiguous()
+    sharq_linear_grouped_gather(tokens.struct, rows.data_ptr(), rows.numel(), w.struct, offsets.data_ptr(),
+                                out.data_ptr(), out.dtype, stream)
     return out

@@ -28,7 +28,7 @@
  *                 row is stored as ceil(R/128) x ceil(S/4) blocks of 512 bytes,
  *                 row-block major; inside a block, row r and scale s sit at
  *                 byte (r%32)*16 + ((r/32)%4)*4 + (s%4);
- *      meta       row-major, 2:4 and 4:8 pair: one nibble per group of 4 (8)
+ *      meta       row-major, 2:4 and 4:8 pair (and 8:16 re-packed): one nibble per group of 4 (8)
  *                 K elements, nibble = i0 | i1 << 2 with the kept element
  *                 (pair) indices i0 < i1, group g in byte g/2, low nibble
  *                 first; 8:16: one little-endian uint16 mask per group of 16.
@@ -63,8 +63,13 @@ typedef enum { SHARQ_MXFP4 = 0, SHARQ_NVFP4 = 1 } sharq_format;
 
 /* Online N:M activation masks: 2:4 (Huawei problem 137-2 asks for MXFP4/HiF4
  * combined with 2:4), the NVFP4 4:8 pair pattern (SharQ Section 2.2: two of four
- * adjacent pairs kept), and 8:16 (paper on 2:4-to-8:16 sparsity patterns, abstract). */
-typedef enum { SHARQ_NM_2_4 = 0, SHARQ_NM_4_8_PAIR = 1, SHARQ_NM_8_16 = 2 } sharq_pattern;
+ * adjacent pairs kept), and 8:16 (paper on 2:4-to-8:16 sparsity patterns, abstract).
+ * SHARQ_NM_8_16_PAIR runs the 8:16 selection on the sparse tensor cores, whose
+ * pattern is the 4:8 pair: the top 8 of each group of 16 are found as for 8:16,
+ * then each group of 8 keeps the two adjacent pairs holding most of them (ties:
+ * the larger magnitude, then the lower pair); the rest goes to the residual.  Its
+ * buffers use the 4:8 pair layouts, and sharq_linear runs the 4:8 pair GEMM. */
+typedef enum { SHARQ_NM_2_4 = 0, SHARQ_NM_4_8_PAIR = 1, SHARQ_NM_8_16 = 2, SHARQ_NM_8_16_PAIR = 3 } sharq_pattern;
 
 typedef enum { SHARQ_F32 = 0, SHARQ_BF16 = 1 } sharq_dtype;
 
@@ -258,6 +263,23 @@ sharq_status sharq_linear_paths(const sharq_prepared* a, const sharq_weight* w, 
  * group are left unwritten. */
 sharq_status sharq_linear_grouped(const sharq_prepared* a, const sharq_weight* w, const int32_t* group_offsets,
                                   void* y, sharq_dtype y_dt, sharq_stream stream);
+
+/* sharq_linear_grouped on rows gathered inside the GEMM (SharQ evaluates
+ * Qwen3-30B-A3B; every token goes to several experts).  The routed operand is
+ * never written out: routed row r (0 <= r < routed_rows) is row rows[r] of the
+ * token-prepared buffers `tokens` (from sharq_prepare over the tokens), read
+ * by index as each tile's operands are loaded; rows[r] < 0 or >= tokens->t
+ * stands for an all-zero input row (the padding rows of an expert's segment).
+ * The result equals sharq_gather_prepared(tokens, rows) followed by
+ * sharq_linear_grouped, bit for bit.
+ * rows: DEVICE, routed_rows int32 values; routed_rows a positive multiple of 128;
+ * group_offsets as in sharq_linear_grouped, last = routed_rows; y: routed_rows * n.
+ * Supported: NVFP4 with the 4:8 pair pattern (a padding row is encoded with zero
+ * E4M3 scales); other formats and patterns return SHARQ_ERR_UNSUPPORTED.  Index
+ * values are not checked on the host. */
+sharq_status sharq_linear_grouped_gather(const sharq_prepared* tokens, const int32_t* rows, int64_t routed_rows,
+                                         const sharq_weight* w, const int32_t* group_offsets, void* y,
+                                         sharq_dtype y_dt, sharq_stream stream);
 
 /* Synchronizes the stream, then reports and clears this device's error word. */
 sharq_status sharq_sync_status(sharq_stream stream);

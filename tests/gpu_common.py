@@ -32,7 +32,7 @@ def readback(p: sharq.Prepared, rows=None) -> dict:
     b = 16 if nv else 32
     sel = np.arange(t) if rows is None else np.asarray(rows)
     out = {}
-    out["meta"] = p.meta.cpu().numpy()[: tp * (k // 16 if p.pat == sharq.NM_4_8_PAIR else k // 8)].reshape(tp, -1)[sel]
+    out["meta"] = p.meta.cpu().numpy()[: tp * (k // 16 if p.pat in (sharq.NM_4_8_PAIR, sharq.NM_8_16_PAIR) else k // 8)].reshape(tp, -1)[sel]
     bbw = k // 2 if p.pat == sharq.NM_8_16 else k // 4
     out["bb_codes"] = p.bb_codes.cpu().numpy()[: tp * bbw].reshape(tp, bbw)[sel]
     sb = k // b if p.pat == sharq.NM_8_16 else k // (2 * b)

@@ -130,3 +130,18 @@ def test_linear_ws_requires_a_workspace(L):
         sharq.sharq_linear_ws(a, w, 16, sharq.BF16, 0, 0, 0)
     assert ei.value.status == 5 and "workspace" in str(ei.value)
     assert sharq.sharq_launch_count() == before
+
+
+def test_grouped_gather_rejects_on_host(L):
+    """The in-GEMM row gather takes NVFP4 with the 4:8 pair only, routed rows in
+    multiples of 128 and an index array; all checked before any launch."""
+    before = sharq.sharq_launch_count()
+    w = sharq.sharq_weight(16, 16, 16, 16, 256, 512, 4, 1)
+    ok = sharq.sharq_prepared(16, 16, 16, 16, 16, 16, 300, 512, 1, 1)
+    for tok, rows, routed, status in ((sharq.sharq_prepared(16, 16, 16, 16, 16, 16, 300, 512, 0, 1), 16, 256, 2),
+                                      (sharq.sharq_prepared(16, 16, 16, 16, 16, 16, 300, 512, 1, 2), 16, 256, 2),
+                                      (ok, 16, 200, 1), (ok, 0, 256, 1), (ok, 18, 256, 1)):
+        with pytest.raises(sharq.SharqError) as ei:
+            sharq.sharq_linear_grouped_gather(tok, rows, routed, w, 16, 16, sharq.BF16, 0)
+        assert ei.value.status == status, str(ei.value)
+    assert sharq.sharq_launch_count() == before

@@ -7,7 +7,7 @@ import torch
 
 import oracle
 from activation_sparsity_fp4_b200 import sharq, workloads
-from gpu_common import assert_prep_equal, readback, to_dev
+from gpu_common import assert_close_gemm, assert_prep_equal, readback, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -101,3 +101,64 @@ def test_gather_full_moe_layer_feeds_grouped_gemm(cuda_ok):
     assert g["tensor"][0] == np.float32(amax)
     ref = oracle.prepare(cfg["x"][sel], "nvfp4", "4:8pair", act_amax=amax)
     assert_prep_equal(g, ref, "4:8pair")
+
+
+def _expert_weight(seed, experts, n, k):
+    rng = np.random.default_rng(seed)
+    return workloads.to_bf16_values((rng.standard_normal((experts, n, k)) * 0.02).astype(np.float32))
+
+
+@pytest.mark.parametrize("y_dtype", [torch.float32, torch.bfloat16])
+def test_gemm_gathers_rows_itself(cuda_ok, y_dtype):
+    """The grouped GEMM reading routed rows by index from the token-prepared
+    buffers equals the materialised gather followed by the grouped GEMM, bit for
+    bit: small ragged routing (padding rows in every segment), repeated rows, and
+    indices at or past the token count (zero rows)."""
+    k, n, t_tok, experts = 768, 512, 300, 8
+    x_tok = _tokens(31, t_tok, k)
+    _, offsets, gather = _routing(32, t_tok, experts, 2)
+    rows = gather.copy()
+    rows[5] = t_tok + 7   # past the tokens: a zero row
+    rows[9] = rows[10]    # the same token twice
+    w = _expert_weight(33, experts, n, k)
+    wq = sharq.FP4Weight.quantize(to_dev(w, "bf16"), "nvfp4")
+    src = sharq.prepare(to_dev(x_tok, "bf16"), "nvfp4", "4:8pair")
+    rows_d = torch.from_numpy(rows.astype(np.int32)).cuda()
+    off_d = torch.from_numpy(offsets.astype(np.int32)).cuda()
+    y_in = sharq.linear_grouped_gather(src, rows_d, wq, off_d, out_dtype=y_dtype)
+    routed = sharq.gather_prepared(src, rows_d)
+    y_mat = sharq.linear_grouped(routed, wq, off_d, out_dtype=y_dtype)
+    sharq.sharq_sync_status()
+    bad = torch.nonzero(y_in != y_mat)
+    assert bad.numel() == 0, f"{bad.shape[0]} outputs differ, first at {bad[:3].tolist()}"
+    # and against the oracle on a few real rows of two experts
+    amax = float(src.tensor[0].item())
+    assert np.float32(amax) == np.float32(oracle.rows_amax(x_tok))
+    yn = y_in.float().cpu().numpy()
+    for e in (0, experts - 1):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        sel = np.array([r for r in range(lo, hi) if 0 <= rows[r] < t_tok][:6])
+        prep = oracle.prepare(x_tok[rows[sel]], "nvfp4", "4:8pair", act_amax=amax)
+        ref = oracle.linear_ref(prep, oracle.quantize_weight(w[e], "nvfp4"))
+        if y_dtype == torch.float32:
+            assert_close_gemm(yn[sel], ref, f"gathered GEMM, expert {e}")
+    # padding rows (index < 0) hold the zero row's output
+    pad = np.flatnonzero(rows < 0)
+    assert pad.size > 0 and float(y_in[torch.from_numpy(pad).cuda()].abs().max()) == 0.0
+
+
+def test_gemm_gathers_rows_full_moe_layer(cuda_ok):
+    """Qwen3-30B-A3B gate/up at full size (4096 tokens, 128 experts, top 8,
+    32768 routed rows): the in-GEMM gather equals gather + grouped GEMM bit for bit."""
+    cfg = workloads.qwen_moe()
+    x_tok, gather, offsets = cfg["x_tok"], cfg["gather"], cfg["offsets"]
+    w = cfg["w_gu"]
+    e_, n, k = w.shape
+    wq = sharq.FP4Weight.quantize(to_dev(w, "bf16"), "nvfp4")
+    src = sharq.prepare(to_dev(x_tok, "bf16"), "nvfp4", "4:8pair")
+    rows_d = torch.from_numpy(gather.astype(np.int32)).cuda()
+    off_d = torch.from_numpy(offsets.astype(np.int32)).cuda()
+    y_in = sharq.linear_grouped_gather(src, rows_d, wq, off_d)
+    y_mat = sharq.linear_grouped(sharq.gather_prepared(src, rows_d), wq, off_d)
+    sharq.sharq_sync_status()
+    assert torch.equal(y_in, y_mat)

@@ -12,7 +12,8 @@ from gpu_common import assert_close_gemm, gpu_prepare, readback, assert_prep_equ
 
 pytestmark = pytest.mark.gpu
 
-LINEAR_CASES = [("nvfp4", "4:8pair"), ("nvfp4", "8:16"), ("mxfp4", "4:8pair"), ("mxfp4", "8:16"), ("mxfp4", "2:4")]
+LINEAR_CASES = [("nvfp4", "4:8pair"), ("nvfp4", "8:16"), ("mxfp4", "4:8pair"), ("mxfp4", "8:16"), ("mxfp4", "2:4"),
+                ("nvfp4", "8:16pair"), ("mxfp4", "8:16pair")]
 
 
 def _w(seed, n, k, scale=0.02):
@@ -221,9 +222,10 @@ def test_linear_down_proj_2048_sampled_rows(cuda_ok):
     assert_close_gemm(y[rows], oracle.linear_ref(prep, wq), "down_proj sampled rows")
 
 
-@pytest.mark.parametrize("pat", ["4:8pair", "8:16"])
+@pytest.mark.parametrize("pat", ["4:8pair", "8:16", "8:16pair"])
 def test_linear_wan_full_size_sampled_rows(cuda_ok, pat):
-    """Wan2.2 DiT linear (32768 x 5120 -> 5120), NVFP4 with RMSNorm, 4:8 pair and 8:16."""
+    """Wan2.2 DiT linear (32768 x 5120 -> 5120), NVFP4 with RMSNorm, 4:8 pair, 8:16
+    and 8:16 re-packed into the 4:8 pair layout."""
     cfg = workloads.wan(pat=pat)
     p, _, y = _run_linear(cfg["x"], cfg["w"], "nvfp4", pat, gamma=cfg["gamma"], out_dtype=torch.float32)
     rows = np.sort(np.random.default_rng(12).choice(32768, 24, replace=False))

@@ -14,7 +14,7 @@ from gpu_common import assert_prep_equal, gpu_prepare, readback
 pytestmark = pytest.mark.gpu
 
 FMTS = ["mxfp4", "nvfp4"]
-PATS = ["2:4", "4:8pair", "8:16"]
+PATS = ["2:4", "4:8pair", "8:16", "8:16pair"]
 
 
 def _x(seed, t, k, outliers=True):
