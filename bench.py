@@ -58,20 +58,25 @@ WORKLOADS = {
            "NVFP4, 4:8 pair",
     "wan_816": "Wan2.2-14B DiT linear: X 32768x5120 bf16 ~N(0,1) + 16 outlier channels x50, RMSNorm; W 5120x5120; "
                "NVFP4, 8:16",
+    "wan_816pair": "Wan2.2-14B DiT linear: X 32768x5120 bf16 ~N(0,1) + 16 outlier channels x50, RMSNorm; W 5120x5120; "
+                   "NVFP4, 8:16 selection re-packed into the 4:8 pair layout (sparse tensor cores)",
     "down_proj_swiglu": "Llama-3.1-8B down_proj from its gate and up inputs: gate, up 2048x14336 bf16 ~N(0,1), "
                         "h = SiLU(gate)*up formed inside the prep kernel; W 4096x14336 ~N(0,0.01^2); MXFP4, 2:4",
     "qwen_moe_gate_up": "Qwen3-30B-A3B MoE gate/up: 4096 tokens top-8 of 128 experts -> 32768 routed rows (each expert "
                         "padded to 128 rows), hidden 2048; per expert W 1536x2048; NVFP4, 4:8 pair, no norm; grouped",
     "qwen_moe_gate_up_gather": "Qwen3-30B-A3B MoE gate/up as qwen_moe_gate_up, but each of the 4096 tokens prepared "
                                "once and its prepared row gathered into the 32768 routed rows; grouped",
+    "qwen_moe_gate_up_gemm_gather": "Qwen3-30B-A3B MoE gate/up as qwen_moe_gate_up, the 4096 tokens prepared once "
+                                    "and the grouped GEMM reading each routed row by index from them (no routed "
+                                    "copy); grouped",
     "qwen_moe_down": "Qwen3-30B-A3B MoE down: 32768 routed rows (expert order, each expert padded to 128 rows) x 768 "
                      "bf16 0.5*t3; per expert W 2048x768; NVFP4, 4:8 pair, no norm; grouped",
 }
 
 # the shapes the headline line also reports (name, rows or None)
 EXTRA = [("tiny", None), ("down_proj", None), ("down_proj", 1), ("down_proj", 16), ("down_proj", 64),
-         ("down_proj", 256), ("wan", None), ("wan_816", None), ("qwen_moe_gate_up_gather", None),
-         ("qwen_moe_down", None)]
+         ("down_proj", 256), ("wan", None), ("wan_816", None), ("wan_816pair", None), ("qwen_moe_gate_up_gather", None),
+         ("qwen_moe_gate_up_gemm_gather", None), ("qwen_moe_down", None)]
 
 L2_BYTES = 126 * 1024 * 1024
 ROTATE_BYTES = 3 * L2_BYTES  # the rotating sets of a workload cover at least this much
@@ -81,7 +86,7 @@ def prep_bytes_per_elem(fmt: str, pat: str, x_bytes: int = 2) -> float:
     """Algorithmic bytes of sharq_prepare per element of X: X read, then backbone codes, metadata,
     backbone scales, residual codes and residual scales written (layouts of sharq.h)."""
     b = 16 if fmt == "nvfp4" else 32
-    meta = 1 / 16 if pat == "4:8pair" else 1 / 8
+    meta = 1 / 16 if pat in ("4:8pair", "8:16pair") else 1 / 8
     bb_codes = 0.5 if pat == "8:16" else 0.25
     bb_sf = 1 / b if pat == "8:16" else 1 / (2 * b)  # 8:16 keeps the dense view (each scale twice)
     return x_bytes + bb_codes + meta + bb_sf + 0.5 + 1 / b
@@ -113,14 +118,15 @@ def make_workload(name: str, tokens: int | None = None) -> dict:
                   pat="4:8pair", offsets=c["offsets"], t=t, k=k, n=n, real_rows=int(c["counts"].sum()),
                   first_group=(int(c["offsets"][0]), int(c["offsets"][1])), gate=None, up=None)
         if name.endswith("_gather"):
-            wl.update(tokens=c["x_tok"], gather=c["gather"])
+            wl.update(tokens=c["x_tok"], gather=c["gather"], gemm_gather=name.endswith("_gemm_gather"))
         return wl
     kw = {"t": tokens} if tokens and name in ("q_proj", "down_proj", "down_proj_swiglu") else {}
     desc = WORKLOADS[name].replace("2048x", f"{tokens}x") if kw else WORKLOADS[name]
     gen = {"tiny": workloads.tiny, "q_proj": workloads.q_proj, "down_proj": workloads.down_proj,
-           "down_proj_swiglu": workloads.down_proj, "wan": workloads.wan, "wan_816": workloads.wan}[name]
-    if name == "wan_816":
-        kw = {"pat": "8:16"}
+           "down_proj_swiglu": workloads.down_proj, "wan": workloads.wan, "wan_816": workloads.wan,
+           "wan_816pair": workloads.wan}[name]
+    if name in ("wan_816", "wan_816pair"):
+        kw = {"pat": "8:16" if name == "wan_816" else "8:16pair"}
     c = _config(gen, **kw)
     t, k = c["x"].shape
     wl = dict(name=name, desc=desc, x=c["x"], x_dtype=c.get("x_dtype", "bf16"), gamma=c["gamma"], eps=c["eps"], w=c["w"],
@@ -322,6 +328,7 @@ class LayerSets:
         T, K, N, fmt, pat = wl["t"], wl["k"], wl["n"], wl["fmt"], wl["pat"]
         self.swiglu = wl["gate"] is not None
         self.gathered = wl.get("gather") is not None
+        self.gemm_gather = bool(wl.get("gemm_gather"))  # rows read by index inside the GEMM
         x_src = wl["gate"] if self.swiglu else (wl["tokens"] if self.gathered else wl["x"])
         self.x_dt = torch.float32 if wl.get("x_dtype") == "f32" else torch.bfloat16
         self.x_host = torch.from_numpy(x_src).to(self.x_dt).pin_memory()
@@ -341,7 +348,7 @@ class LayerSets:
         for i in range(self.R):
             self.x.append(self.x_host.to(dev))
             self.up.append(self.up_host.to(dev) if self.swiglu else None)
-            self.prep.append(sharq.Prepared(T, K, fmt, pat, dev))
+            self.prep.append(None if self.gemm_gather else sharq.Prepared(T, K, fmt, pat, dev))
             self.prep_tok.append(sharq.Prepared(self.x_host.shape[0], K, fmt, pat, dev) if self.gathered else None)
             self.y.append(torch.zeros((T, N), dtype=torch.bfloat16, device=dev))
             self.wq.append(sharq.FP4Weight.quantize(w, fmt))  # the same codes in every set
@@ -357,7 +364,8 @@ class LayerSets:
         elif self.gathered:
             sharq.prepare(self.x[i], wl["fmt"], wl["pat"], self.gamma, wl["eps"], act_amax=act_amax,
                           out=self.prep_tok[i], stream=stream)
-            sharq.gather_prepared(self.prep_tok[i], self.rows, out=self.prep[i], stream=stream)
+            if not self.gemm_gather:
+                sharq.gather_prepared(self.prep_tok[i], self.rows, out=self.prep[i], stream=stream)
         else:
             sharq.prepare(self.x[i], wl["fmt"], wl["pat"], self.gamma, wl["eps"], act_amax=act_amax,
                           out=self.prep[i], stream=stream)
@@ -366,6 +374,9 @@ class LayerSets:
         from activation_sparsity_fp4_b200 import sharq
         if self.offsets is None:
             sharq.linear(self.prep[i], self.wq[i], out=self.y[i], workspace=self.ws[i], stream=stream)
+        elif self.gemm_gather:
+            sharq.linear_grouped_gather(self.prep_tok[i], self.rows, self.wq[i], self.offsets, out=self.y[i],
+                                        stream=stream)
         else:
             sharq.linear_grouped(self.prep[i], self.wq[i], self.offsets, out=self.y[i], stream=stream)
 
@@ -431,7 +442,7 @@ def measure(name: str, tokens, steps: int, warmup: int, e2e_steps: int, dev, pg,
         gemm_ms = timed_replay_ms(g_gemm, stream) / m
     sharq.sharq_sync_status()
     # caller-given amax variant of prep (no extra read of x), for the prep roofline
-    amax = float(L.prep[0].tensor[0].item())
+    amax = float((L.prep_tok[0] if L.gemm_gather else L.prep[0]).tensor[0].item())
     g_given = graph_of(lambda i: L.do_prep(i, amax if fmt == "nvfp4" else 0.0), m, R)
     given_ms = timed_replay_ms(g_given, stream) / m
     sharq.sharq_sync_status()
@@ -498,14 +509,17 @@ def measure(name: str, tokens, steps: int, warmup: int, e2e_steps: int, dev, pg,
     achieved = work / gemm_s / 1e12
     bpe = prep_bytes_per_elem(fmt, pat, 4 if (L.swiglu or L.x_dt == torch.float32) else 2)
     prep_bytes = bpe * T * K
-    if L.gathered:  # prep of the tokens, then each routed row's prepared bytes read and written once
+    if L.gemm_gather:  # prep of the tokens only (the GEMM reads the routed rows by index)
+        prep_bytes = bpe * L.x_host.shape[0] * K
+    elif L.gathered:  # prep of the tokens, then each routed row's prepared bytes read and written once
         prep_bytes = bpe * L.x_host.shape[0] * K + 2 * (bpe - 2) * T * K + 4 * T
     prep_gbs = prep_bytes / (prep_ms / 1e3) / 1e9
     given_gbs = prep_bytes / (given_ms / 1e3) / 1e9
     grouped = wl["offsets"] is not None
-    kernel = {"4:8pair": "sparse", "2:4": "sparse", "8:16": "dense backbone"}[pat]
+    kernel = {"4:8pair": "sparse", "8:16pair": "sparse", "2:4": "sparse", "8:16": "dense backbone"}[pat]
     kname = ("gemv_kernel" if (not grouped and T <= 4) else
-             "gemm_pair_kernel" if (not grouped and pat == "4:8pair" and ((T + 127) // 128 * 128) % 256 == 0)
+             "gemm_pair_kernel" if (not grouped and pat in ("4:8pair", "8:16pair")
+                                    and ((T + 127) // 128 * 128) % 256 == 0)
              else "gemm_kernel")
     kkind = "MXF8" if (fmt == "mxfp4" and pat == "2:4") else ("NVF4" if fmt == "nvfp4" else "MXF4")
     klabel = (f"gemv_kernel<{'MX' if fmt == 'mxfp4' else 'NV'}, {pat}, {T} rows>" if kname == "gemv_kernel"
