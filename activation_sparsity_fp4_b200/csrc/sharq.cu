@@ -14,6 +14,7 @@
 #include "../../include/sharq.h"
 #include "gemm.cuh"
 #include "gemm_pair.cuh"
+#include "gemm_swap.cuh"
 #include "gemv.cuh"
 #include "prep.cuh"
 
@@ -87,6 +88,15 @@ bool stream_k_enabled() {
 bool gemv_enabled() {
   static const bool v = [] {
     const char* e = getenv("SHARQ_GEMV");
+    return !(e && e[0] == '0');
+  }();
+  return v;
+}
+
+// SHARQ_SWAP=0 keeps few-row products (5..64 rows) on the activation-as-A kernels (for comparison).
+bool swap_enabled() {
+  static const bool v = [] {
+    const char* e = getenv("SHARQ_SWAP");
     return !(e && e[0] == '0');
   }();
   return v;
@@ -481,6 +491,92 @@ sharq_status run_gemv(const sharq_prepared* a, const sharq_weight* w, void* y, s
   }
 }
 
+// Few rows: the weight as the 128-row MMA operand (gemm_swap.cuh), the K loop of
+// each 128-row weight tile split over the SMs when a workspace is given.
+// Measured on B200 (GEMM alone): down_proj 4 rows 42.9 -> 23.0 us, 16 rows 28.3
+// -> 23.2 us, q_proj 16 rows 22.8 -> 16.8 us; at 1 row the CUDA-core form is
+// faster (19.3 vs 23.4 us), at 64 rows the activation-as-A kernels (30.3 vs
+// 36.0 us), so it serves 2..32 rows.
+constexpr int64_t kSwapMinRows = 2, kSwapMaxRows = 32;
+template <int KIND, int BL, int TN>
+sharq_status launch_swap(const sharq_prepared* a, const sharq_weight* w, void* y, sharq_dtype y_dt, void* ws,
+                         size_t ws_bytes, cudaStream_t s) {
+  using C = SwapCfg<KIND, BL, TN>;
+  static bool configured = false;
+  if (!configured) {
+    SHARQ_CUDA(cudaFuncSetAttribute(gemm_swap_kernel<KIND, BL, TN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    C::kSmemBytes));
+    configured = true;
+  }
+  const int64_t t_pad = round_up(a->t, 128), k = w->k;
+  SwapMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  sharq_status st = make_map(&maps.w, w->codes, k / 2, w->n, 128, C::BM, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != SHARQ_OK) return st;
+  st = make_map(&maps.r, a->res_codes, k / 2, t_pad, 128, TN, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != SHARQ_OK) return st;
+  if (BL == SW_DENSE) {
+    st = make_map(&maps.c, a->bb_codes, k / 2, t_pad, 128, TN, CU_TENSOR_MAP_SWIZZLE_128B);
+  } else {
+    st = make_map(&maps.c, a->bb_codes, k / 4, t_pad, C::kCRow, TN, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != SHARQ_OK) return st;
+    st = make_map(&maps.e, a->meta, meta_row_bytes(k, a->pat), t_pad, C::kMetaRow, TN, CU_TENSOR_MAP_SWIZZLE_NONE);
+  }
+  if (st != SHARQ_OK) return st;
+  SwapParams sp;
+  memset(&sp, 0, sizeof(sp));
+  sp.t = a->t;
+  sp.n = w->n;
+  sp.k = k;
+  sp.k_tiles = k / C::BK;
+  sp.w_codes = static_cast<const uint8_t*>(w->codes);
+  sp.sf_w = static_cast<const uint8_t*>(w->scales_dense);
+  sp.sf_res = static_cast<const uint8_t*>(a->res_scales);
+  sp.sf_bb = static_cast<const uint8_t*>(a->bb_scales);
+  sp.tensor_x = a->tensor;
+  sp.tensor_w = w->tensor;
+  sp.y = y;
+  sp.y_bf16 = y_dt == SHARQ_BF16;
+  sp.timeout_ns = wait_timeout_ns();
+  const int64_t tiles = w->n / C::BM;
+  const int sms = sm_count();
+  int64_t split = 1;
+  if (ws && tiles <= sms) {
+    // slices: enough work items for every SM, at least two K tiles each, and one
+    // fp32 slot of [n][TN] raw sums per slice in the workspace
+    split = sms / tiles;
+    if (split > sp.k_tiles / 2) split = sp.k_tiles / 2;
+    const size_t slot = (size_t)w->n * TN * sizeof(float);
+    while (split > 1 && ws_data_offset() + (size_t)split * slot > ws_bytes) split--;
+    if (split < 1) split = 1;
+  }
+  sp.split = (int32_t)split;
+  if (split > 1) {
+    sp.acc = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + ws_data_offset());
+    sp.cnt = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + ws_split_cnt_offset());
+  }
+  return launch_ex(gemm_swap_kernel<KIND, BL, TN>, dim3((unsigned)(tiles * split)), dim3(192), C::kSmemBytes, s, 1,
+                   maps, sp);
+}
+
+template <int KIND, int BL>
+sharq_status swap_rows(const sharq_prepared* a, const sharq_weight* w, void* y, sharq_dtype y_dt, void* ws,
+                       size_t ws_bytes, cudaStream_t s) {
+  static_assert(kSwapMaxRows <= 32, "one activation tile width");
+  return launch_swap<KIND, BL, 32>(a, w, y, y_dt, ws, ws_bytes, s);
+}
+
+sharq_status run_swap(const sharq_prepared* a, const sharq_weight* w, void* y, sharq_dtype y_dt, void* ws,
+                      size_t ws_bytes, cudaStream_t s) {
+  const bool pair = a->pat == SHARQ_NM_4_8_PAIR || a->pat == SHARQ_NM_8_16_PAIR;
+  if (a->fmt == SHARQ_NVFP4)
+    return pair ? swap_rows<GK_NVF4, SW_PAIR>(a, w, y, y_dt, ws, ws_bytes, s)
+                : swap_rows<GK_NVF4, SW_DENSE>(a, w, y, y_dt, ws, ws_bytes, s);
+  if (pair) return swap_rows<GK_MXF4, SW_PAIR>(a, w, y, y_dt, ws, ws_bytes, s);
+  return a->pat == SHARQ_NM_2_4 ? swap_rows<GK_MXF4, SW_24>(a, w, y, y_dt, ws, ws_bytes, s)
+                                : swap_rows<GK_MXF4, SW_DENSE>(a, w, y, y_dt, ws, ws_bytes, s);
+}
+
 sharq_status run_linear(const sharq_prepared* a, const sharq_weight* w, const int32_t* offsets, void* y,
                         sharq_dtype y_dt, int32_t paths, cudaStream_t s, void* ws = nullptr, size_t ws_bytes = 0) {
   sharq_status st = check_prepared(a);
@@ -497,7 +593,13 @@ sharq_status run_linear(const sharq_prepared* a, const sharq_weight* w, const in
     return fail(SHARQ_ERR_INVALID, "a stacked weight needs sharq_linear_grouped");
   if (a->fmt == SHARQ_NVFP4 && a->pat == SHARQ_NM_2_4)
     return fail(SHARQ_ERR_UNSUPPORTED, "NVFP4 with element-wise 2:4 has no sparse tensor-core kind");
-  if (offsets == nullptr && a->t <= kGemvMaxRows && gemv_enabled()) return run_gemv(a, w, y, y_dt, paths, s);
+  const bool swap = offsets == nullptr && a->t >= kSwapMinRows && a->t <= kSwapMaxRows && paths == 3 && swap_enabled();
+  if (offsets == nullptr && a->t <= kGemvMaxRows && gemv_enabled() && !swap) return run_gemv(a, w, y, y_dt, paths, s);
+  if (swap) {
+    if (ws && (ws_bytes < sk_workspace_bytes() || !aligned(ws, 16)))
+      return fail(SHARQ_ERR_WORKSPACE, "workspace: %zu bytes, 16-byte aligned, needed", sk_workspace_bytes());
+    return run_swap(a, w, y, y_dt, ws, ws_bytes, s);
+  }
 
   const int64_t t_pad = round_up(a->t, 128);
   const bool sparse = a->pat != SHARQ_NM_8_16;

@@ -278,3 +278,32 @@ def test_linear_q_proj_full_size_sampled_rows(cuda_ok):
     prep = oracle.prepare(cfg["x"][rows], "nvfp4", "4:8pair", gamma=cfg["gamma"], act_amax=amax)
     wq = oracle.quantize_weight(cfg["w"], "nvfp4")
     assert_close_gemm(y[rows], oracle.linear_ref(prep, wq), "q_proj sampled rows")
+
+
+SWAP_CASES = [("nvfp4", "4:8pair"), ("nvfp4", "8:16"), ("nvfp4", "8:16pair"), ("mxfp4", "2:4"),
+              ("mxfp4", "4:8pair"), ("mxfp4", "8:16")]
+
+
+@pytest.mark.parametrize("fmt,pat", SWAP_CASES)
+@pytest.mark.parametrize("t", [2, 5, 32, 33, 64])
+def test_linear_few_rows_weight_as_operand_a(cuda_ok, fmt, pat, t):
+    """2..32 rows: the weight tile is the 128-row MMA operand and the rows the
+    narrow one (backbone expanded on chip); 33 and 64 rows: the activation-as-A
+    kernels next to it.  With and without the K split over the SMs, against
+    fp64; bf16 = rounded fp32; the split repeats bit for bit."""
+    k, n = 2048, 1024
+    x, w = _x(60 + t, t, k), _w(61, n, k)
+    p = gpu_prepare(x, "bf16", fmt, pat)
+    wq = gpu_weight(w, "bf16", fmt)
+    ws = sharq.linear_workspace()
+    y1 = sharq.linear(p, wq, out_dtype=torch.float32).clone()
+    y2 = sharq.linear(p, wq, out_dtype=torch.float32, workspace=ws).clone()
+    y3 = sharq.linear(p, wq, out_dtype=torch.float32, workspace=ws).clone()
+    yb = sharq.linear(p, wq, out_dtype=torch.bfloat16, workspace=ws)
+    sharq.sharq_sync_status()
+    prep, wqo = _ref(x, w, fmt, pat)
+    ref = oracle.linear_ref(prep, wqo)
+    assert_close_gemm(y1.cpu().numpy(), ref, f"{fmt} {pat} t={t}, one slice")
+    assert_close_gemm(y2.cpu().numpy(), ref, f"{fmt} {pat} t={t}, K split")
+    assert torch.equal(y2, y3), "the K split is not reproducible"
+    assert torch.equal(yb, y2.to(torch.bfloat16)), "bf16 output != fp32 output rounded to bf16"
