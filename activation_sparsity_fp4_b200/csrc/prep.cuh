@@ -821,6 +821,40 @@ __device__ __forceinline__ void quantize_unit(float (&h)[32], float g_enc, float
   }
 }
 
+// Writes one unit's outputs (row r, unit u) in the documented layouts.
+template <int FMT, int PAT>
+__device__ __forceinline__ void store_unit(const PrepParams& p, int64_t r, int u, int64_t s_bb, int64_t s_res,
+                                           uint32_t meta, const uint32_t (&bc)[4], uint32_t bsc,
+                                           const uint32_t (&rc)[4], uint32_t rsc0, uint32_t rsc1) {
+  const int64_t k = p.k;
+  if constexpr (pair_layout(PAT)) {
+    *reinterpret_cast<uint16_t*>(p.meta + r * (k / 16) + 2 * u) = (uint16_t)meta;
+  } else {
+    *reinterpret_cast<uint32_t*>(p.meta + r * (k / 8) + 4 * u) = meta;
+  }
+  if constexpr (PAT == PAT_816) {
+    *reinterpret_cast<uint4*>(p.bb_codes + r * (k / 2) + 16 * u) = make_uint4(bc[0], bc[1], bc[2], bc[3]);
+  } else {
+    *reinterpret_cast<uint2*>(p.bb_codes + r * (k / 4) + 8 * u) = make_uint2(bc[0], bc[1]);
+  }
+  *reinterpret_cast<uint4*>(p.res_codes + r * (k / 2) + 16 * u) = make_uint4(rc[0], rc[1], rc[2], rc[3]);
+  if constexpr (FMT == FMT_NV) {
+    if constexpr (PAT == PAT_816) {
+      *reinterpret_cast<uint16_t*>(p.bb_scales + tiled_sf_offset(r, 2 * u, s_bb)) = (uint16_t)(bsc | (bsc << 8));
+    } else {
+      p.bb_scales[tiled_sf_offset(r, u, s_bb)] = (uint8_t)bsc;
+    }
+    *reinterpret_cast<uint16_t*>(p.res_scales + tiled_sf_offset(r, 2 * u, s_res)) = (uint16_t)(rsc0 | (rsc1 << 8));
+  } else {
+    if constexpr (PAT == PAT_816) {
+      p.bb_scales[tiled_sf_offset(r, u, s_bb)] = (uint8_t)bsc;
+    } else {
+      if ((u & 1) == 0) p.bb_scales[tiled_sf_offset(r, u >> 1, s_bb)] = (uint8_t)bsc;
+    }
+    p.res_scales[tiled_sf_offset(r, u, s_res)] = (uint8_t)rsc0;
+  }
+}
+
 template <int FMT, int PAT, bool NORM, bool XBF16, bool ACT = false>
 __global__ void __launch_bounds__(128, ACT ? 6 : 7) prep_kernel(PrepParams p) {
   static_assert(!(NORM && ACT), "the SwiGLU form has no RMSNorm");
@@ -887,32 +921,7 @@ __global__ void __launch_bounds__(128, ACT ? 6 : 7) prep_kernel(PrepParams p) {
       quantize_unit<FMT, PAT>(h, g_enc, g_dec, inv_tab, meta, bc, bsc, rc, rsc0, rsc1);
       if (!active || !in_pad) continue;
 
-      if constexpr (pair_layout(PAT)) {
-        *reinterpret_cast<uint16_t*>(p.meta + r * (k / 16) + 2 * u) = (uint16_t)meta;
-      } else {
-        *reinterpret_cast<uint32_t*>(p.meta + r * (k / 8) + 4 * u) = meta;
-      }
-      if constexpr (PAT == PAT_816) {
-        *reinterpret_cast<uint4*>(p.bb_codes + r * (k / 2) + 16 * u) = make_uint4(bc[0], bc[1], bc[2], bc[3]);
-      } else {
-        *reinterpret_cast<uint2*>(p.bb_codes + r * (k / 4) + 8 * u) = make_uint2(bc[0], bc[1]);
-      }
-      *reinterpret_cast<uint4*>(p.res_codes + r * (k / 2) + 16 * u) = make_uint4(rc[0], rc[1], rc[2], rc[3]);
-      if constexpr (FMT == FMT_NV) {
-        if constexpr (PAT == PAT_816) {
-          *reinterpret_cast<uint16_t*>(p.bb_scales + tiled_sf_offset(r, 2 * u, s_bb)) = (uint16_t)(bsc | (bsc << 8));
-        } else {
-          p.bb_scales[tiled_sf_offset(r, u, s_bb)] = (uint8_t)bsc;
-        }
-        *reinterpret_cast<uint16_t*>(p.res_scales + tiled_sf_offset(r, 2 * u, s_res)) = (uint16_t)(rsc0 | (rsc1 << 8));
-      } else {
-        if constexpr (PAT == PAT_816) {
-          p.bb_scales[tiled_sf_offset(r, u, s_bb)] = (uint8_t)bsc;
-        } else {
-          if ((u & 1) == 0) p.bb_scales[tiled_sf_offset(r, u >> 1, s_bb)] = (uint8_t)bsc;
-        }
-        p.res_scales[tiled_sf_offset(r, u, s_res)] = (uint8_t)rsc0;
-      }
+      store_unit<FMT, PAT>(p, r, u, s_bb, s_res, meta, bc, bsc, rc, rsc0, rsc1);
     }
   }
 }
