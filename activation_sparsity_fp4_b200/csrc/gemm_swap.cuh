@@ -172,11 +172,9 @@ __global__ void __launch_bounds__(192, 1) gemm_swap_kernel(const __grid_constant
       if (BL != SW_DENSE) tma_prefetch(&maps.e);
     }
     // while the kernel before this one finishes: warm L2 with this slice of the
-    // weight tile (the weight is not written by the preparation kernels)
-    const int64_t row_bytes = p.k / 2;
-    for (int r = lane; r < C::BM; r += 32)
-      if (n0 + r < p.n)
-        prefetch_l2(p.w_codes + (n0 + r) * row_bytes + (int64_t)k0 * 128, (uint32_t)((k1 - k0) * 128));
+    // weight tile, one box (the stage's 128 rows x 128 bytes) per lane (the
+    // weight is not written by the preparation kernels)
+    for (int kt = k0 + lane; kt < k1; kt += 32) tma_prefetch_l2_2d(&maps.w, kt * 128, (int32_t)n0);
   }
   tc_fence_before();
   __syncthreads();
@@ -352,20 +350,39 @@ __global__ void __launch_bounds__(192, 1) gemm_swap_kernel(const __grid_constant
           float f[TN];
 #pragma unroll
           for (int t = 0; t < TN; t++) f[t] = 0.0f;
-          for (int s = 0; s < p.split; s++) {
-            const float4* src = reinterpret_cast<const float4*>(p.acc + ((int64_t)s * p.n + n) * TN);
+          // slots in slice order, two slots' loads in flight at a time
+          auto add_slot = [&](const float4 (&a)[TN / 4], bool first) {
 #pragma unroll
             for (int j = 0; j < TN / 4; j++) {
-              const float4 a = __ldcg(src + j);
-              if (s == 0) {
-                f[4 * j] = a.x; f[4 * j + 1] = a.y; f[4 * j + 2] = a.z; f[4 * j + 3] = a.w;
+              if (first) {
+                f[4 * j] = a[j].x; f[4 * j + 1] = a[j].y; f[4 * j + 2] = a[j].z; f[4 * j + 3] = a[j].w;
               } else {
-                f[4 * j] = __fadd_rn(f[4 * j], a.x);
-                f[4 * j + 1] = __fadd_rn(f[4 * j + 1], a.y);
-                f[4 * j + 2] = __fadd_rn(f[4 * j + 2], a.z);
-                f[4 * j + 3] = __fadd_rn(f[4 * j + 3], a.w);
+                f[4 * j] = __fadd_rn(f[4 * j], a[j].x);
+                f[4 * j + 1] = __fadd_rn(f[4 * j + 1], a[j].y);
+                f[4 * j + 2] = __fadd_rn(f[4 * j + 2], a[j].z);
+                f[4 * j + 3] = __fadd_rn(f[4 * j + 3], a[j].w);
               }
             }
+          };
+          int s = 0;
+          for (; s + 1 < p.split; s += 2) {
+            const float4* s0 = reinterpret_cast<const float4*>(p.acc + ((int64_t)s * p.n + n) * TN);
+            const float4* s1 = reinterpret_cast<const float4*>(p.acc + ((int64_t)(s + 1) * p.n + n) * TN);
+            float4 a0[TN / 4], a1[TN / 4];
+#pragma unroll
+            for (int j = 0; j < TN / 4; j++) {
+              a0[j] = __ldcg(s0 + j);
+              a1[j] = __ldcg(s1 + j);
+            }
+            add_slot(a0, s == 0);
+            add_slot(a1, false);
+          }
+          if (s < p.split) {
+            const float4* s0 = reinterpret_cast<const float4*>(p.acc + ((int64_t)s * p.n + n) * TN);
+            float4 a0[TN / 4];
+#pragma unroll
+            for (int j = 0; j < TN / 4; j++) a0[j] = __ldcg(s0 + j);
+            add_slot(a0, s == 0);
           }
           store_y(f);
           if (q == 0 && lane == 0) p.cnt[tile] = 0u;  // the counter as it was found
