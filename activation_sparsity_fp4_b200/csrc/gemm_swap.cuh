@@ -12,8 +12,8 @@
 // viewed per b) and both products run as dense block-scaled MMAs into one
 // tensor-memory accumulator; at this size their cost is far below the weight
 // stream's.  The K loop of each 128-row weight tile is split into slices on
-// different SMs (with a workspace), slices summed in slice order by the CTA
-// that completes the tile's last one.
+// different SMs that form one thread-block cluster; the cluster's first CTA
+// sums the slices in slice order through distributed shared memory.
 //
 // Per CTA (192 threads, one work item = one weight tile x one K slice):
 //   warp 0      TMA producer: weight tile, residual rows, backbone rows (compressed,
@@ -22,7 +22,8 @@
 //   warps 2-5   per stage: the backbone expanded into its swizzled dense tile,
 //               the scale chunks into the stage's tensor-memory slot (one warp per
 //               32-lane quadrant, warp % 4); at the end the accumulator drain (lane = weight
-//               row, column = activation row) into y or the slice's workspace slot.
+//               row, column = activation row) into y, or into shared memory for the
+//               cluster's first CTA.
 // Every wait is bounded in time and reports through the device error word.
 #pragma once
 #include <cuda_bf16.h>
@@ -71,7 +72,7 @@ struct SwapCfg {
 struct SwapParams {
   int64_t t, n, k;          // activation rows (<= TN), weight rows, K
   int64_t k_tiles;          // K tiles of 256
-  int32_t split;            // K slices per weight tile (1 = no workspace)
+  int32_t split;            // K slices per weight tile = CTAs per cluster (1: no split)
   const uint8_t* w_codes;   // weight codes [n][k / 2] (L2 warm-up only)
   const uint8_t* sf_w;      // weight scales, dense view, tiled
   const uint8_t* sf_res;    // activation scales, tiled (rows of the first 128-row block)
@@ -81,8 +82,6 @@ struct SwapParams {
   void* y;
   int y_bf16;
   uint64_t timeout_ns;
-  float* acc;               // split > 1: slot per slice, [n][TN] fp32 raw sums
-  uint32_t* cnt;            // split > 1: one counter per weight tile
 };
 
 struct SwapMaps {
@@ -136,13 +135,11 @@ __global__ void __launch_bounds__(192, 1) gemm_swap_kernel(const __grid_constant
   uint64_t* ready = empty + C::kStages;  // backbone expanded, scales in tensor memory
   uint64_t* acc_full = ready + C::kStages;
   uint64_t* drain = acc_full + 1;
-  uint64_t* ep_bar = drain + 1;          // split: the 4 drain warps have written their slice
-  uint64_t* verdict = ep_bar + 1;        // split: `last` is set
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(verdict + 1);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  volatile uint32_t* last = reinterpret_cast<volatile uint32_t*>(tmem_holder + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // work item: weight tile blockIdx / split, K slice = rank in the cluster of split CTAs
   const int tile = (int)(blockIdx.x / p.split), slice = (int)(blockIdx.x % p.split);
   const int k0 = (int)((int64_t)slice * p.k_tiles / p.split), k1 = (int)((int64_t)(slice + 1) * p.k_tiles / p.split);
   const int64_t n0 = (int64_t)tile * C::BM;
@@ -155,8 +152,6 @@ __global__ void __launch_bounds__(192, 1) gemm_swap_kernel(const __grid_constant
     }
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
-    mbar_init(ep_bar, 4);
-    mbar_init(verdict, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -183,6 +178,7 @@ __global__ void __launch_bounds__(192, 1) gemm_swap_kernel(const __grid_constant
   grid_dep_wait();  // the prepared rows are complete
 
   const int64_t sw_blocks = (p.k / C::kVec + 3) / 4;  // 512-byte chunks per 128-row block of the weight scales
+  float f[TN];  // drain warps: this CTA's raw sums of its row (lane) for each activation row
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -304,95 +300,59 @@ __global__ void __launch_bounds__(192, 1) gemm_swap_kernel(const __grid_constant
       if (++stage == C::kStages) { stage = 0; phase ^= 1; }
     }
     // drain: lane = weight row n0 + 32 q + lane, column = activation row
-    if (!*abort_flag && mbar_wait(acc_full, 0, p.timeout_ns, abort_flag)) {
+    if (!*abort_flag && !mbar_wait(acc_full, 0, p.timeout_ns, abort_flag)) *abort_flag = 1;
+    if (!*abort_flag) {
       tc_fence_after();
       uint32_t v[TN];
       tmem_ld32_nowait(tq, *reinterpret_cast<uint32_t(*)[32]>(v));
       if constexpr (TN == 64) tmem_ld32_nowait(tq + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
       tmem_ld_wait();
-      const int64_t n = n0 + 32 * q + lane;
-      const float alpha = __fmul_rn(__ldg(p.tensor_x + 2), __ldg(p.tensor_w + 2));
-      auto store_y = [&](const float (&f)[TN]) {
-        if (n >= p.n) return;
 #pragma unroll
-        for (int t = 0; t < TN; t++) {  // lanes write consecutive n of row t
-          if (t >= p.t) break;
-          const float yv = __fmul_rn(f[t], alpha);
-          if (p.y_bf16) reinterpret_cast<__nv_bfloat16*>(p.y)[t * p.n + n] = __float2bfloat16_rn(yv);
-          else reinterpret_cast<float*>(p.y)[t * p.n + n] = yv;
-        }
-      };
-      if (p.split <= 1) {
-        float f[TN];
+      for (int t = 0; t < TN; t++) f[t] = __uint_as_float(v[t]);
+      if (p.split > 1 && slice != 0) {
+        // this slice's raw sums for the cluster's first CTA: column-major
+        // [TN][128] fp32 in the (now idle) stage buffers, consecutive lanes on
+        // consecutive words
+        float* part = reinterpret_cast<float*>(smem);
 #pragma unroll
-        for (int t = 0; t < TN; t++) f[t] = __uint_as_float(v[t]);
-        store_y(f);
-      } else {
-        // this slice's raw sums into its slot, then the CTA that completes the
-        // tile's last slice adds the slots in slice order
-        float4* mine = reinterpret_cast<float4*>(p.acc + ((int64_t)slice * p.n + n) * TN);
-#pragma unroll
-        for (int j = 0; j < TN / 4; j++)
-          __stcg(mine + j, make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                       __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3])));
-        __threadfence();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(ep_bar);
-        if (q == 0 && lane == 0) {
-          if (mbar_wait(ep_bar, 0, p.timeout_ns, abort_flag))
-            *last = atomicAdd(p.cnt + tile, 1u) == (uint32_t)(p.split - 1) ? 1u : 0u;
-          else
-            *last = 0u;
-          mbar_arrive(verdict);
-        }
-        if (mbar_wait(verdict, 0, p.timeout_ns, abort_flag) && *last) {
-          __threadfence();
-          float f[TN];
-#pragma unroll
-          for (int t = 0; t < TN; t++) f[t] = 0.0f;
-          // slots in slice order, two slots' loads in flight at a time
-          auto add_slot = [&](const float4 (&a)[TN / 4], bool first) {
-#pragma unroll
-            for (int j = 0; j < TN / 4; j++) {
-              if (first) {
-                f[4 * j] = a[j].x; f[4 * j + 1] = a[j].y; f[4 * j + 2] = a[j].z; f[4 * j + 3] = a[j].w;
-              } else {
-                f[4 * j] = __fadd_rn(f[4 * j], a[j].x);
-                f[4 * j + 1] = __fadd_rn(f[4 * j + 1], a[j].y);
-                f[4 * j + 2] = __fadd_rn(f[4 * j + 2], a[j].z);
-                f[4 * j + 3] = __fadd_rn(f[4 * j + 3], a[j].w);
-              }
-            }
-          };
-          int s = 0;
-          for (; s + 1 < p.split; s += 2) {
-            const float4* s0 = reinterpret_cast<const float4*>(p.acc + ((int64_t)s * p.n + n) * TN);
-            const float4* s1 = reinterpret_cast<const float4*>(p.acc + ((int64_t)(s + 1) * p.n + n) * TN);
-            float4 a0[TN / 4], a1[TN / 4];
-#pragma unroll
-            for (int j = 0; j < TN / 4; j++) {
-              a0[j] = __ldcg(s0 + j);
-              a1[j] = __ldcg(s1 + j);
-            }
-            add_slot(a0, s == 0);
-            add_slot(a1, false);
-          }
-          if (s < p.split) {
-            const float4* s0 = reinterpret_cast<const float4*>(p.acc + ((int64_t)s * p.n + n) * TN);
-            float4 a0[TN / 4];
-#pragma unroll
-            for (int j = 0; j < TN / 4; j++) a0[j] = __ldcg(s0 + j);
-            add_slot(a0, s == 0);
-          }
-          store_y(f);
-          if (q == 0 && lane == 0) p.cnt[tile] = 0u;  // the counter as it was found
-        }
+        for (int t = 0; t < TN; t++) part[t * C::BM + 32 * q + lane] = f[t];
       }
     }
   }
 
+  // Split K: the K slices of a weight tile are the CTAs of one cluster.  After
+  // the first cluster barrier every slice's raw sums are in its shared memory;
+  // the first CTA adds them in slice order (a fixed order) through distributed
+  // shared memory and stores y; the second barrier keeps the other CTAs (and
+  // their shared memory) alive until it has read them.
   tc_fence_before();
   __syncthreads();
+  __syncwarp();
+  if (p.split > 1) cluster_sync_all();
+  if (warp >= 2 && (p.split <= 1 || slice == 0) && !*abort_flag) {
+    const int q = warp & 3;
+    const int64_t n = n0 + 32 * q + lane;
+    if (p.split > 1) {
+      const uint32_t part = smem_u32(smem) + (uint32_t)((32 * q + lane) * 4);
+      for (int r = 1; r < p.split; r++) {
+        const uint32_t peer = mapa_u32(part, (uint32_t)r);
+#pragma unroll
+        for (int t = 0; t < TN; t++) f[t] = __fadd_rn(f[t], ld_cluster_f32(peer + (uint32_t)(t * C::BM * 4)));
+      }
+    }
+    const float alpha = __fmul_rn(__ldg(p.tensor_x + 2), __ldg(p.tensor_w + 2));
+    if (n < p.n) {
+#pragma unroll
+      for (int t = 0; t < TN; t++) {  // lanes write consecutive n of row t
+        if (t >= p.t) break;
+        const float yv = __fmul_rn(f[t], alpha);
+        if (p.y_bf16) reinterpret_cast<__nv_bfloat16*>(p.y)[t * p.n + n] = __float2bfloat16_rn(yv);
+        else reinterpret_cast<float*>(p.y)[t * p.n + n] = yv;
+      }
+    }
+  }
+  __syncwarp();
+  if (p.split > 1) cluster_sync_all();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();

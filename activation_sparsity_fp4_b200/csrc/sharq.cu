@@ -151,6 +151,28 @@ int sm_count() {
   return n > 0 ? n : 148;
 }
 
+// Clusters of `csize` CTAs of this kernel that can be resident at once (0 on error).
+template <typename Kern>
+int max_active_clusters(Kern kern, int threads, size_t smem, int csize) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)csize);
+  cfg.blockDim = dim3((unsigned)threads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)csize;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -499,8 +521,7 @@ sharq_status run_gemv(const sharq_prepared* a, const sharq_weight* w, void* y, s
 // 36.0 us), so it serves 2..32 rows.
 constexpr int64_t kSwapMinRows = 2, kSwapMaxRows = 32;
 template <int KIND, int BL, int TN>
-sharq_status launch_swap(const sharq_prepared* a, const sharq_weight* w, void* y, sharq_dtype y_dt, void* ws,
-                         size_t ws_bytes, cudaStream_t s) {
+sharq_status launch_swap(const sharq_prepared* a, const sharq_weight* w, void* y, sharq_dtype y_dt, cudaStream_t s) {
   using C = SwapCfg<KIND, BL, TN>;
   static bool configured = false;
   if (!configured) {
@@ -540,41 +561,40 @@ sharq_status launch_swap(const sharq_prepared* a, const sharq_weight* w, void* y
   sp.timeout_ns = wait_timeout_ns();
   const int64_t tiles = w->n / C::BM;
   const int sms = sm_count();
+  // K slices per weight tile = CTAs per cluster: enough work items for every
+  // SM, at least two K tiles each, at most 8 (the portable cluster size), and
+  // only as many as let every cluster be resident at once
   int64_t split = 1;
-  if (ws && tiles <= sms) {
-    // slices: enough work items for every SM, at least two K tiles each, and one
-    // fp32 slot of [n][TN] raw sums per slice in the workspace
+  if (tiles <= sms) {
     split = sms / tiles;
     if (split > sp.k_tiles / 2) split = sp.k_tiles / 2;
-    const size_t slot = (size_t)w->n * TN * sizeof(float);
-    while (split > 1 && ws_data_offset() + (size_t)split * slot > ws_bytes) split--;
+    if (split > 8) split = 8;
+    static int resident[9] = {-1, -1, -1, -1, -1, -1, -1, -1, -1};  // clusters of each size (per device kind)
+    auto fits = [&](int64_t cs) {
+      if (resident[cs] < 0) resident[cs] = max_active_clusters(gemm_swap_kernel<KIND, BL, TN>, 192, C::kSmemBytes, (int)cs);
+      return resident[cs] >= tiles;
+    };
+    while (split > 1 && !fits(split)) split--;
     if (split < 1) split = 1;
   }
   sp.split = (int32_t)split;
-  if (split > 1) {
-    sp.acc = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + ws_data_offset());
-    sp.cnt = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + ws_split_cnt_offset());
-  }
-  return launch_ex(gemm_swap_kernel<KIND, BL, TN>, dim3((unsigned)(tiles * split)), dim3(192), C::kSmemBytes, s, 1,
-                   maps, sp);
+  return launch_ex(gemm_swap_kernel<KIND, BL, TN>, dim3((unsigned)(tiles * split)), dim3(192), C::kSmemBytes, s,
+                   (unsigned)split, maps, sp);
 }
 
 template <int KIND, int BL>
-sharq_status swap_rows(const sharq_prepared* a, const sharq_weight* w, void* y, sharq_dtype y_dt, void* ws,
-                       size_t ws_bytes, cudaStream_t s) {
+sharq_status swap_rows(const sharq_prepared* a, const sharq_weight* w, void* y, sharq_dtype y_dt, cudaStream_t s) {
   static_assert(kSwapMaxRows <= 32, "one activation tile width");
-  return launch_swap<KIND, BL, 32>(a, w, y, y_dt, ws, ws_bytes, s);
+  return launch_swap<KIND, BL, 32>(a, w, y, y_dt, s);
 }
 
-sharq_status run_swap(const sharq_prepared* a, const sharq_weight* w, void* y, sharq_dtype y_dt, void* ws,
-                      size_t ws_bytes, cudaStream_t s) {
+sharq_status run_swap(const sharq_prepared* a, const sharq_weight* w, void* y, sharq_dtype y_dt, cudaStream_t s) {
   const bool pair = a->pat == SHARQ_NM_4_8_PAIR || a->pat == SHARQ_NM_8_16_PAIR;
   if (a->fmt == SHARQ_NVFP4)
-    return pair ? swap_rows<GK_NVF4, SW_PAIR>(a, w, y, y_dt, ws, ws_bytes, s)
-                : swap_rows<GK_NVF4, SW_DENSE>(a, w, y, y_dt, ws, ws_bytes, s);
-  if (pair) return swap_rows<GK_MXF4, SW_PAIR>(a, w, y, y_dt, ws, ws_bytes, s);
-  return a->pat == SHARQ_NM_2_4 ? swap_rows<GK_MXF4, SW_24>(a, w, y, y_dt, ws, ws_bytes, s)
-                                : swap_rows<GK_MXF4, SW_DENSE>(a, w, y, y_dt, ws, ws_bytes, s);
+    return pair ? swap_rows<GK_NVF4, SW_PAIR>(a, w, y, y_dt, s) : swap_rows<GK_NVF4, SW_DENSE>(a, w, y, y_dt, s);
+  if (pair) return swap_rows<GK_MXF4, SW_PAIR>(a, w, y, y_dt, s);
+  return a->pat == SHARQ_NM_2_4 ? swap_rows<GK_MXF4, SW_24>(a, w, y, y_dt, s)
+                                : swap_rows<GK_MXF4, SW_DENSE>(a, w, y, y_dt, s);
 }
 
 sharq_status run_linear(const sharq_prepared* a, const sharq_weight* w, const int32_t* offsets, void* y,
@@ -598,7 +618,7 @@ sharq_status run_linear(const sharq_prepared* a, const sharq_weight* w, const in
   if (swap) {
     if (ws && (ws_bytes < sk_workspace_bytes() || !aligned(ws, 16)))
       return fail(SHARQ_ERR_WORKSPACE, "workspace: %zu bytes, 16-byte aligned, needed", sk_workspace_bytes());
-    return run_swap(a, w, y, y_dt, ws, ws_bytes, s);
+    return run_swap(a, w, y, y_dt, s);
   }
 
   const int64_t t_pad = round_up(a->t, 128);

@@ -215,10 +215,16 @@ sharq_status sharq_prepare_noalloc(const void* x, sharq_dtype x_dt, const void* 
  *   y[t][n] = g_dec_x * g_dec_w * sum_k (B[t][k] + R[t][k]) * W[n][k]
  * y: t * n row-major, dtype y_dt.  Supported: MXFP4 with every pattern, NVFP4 with
  * 4:8 pair and 8:16 (NVFP4 2:4 returns SHARQ_ERR_UNSUPPORTED: no sparse tensor-core
- * kind takes E4M3 block-16 scales with element-wise 2:4 metadata).  With t <= 4 the
+ * kind takes E4M3 block-16 scales with element-wise 2:4 metadata).  With t = 1 the
  * product is a weight stream and runs on the CUDA cores (same operands and output,
  * fp32 sums in another order; SHARQ_GEMV=0 in the environment keeps the tensor
- * cores). */
+ * cores).  With 2 <= t <= 32 the weight is the 128-row MMA operand and the rows the
+ * other one (the backbone expanded to its dense form on chip); each 128-row weight
+ * tile's K loop is split over the CTAs of one thread-block cluster (up to 8, as many
+ * as keep every cluster resident at once), whose first CTA adds the slices' fp32
+ * sums in slice order through distributed shared memory, so the results repeat bit
+ * for bit and no workspace is needed (SHARQ_SWAP=0 keeps the activation-as-A
+ * kernels). */
 sharq_status sharq_linear(const sharq_prepared* a, const sharq_weight* w, void* y, sharq_dtype y_dt,
                           sharq_stream stream);
 
