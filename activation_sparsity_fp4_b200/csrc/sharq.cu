@@ -93,7 +93,7 @@ bool gemv_enabled() {
   return v;
 }
 
-// SHARQ_SWAP=0 keeps few-row products (5..64 rows) on the activation-as-A kernels (for comparison).
+// SHARQ_SWAP=0 keeps few-row products (2..64 rows) on the activation-as-A kernels (for comparison).
 bool swap_enabled() {
   static const bool v = [] {
     const char* e = getenv("SHARQ_SWAP");
@@ -514,12 +514,12 @@ sharq_status run_gemv(const sharq_prepared* a, const sharq_weight* w, void* y, s
 }
 
 // Few rows: the weight as the 128-row MMA operand (gemm_swap.cuh), the K loop of
-// each 128-row weight tile split over the SMs when a workspace is given.
-// Measured on B200 (GEMM alone): down_proj 4 rows 42.9 -> 23.0 us, 16 rows 28.3
-// -> 23.2 us, q_proj 16 rows 22.8 -> 16.8 us; at 1 row the CUDA-core form is
-// faster (19.3 vs 23.4 us), at 64 rows the activation-as-A kernels (30.3 vs
-// 36.0 us), so it serves 2..32 rows.
-constexpr int64_t kSwapMinRows = 2, kSwapMaxRows = 32;
+// each 128-row weight tile split over the CTAs of a cluster.  Measured on B200
+// (GEMM alone, down_proj, back-to-back over rotating weights): 2 rows 16.2 us,
+// 16 rows 16.9 us, 33-64 rows 22.0-22.6 us against 27.7-28.2 us for the
+// activation-as-A split-K kernel; at 1 row the CUDA-core form is faster, so it
+// serves 2..64 rows (activation tiles of 32 or 64 columns).
+constexpr int64_t kSwapMinRows = 2, kSwapMaxRows = 64;
 template <int KIND, int BL, int TN>
 sharq_status launch_swap(const sharq_prepared* a, const sharq_weight* w, void* y, sharq_dtype y_dt, cudaStream_t s) {
   using C = SwapCfg<KIND, BL, TN>;
@@ -584,7 +584,8 @@ sharq_status launch_swap(const sharq_prepared* a, const sharq_weight* w, void* y
 
 template <int KIND, int BL>
 sharq_status swap_rows(const sharq_prepared* a, const sharq_weight* w, void* y, sharq_dtype y_dt, cudaStream_t s) {
-  static_assert(kSwapMaxRows <= 32, "one activation tile width");
+  static_assert(kSwapMaxRows <= 64, "activation tile widths 32 and 64");
+  if (a->t > 32) return launch_swap<KIND, BL, 64>(a, w, y, y_dt, s);
   return launch_swap<KIND, BL, 32>(a, w, y, y_dt, s);
 }
 

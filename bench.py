@@ -518,13 +518,13 @@ def measure(name: str, tokens, steps: int, warmup: int, e2e_steps: int, dev, pg,
     grouped = wl["offsets"] is not None
     kernel = {"4:8pair": "sparse", "8:16pair": "sparse", "2:4": "sparse", "8:16": "dense backbone"}[pat]
     kname = ("gemv_kernel" if (not grouped and T == 1) else
-             "gemm_swap_kernel" if (not grouped and 2 <= T <= 32) else
+             "gemm_swap_kernel" if (not grouped and 2 <= T <= 64) else
              "gemm_pair_kernel" if (not grouped and pat in ("4:8pair", "8:16pair")
                                     and ((T + 127) // 128 * 128) % 256 == 0)
              else "gemm_kernel")
     kkind = "MXF8" if (fmt == "mxfp4" and pat == "2:4") else ("NVF4" if fmt == "nvfp4" else "MXF4")
     klabel = (f"gemv_kernel<{'MX' if fmt == 'mxfp4' else 'NV'}, {pat}, {T} rows>" if kname == "gemv_kernel"
-              else f"gemm_swap_kernel<{'NVF4' if fmt == 'nvfp4' else 'MXF4'}, {pat} expanded, N=32>"
+              else f"gemm_swap_kernel<{'NVF4' if fmt == 'nvfp4' else 'MXF4'}, {pat} expanded, N={32 if T <= 32 else 64}>"
               if kname == "gemm_swap_kernel" else f"{kname}<{kkind}, {kernel}>")
     set_mb = L.set_bytes / 2 ** 20
     res = {

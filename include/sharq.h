@@ -218,8 +218,9 @@ sharq_status sharq_prepare_noalloc(const void* x, sharq_dtype x_dt, const void* 
  * kind takes E4M3 block-16 scales with element-wise 2:4 metadata).  With t = 1 the
  * product is a weight stream and runs on the CUDA cores (same operands and output,
  * fp32 sums in another order; SHARQ_GEMV=0 in the environment keeps the tensor
- * cores).  With 2 <= t <= 32 the weight is the 128-row MMA operand and the rows the
- * other one (the backbone expanded to its dense form on chip); each 128-row weight
+ * cores).  With 2 <= t <= 64 the weight is the 128-row MMA operand and the rows
+ * (padded to 32 or 64) the other one (the backbone expanded to its dense form on
+ * chip); each 128-row weight
  * tile's K loop is split over the CTAs of one thread-block cluster (up to 8, as many
  * as keep every cluster resident at once), whose first CTA adds the slices' fp32
  * sums in slice order through distributed shared memory, so the results repeat bit

@@ -106,10 +106,13 @@ def test_stream_k_falls_back_where_it_does_not_apply(cuda_ok):
     assert (_flags(ws) == 0).all()
 
 
-# single-CTA kernel, few tiles with long K (decode-size row counts): K split
-# into slices over the SMs, slices summed in a fixed order by the last one
+# few tiles with long K (decode-size row counts), K split into slices over the
+# SMs and the slices summed in a fixed order: 65..256 rows on the single-CTA
+# kernel (workspace slots, the last slice adds them), 2..64 rows on the few-row
+# kernel (a cluster per weight tile), 1 row on the CUDA cores
 SPLIT_CASES = [("mxfp4", "2:4", 1, 4096, 14336), ("mxfp4", "2:4", 16, 4096, 14336),
-               ("mxfp4", "2:4", 64, 4096, 14336), ("mxfp4", "2:4", 256, 4096, 14336),
+               ("mxfp4", "2:4", 64, 4096, 14336), ("mxfp4", "2:4", 128, 4096, 14336),
+               ("mxfp4", "2:4", 256, 4096, 14336),
                ("nvfp4", "4:8pair", 16, 4096, 8192), ("nvfp4", "8:16", 100, 1024, 8192),
                ("mxfp4", "4:8pair", 40, 2048, 8192)]
 
