@@ -254,13 +254,15 @@ __global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ Ge
   const int k_tiles = (int)(p.k / C::BK);
   if (warp == 0 && lane == 0 && p.experts <= 1 && (int)blockIdx.x < num_tiles) {
     // while the kernel before this one finishes: warm L2 with this CTA's share
-    // of the weight rows of its first tile (the CTAs on one column of tiles
-    // split them); the weight is not written by the preparation kernels
+    // of the weight tile of its first tile, whole TMA boxes (the CTAs on one
+    // column of tiles split its K tiles); the weight is not written by the
+    // preparation kernels
     const TileXY x = tile_xy((int)blockIdx.x, m_tiles, n_tiles, C::kBandTiles);
-    const int per = (C::BN + x.h - 1) / x.h, i = x.mt - x.lo;
-    const int64_t row_bytes = p.k / 2;
-    const uint8_t* w0 = static_cast<const uint8_t*>(p.w_codes) + ((int64_t)x.nt * C::BN + (int64_t)i * per) * row_bytes;
-    for (int r = 0; r < per && i * per + r < C::BN; r++) prefetch_l2(w0 + r * row_bytes, (uint32_t)row_bytes);
+    const int per = (k_tiles + x.h - 1) / x.h, i = x.mt - x.lo;
+    const int32_t wrow = (int32_t)((int64_t)x.nt * C::BN);
+    for (int kt = i * per; kt < (i + 1) * per && kt < k_tiles; kt++)
+#pragma unroll
+      for (int bx = 0; bx < C::kBoxesDense; bx++) tma_prefetch_l2_2d(&maps.w, kt * C::kXStage + 128 * bx, wrow);
   }
   grid_dep_wait();  // the prepared activations (and scales) are complete
   // work items: (tile, K slice) with SPLIT, else whole tiles

@@ -143,14 +143,14 @@ __global__ void __launch_bounds__(448, 1) gemm_pair_kernel(const __grid_constant
   const int k_tiles = (int)(p.k / C::BK);
   if (warp == 0 && lane == 0 && cluster < num_tiles) {
     // while the kernel before this one finishes: warm L2 with this CTA's share
-    // of the weight rows of its first tile (the pairs on one column of tiles
-    // split them); the weight is not written by the preparation kernels
+    // of the weight tile of its first tile, whole TMA boxes (the pairs on one
+    // column of tiles split its K tiles); the weight is not written by the
+    // preparation kernels
     const TileXY x = tile_xy(cluster, m_pairs, n_tiles, C::kBandTiles);
-    const int per = (C::BNh + x.h - 1) / x.h, i = x.mt - x.lo;
-    const int64_t row_bytes = p.k / 2;
-    const uint8_t* w0 = static_cast<const uint8_t*>(p.w_codes) +
-                        ((int64_t)x.nt * C::BN + C::BNh * (int64_t)rank + (int64_t)i * per) * row_bytes;
-    for (int r = 0; r < per && i * per + r < C::BNh; r++) prefetch_l2(w0 + r * row_bytes, (uint32_t)row_bytes);
+    const int per = (k_tiles + x.h - 1) / x.h, i = x.mt - x.lo;
+    const int32_t wrow = (int32_t)((int64_t)x.nt * C::BN + C::BNh * rank);
+    for (int kt = i * per; kt < (i + 1) * per && kt < k_tiles; kt++)
+      tma_prefetch_l2_2d(&maps.w, kt * C::kXStage, wrow);
   }
   grid_dep_wait();  // the prepared activations (and scales) are complete
 
