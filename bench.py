@@ -502,11 +502,18 @@ def measure(name: str, tokens, steps: int, warmup: int, e2e_steps: int, dev, pg,
     gemm_s = gemm_ms / 1e3
     work, kind, work_desc = gemm_roofline(wl)
     b_blk = 16 if fmt == "nvfp4" else 32
-    wbytes = (N * K / 2 + N * K / (2 * b_blk) * (2 if pat == "8:16" else 1)
+    experts = wl["w"].shape[0] if wl["offsets"] is not None else 1
+    # algorithmic bytes of one launch: every expert's weight codes and sparse-view
+    # scales once, the prepared rows (codes, scales, metadata) once, y (bf16) once
+    wbytes = (experts * (N * K / 2 + N * K / (2 * b_blk) * (2 if pat == "8:16" else 1))
               + prep_bytes_per_elem(fmt, pat, 0) * T * K + 2 * T * N)
     ratio = FP4_OVER_BF16 if kind == "fp4" else FP8_OVER_BF16
     peak = pk["bf16_tflops"] * ratio
     achieved = work / gemm_s / 1e12
+    # roofline time = max(compute at the tensor peak, bytes at the HBM peak)
+    t_compute_us = work / (peak * 1e12) * 1e6
+    t_bytes_us = wbytes / (pk["hbm_gbs"] * 1e9) * 1e6
+    hbm_bound = t_bytes_us > t_compute_us
     bpe = prep_bytes_per_elem(fmt, pat, 4 if (L.swiglu or L.x_dt == torch.float32) else 2)
     prep_bytes = bpe * T * K
     if L.gemm_gather:  # prep of the tokens only (the GEMM reads the routed rows by index)
@@ -541,15 +548,19 @@ def measure(name: str, tokens, steps: int, warmup: int, e2e_steps: int, dev, pg,
                       "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
                       "frac": round(achieved / peak, 4), "traffic": None,
                       "peak_source": f"{src}: bf16 burst x {ratio:g} (nominal {kind.upper()}/BF16)",
-                      "work": work_desc, "avg_launch_us": round(gemm_s * 1e6, 2)}
-                     if T > 64 else
-                     # decode-size rows: the GEMM streams the weight; HBM bound
+                      "work": work_desc, "avg_launch_us": round(gemm_s * 1e6, 2),
+                      "t_compute_us": round(t_compute_us, 2), "t_bytes_us": round(t_bytes_us, 2)}
+                     if not hbm_bound else
+                     # the bytes take longer than the arithmetic at peak (decode-size rows,
+                     # short-K layers with many experts' weights): HBM bound
                      {"bound": "hbm", "kernel": klabel,
                       "achieved": round(wbytes / gemm_s / 1e9, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                       "frac": round(wbytes / gemm_s / 1e9 / pk["hbm_gbs"], 4), "traffic": None,
                       "peak_source": src,
-                      "work": "weight codes N*K/2 + sparse-view scales N*K/(2b) + prepared X + y bytes",
-                      "avg_launch_us": round(gemm_s * 1e6, 2)}),
+                      "work": ("weight codes E*N*K/2 + sparse-view scales E*N*K/(2b) (E experts) + prepared X "
+                               "+ y bytes"),
+                      "avg_launch_us": round(gemm_s * 1e6, 2),
+                      "t_compute_us": round(t_compute_us, 2), "t_bytes_us": round(t_bytes_us, 2)}),
         "prep": {"gbs_device_amax": round(prep_gbs, 1), "gbs_given_amax": round(given_gbs, 1),
                  "peak_gbs": pk["hbm_gbs"], "frac_given_amax": round(given_gbs / pk["hbm_gbs"], 4),
                  "frac_device_amax": round(prep_gbs / pk["hbm_gbs"], 4),
