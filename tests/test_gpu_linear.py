@@ -313,3 +313,25 @@ def test_linear_few_rows_weight_as_operand_a(cuda_ok, fmt, pat, t, k):
     if t <= 64:
         assert torch.equal(y1, y2), "the few-row kernel must not depend on the workspace"
     assert torch.equal(yb, y2.to(torch.bfloat16)), "bf16 output != fp32 output rounded to bf16"
+
+
+# cluster sizes of the few-row kernel's K split: slices = min(SMs / weight tiles,
+# K tiles / 2, 8), fewer when not every cluster would be resident at once
+CLUSTER_CASES = [(1024, 4096, 8), (5120, 2048, 3), (2048, 1024, 2)]
+
+
+@pytest.mark.parametrize("n,k,slices", CLUSTER_CASES)
+def test_few_rows_cluster_sizes(cuda_ok, n, k, slices):
+    """16 rows, MXFP4 2:4: the K slices of each weight tile summed in slice order
+    inside a cluster of 8, 3 and 2 CTAs (on a 148-SM part), against fp64; two
+    calls give the same bits."""
+    t = 16
+    x, w = _x(70 + slices, t, k), _w(71, n, k)
+    p = gpu_prepare(x, "bf16", "mxfp4", "2:4")
+    wq = gpu_weight(w, "bf16", "mxfp4")
+    y1 = sharq.linear(p, wq, out_dtype=torch.float32).clone()
+    y2 = sharq.linear(p, wq, out_dtype=torch.float32).clone()
+    sharq.sharq_sync_status()
+    prep, wqo = _ref(x, w, "mxfp4", "2:4")
+    assert_close_gemm(y1.cpu().numpy(), oracle.linear_ref(prep, wqo), f"n={n} k={k}, {slices} slices")
+    assert torch.equal(y1, y2)
