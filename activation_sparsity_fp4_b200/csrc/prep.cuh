@@ -163,6 +163,12 @@ __device__ __forceinline__ uint32_t ge_mask(float a, float b) {
   asm("set.ge.u32.f32 %0, %1, %2;" : "=r"(r) : "f"(a), "f"(b));
   return r;
 }
+// 0xFFFFFFFF if a > b, else 0.
+__device__ __forceinline__ uint32_t gt_mask(float a, float b) {
+  uint32_t r;
+  asm("set.gt.u32.f32 %0, %1, %2;" : "=r"(r) : "f"(a), "f"(b));
+  return r;
+}
 __device__ __forceinline__ uint32_t maj3(uint32_t a, uint32_t b, uint32_t c) { return (a & b) | (c & (a | b)); }
 // The same top-2-of-4 rule as four masks (0 or ~0), from bitwise majorities of
 // the comparison masks: entry p wins against q < p when s_p > s_q and against
@@ -213,21 +219,28 @@ __device__ __forceinline__ uint32_t unit_mask(const float (&h)[32], uint32_t& me
       keep |= kg << (4 * g);
     }
   } else {
+    // each of the 120 pairs (i < j) of a group of 16 compared once: j beats i
+    // if |h_j| > |h_i|, otherwise i beats j (equal magnitudes: the lower index)
 #pragma unroll
     for (int g = 0; g < 2; g++) {
-      uint32_t kg = 0;
+      float a[16];
+      int rank[16];
 #pragma unroll
       for (int i = 0; i < 16; i++) {
-        const float ai = fabsf(h[16 * g + i]);
-        int beat = 0;
-#pragma unroll
-        for (int j = 0; j < 16; j++) {
-          const float aj = fabsf(h[16 * g + j]);
-          if (j < i) beat += (aj >= ai) ? 1 : 0;
-          if (j > i) beat += (aj > ai) ? 1 : 0;
-        }
-        kg |= (beat < 8 ? 1u : 0u) << i;
+        a[i] = fabsf(h[16 * g + i]);
+        rank[i] = 0;
       }
+#pragma unroll
+      for (int i = 0; i < 16; i++)
+#pragma unroll
+        for (int j = i + 1; j < 16; j++) {
+          const int m = (int)gt_mask(a[j], a[i]);  // -1: j beats i, 0: i beats j
+          rank[i] -= m;
+          rank[j] += 1 + m;
+        }
+      uint32_t kg = 0;
+#pragma unroll
+      for (int i = 0; i < 16; i++) kg |= (rank[i] < 8 ? 1u : 0u) << i;
       meta |= kg << (16 * g);
       keep |= kg << (16 * g);
     }
