@@ -163,12 +163,6 @@ __device__ __forceinline__ uint32_t ge_mask(float a, float b) {
   asm("set.ge.u32.f32 %0, %1, %2;" : "=r"(r) : "f"(a), "f"(b));
   return r;
 }
-// 0xFFFFFFFF if a > b, else 0.
-__device__ __forceinline__ uint32_t gt_mask(float a, float b) {
-  uint32_t r;
-  asm("set.gt.u32.f32 %0, %1, %2;" : "=r"(r) : "f"(a), "f"(b));
-  return r;
-}
 __device__ __forceinline__ uint32_t maj3(uint32_t a, uint32_t b, uint32_t c) { return (a & b) | (c & (a | b)); }
 // The same top-2-of-4 rule as four masks (0 or ~0), from bitwise majorities of
 // the comparison masks: entry p wins against q < p when s_p > s_q and against
@@ -195,6 +189,22 @@ __device__ __forceinline__ uint32_t pair_nibble(uint32_t kp) {
   return (uint32_t)(LUT >> (4 * kp)) & 15u;
 }
 
+// Sorts 8 values in descending order with a 19-comparator network (each
+// comparator: max to the lower position, min to the higher).
+__device__ __forceinline__ void sort8_desc(float (&v)[8]) {
+  auto ce = [&](int i, int j) {
+    const float hi = fmaxf(v[i], v[j]), lo = fminf(v[i], v[j]);
+    v[i] = hi;
+    v[j] = lo;
+  };
+  ce(0, 2); ce(1, 3); ce(4, 6); ce(5, 7);
+  ce(0, 4); ce(1, 5); ce(2, 6); ce(3, 7);
+  ce(0, 1); ce(2, 3); ce(4, 5); ce(6, 7);
+  ce(2, 4); ce(3, 5);
+  ce(1, 4); ce(3, 6);
+  ce(1, 2); ce(3, 4); ce(5, 6);
+}
+
 template <int PAT>
 __device__ __forceinline__ uint32_t unit_mask(const float (&h)[32], uint32_t& meta) {
   uint32_t keep = 0;
@@ -219,28 +229,41 @@ __device__ __forceinline__ uint32_t unit_mask(const float (&h)[32], uint32_t& me
       keep |= kg << (4 * g);
     }
   } else {
-    // each of the 120 pairs (i < j) of a group of 16 compared once: j beats i
-    // if |h_j| > |h_i|, otherwise i beats j (equal magnitudes: the lower index)
+    // top 8 of each group of 16 by magnitude, ties to the lower index: T, the
+    // 8th largest magnitude, is the smallest of max(A_i, B_(7-i)) over the two
+    // halves sorted in descending order (the first step of a bitonic merge);
+    // every magnitude above T is kept, and of those equal to T the ones with
+    // the lowest indices, as many as are still missing.  Equal to ranking each
+    // element against the other 15.
 #pragma unroll
     for (int g = 0; g < 2; g++) {
-      float a[16];
-      int rank[16];
+      float a[16], A[8], B[8];
+#pragma unroll
+      for (int i = 0; i < 16; i++) a[i] = fabsf(h[16 * g + i]);
+#pragma unroll
+      for (int i = 0; i < 8; i++) {
+        A[i] = a[i];
+        B[i] = a[8 + i];
+      }
+      sort8_desc(A);
+      sort8_desc(B);
+      float thr = fmaxf(A[0], B[7]);
+#pragma unroll
+      for (int i = 1; i < 8; i++) thr = fminf(thr, fmaxf(A[i], B[7 - i]));
+      uint32_t gt = 0, eq = 0;
 #pragma unroll
       for (int i = 0; i < 16; i++) {
-        a[i] = fabsf(h[16 * g + i]);
-        rank[i] = 0;
+        gt |= (a[i] > thr ? 1u : 0u) << i;
+        eq |= (a[i] == thr ? 1u : 0u) << i;
       }
+      const int need = 8 - __popc(gt);  // >= 1: at most 7 magnitudes exceed the 8th largest
+      uint32_t kg = gt;
 #pragma unroll
-      for (int i = 0; i < 16; i++)
-#pragma unroll
-        for (int j = i + 1; j < 16; j++) {
-          const int m = (int)gt_mask(a[j], a[i]);  // -1: j beats i, 0: i beats j
-          rank[i] -= m;
-          rank[j] += 1 + m;
-        }
-      uint32_t kg = 0;
-#pragma unroll
-      for (int i = 0; i < 16; i++) kg |= (rank[i] < 8 ? 1u : 0u) << i;
+      for (int q = 0; q < 8; q++) {  // the lowest `need` set bits of eq
+        const uint32_t low = eq & (0u - eq);
+        if (q < need) kg |= low;
+        eq ^= low;
+      }
       meta |= kg << (16 * g);
       keep |= kg << (16 * g);
     }
