@@ -145,3 +145,29 @@ def test_grouped_gather_rejects_on_host(L):
             sharq.sharq_linear_grouped_gather(tok, rows, routed, w, 16, 16, sharq.BF16, 0)
         assert ei.value.status == status, str(ei.value)
     assert sharq.sharq_launch_count() == before
+
+
+def test_empty_inputs_are_rejected_without_launch(L):
+    """Zero rows (and a non-positive row count in the size queries) is an argument
+    error on the host: prepare, linear, the grouped and gathered forms and the
+    row gather all refuse it before any launch."""
+    before = sharq.sharq_launch_count()
+    with pytest.raises(sharq.SharqError) as ei:
+        sharq.sharq_prepared_sizes(0, 256, "nvfp4", "4:8pair")
+    assert ei.value.status == 1
+    empty = sharq.sharq_prepared(16, 16, 16, 16, 16, 16, 0, 256, 1, 1)
+    wq = sharq.sharq_weight(16, 16, 16, 16, 256, 256, 1, 1)
+    with pytest.raises(sharq.SharqError) as ei:
+        sharq.sharq_prepare(16, sharq.BF16, None, 1e-6, 0.0, empty, None, 0, 0)
+    assert ei.value.status == 1
+    with pytest.raises(sharq.SharqError) as ei:
+        sharq.sharq_linear(empty, wq, 16, sharq.BF16, 0)
+    assert ei.value.status == 1
+    with pytest.raises(sharq.SharqError) as ei:
+        sharq.sharq_linear_grouped(empty, wq, 16, 16, sharq.BF16, 0)
+    assert ei.value.status == 1
+    ok = sharq.sharq_prepared(16, 16, 16, 16, 16, 16, 128, 256, 1, 1)
+    with pytest.raises(sharq.SharqError) as ei:
+        sharq.sharq_gather_prepared(ok, 16, empty, 0)
+    assert ei.value.status == 1
+    assert sharq.sharq_launch_count() == before
