@@ -8,6 +8,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <string>
 
@@ -240,11 +241,18 @@ struct RowLaunch {
   unsigned grid;
   int tpr;
 };
-template <typename Kern>
-RowLaunch row_launch(Kern kern, int64_t rows, int64_t k) {
-  static int per_sm = 0;
+// The occupancy is looked up once per kernel (a template argument, so that
+// kernels of one signature keep separate figures).
+template <auto Kern>
+RowLaunch row_launch(int64_t rows, int64_t k) {
+  static std::atomic<int> cached{0};
+  int per_sm = cached.load(std::memory_order_relaxed);
   if (per_sm == 0) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 128, 0) != cudaSuccess || per_sm < 1) per_sm = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, Kern, 128, 0) != cudaSuccess || per_sm < 1) {
+      (void)cudaGetLastError();
+      per_sm = 1;
+    }
+    cached.store(per_sm, std::memory_order_relaxed);
   }
   const int64_t cap = (int64_t)sm_count() * per_sm;
   const int tpr = rows_tpr(k / 32, rows, cap);
@@ -257,7 +265,7 @@ template <int FMT, int PAT, bool NORM, bool XBF16>
 sharq_status launch_prep(const PrepParams& pp, cudaStream_t s) {
   auto kern = prep_kernel<FMT, PAT, NORM, XBF16>;
   PrepParams q = pp;
-  const RowLaunch rl = row_launch(kern, pp.t_pad, pp.k);
+  const RowLaunch rl = row_launch<prep_kernel<FMT, PAT, NORM, XBF16>>(pp.t_pad, pp.k);
   q.tpr = rl.tpr;
   return launch_ex(kern, dim3(rl.grid), dim3(128), 0, s, 1, q);
 }
@@ -270,7 +278,7 @@ sharq_status launch_amax(const void* x, const void* gamma, float eps, int64_t t,
     return launched();
   }
   auto kern = amax_kernel<NORM, XBF16>;
-  const RowLaunch rl = row_launch(kern, t, k);
+  const RowLaunch rl = row_launch<amax_kernel<NORM, XBF16>>(t, k);
   kern<<<rl.grid, 128, 0, s>>>(x, gamma, eps, t, k, out, rstd_out, nullptr, rl.tpr);
   return launched();
 }
@@ -297,7 +305,7 @@ sharq_status prep_dispatch_p(const PrepParams& pp, int pat, bool norm, bool xbf1
 template <int FMT, int PAT, bool XBF16>
 sharq_status launch_prep_swiglu(const PrepParams& pp, cudaStream_t s) {
   auto kern = prep_kernel<FMT, PAT, false, XBF16, true>;
-  const RowLaunch rl = row_launch(kern, pp.t_pad, pp.k);
+  const RowLaunch rl = row_launch<prep_kernel<FMT, PAT, false, XBF16, true>>(pp.t_pad, pp.k);
   PrepParams q = pp;
   q.tpr = rl.tpr;
   return launch_ex(kern, dim3(rl.grid), dim3(128), 0, s, 1, q);
@@ -318,20 +326,30 @@ sharq_status swiglu_dispatch_p(const PrepParams& pp, int pat, bool xbf16, cudaSt
 template <bool XBF16>
 sharq_status launch_amax_swiglu(const void* gate, const void* up, int64_t t, int64_t k, float* out, cudaStream_t s) {
   auto kern = amax_kernel<false, XBF16, true>;
-  const RowLaunch rl = row_launch(kern, t, k);
+  const RowLaunch rl = row_launch<amax_kernel<false, XBF16, true>>(t, k);
   kern<<<rl.grid, 128, 0, s>>>(gate, nullptr, 0.0f, t, k, out, nullptr, up, rl.tpr);
   return launched();
+}
+
+// cudaFuncSetAttribute acts on the current device's context: a kernel's
+// dynamic shared-memory limit is raised once per (kernel, device).
+template <auto Kern>
+sharq_status ensure_smem_limit(int bytes) {
+  static std::atomic<uint64_t> done{0};  // bit d: set on device d
+  int dev = 0;
+  SHARQ_CUDA(cudaGetDevice(&dev));
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return SHARQ_OK;
+  SHARQ_CUDA(cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  if (bit) done.fetch_or(bit, std::memory_order_release);
+  return SHARQ_OK;
 }
 
 template <int KIND, bool SPARSE, bool SPLIT = false, bool GATHER = false>
 sharq_status launch_gemm(const GemmMaps& maps, const GemmParams& gp, cudaStream_t s) {
   using C = GemmCfg<KIND, SPARSE>;
-  static bool configured = false;
-  if (!configured) {
-    SHARQ_CUDA(cudaFuncSetAttribute(gemm_kernel<KIND, SPARSE, SPLIT, GATHER>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes));
-    configured = true;
-  }
+  sharq_status st = ensure_smem_limit<gemm_kernel<KIND, SPARSE, SPLIT, GATHER>>(C::kSmemBytes);
+  if (st != SHARQ_OK) return st;
   const int items = (int)(gp.t_pad / C::BM) * (int)(gp.n / C::BN) * (SPLIT ? gp.split : 1);
   const int sms = sm_count();
   dim3 grid(items < sms ? items : sms);
@@ -419,7 +437,7 @@ int pair_max_resident() {
   static int v = -1;
   if (v < 0) {
     using C = PairCfg<KIND>;
-    cudaFuncSetAttribute(gemm_pair_kernel<KIND, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (ensure_smem_limit<gemm_pair_kernel<KIND, true>>(C::kSmemBytes) != SHARQ_OK) return 0;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(sm_count() & ~1));
     cfg.blockDim = dim3(448);
@@ -445,14 +463,10 @@ int pair_max_resident() {
 template <int KIND>
 sharq_status launch_pair(const GemmMaps& maps, const GemmParams& gp, cudaStream_t s) {
   using C = PairCfg<KIND>;
-  static bool configured = false;
-  if (!configured) {
-    SHARQ_CUDA(cudaFuncSetAttribute(gemm_pair_kernel<KIND, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    C::kSmemBytes));
-    SHARQ_CUDA(cudaFuncSetAttribute(gemm_pair_kernel<KIND, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    C::kSmemBytes));
-    configured = true;
-  }
+  sharq_status st = ensure_smem_limit<gemm_pair_kernel<KIND, false>>(C::kSmemBytes);
+  if (st != SHARQ_OK) return st;
+  st = ensure_smem_limit<gemm_pair_kernel<KIND, true>>(C::kSmemBytes);
+  if (st != SHARQ_OK) return st;
   const int tiles = (int)(gp.t_pad / 256) * (int)(gp.n / C::BN);
   const int pairs = sm_count() / 2;
   int clusters = tiles < pairs ? tiles : pairs;
@@ -523,12 +537,8 @@ constexpr int64_t kSwapMinRows = 2, kSwapMaxRows = 64;
 template <int KIND, int BL, int TN>
 sharq_status launch_swap(const sharq_prepared* a, const sharq_weight* w, void* y, sharq_dtype y_dt, cudaStream_t s) {
   using C = SwapCfg<KIND, BL, TN>;
-  static bool configured = false;
-  if (!configured) {
-    SHARQ_CUDA(cudaFuncSetAttribute(gemm_swap_kernel<KIND, BL, TN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    C::kSmemBytes));
-    configured = true;
-  }
+  sharq_status st0 = ensure_smem_limit<gemm_swap_kernel<KIND, BL, TN>>(C::kSmemBytes);
+  if (st0 != SHARQ_OK) return st0;
   const int64_t t_pad = round_up(a->t, 128), k = w->k;
   SwapMaps maps;
   memset(&maps, 0, sizeof(maps));
