@@ -644,6 +644,17 @@ __device__ __forceinline__ uint32_t nibble_mask8(uint32_t keep8) {
   for (int i = 0; i < 8; i++) m |= ((keep8 >> i) & 1u) ? (0xFu << (4 * i)) : 0u;
   return m;
 }
+// The same mask by bit spreading: bit i is moved to position 4i in three
+// shift-or-mask steps, then each becomes a nibble by multiplying with 15 (no
+// carries: every nibble holds 0 or 1).  Fewer instructions; used by the 8:16
+// path, where it was measured faster (the 2:4 path keeps the loop above).
+__device__ __forceinline__ uint32_t nibble_spread8(uint32_t keep8) {
+  uint32_t x = keep8 & 0xFFu;
+  x = (x | (x << 12)) & 0x000F000Fu;
+  x = (x | (x << 6)) & 0x03030303u;
+  x = (x | (x << 3)) & 0x11111111u;
+  return x * 0xFu;
+}
 // Compact the codes of the two kept bytes (pairs p0 < p1) of a 4-byte word.
 __device__ __forceinline__ uint32_t compact_pairs(uint32_t w, uint32_t p0, uint32_t p1) {
   return __byte_perm(w, 0u, p0 | (p1 << 4) | 0x4400u);  // bytes p0, p1 -> positions 0, 1; zeros above
@@ -767,7 +778,7 @@ __device__ __forceinline__ void quantize_unit(float (&h)[32], float g_enc, float
 #pragma unroll
     for (int i = 0; i < 32; i++) bamax = fmaxf(bamax, fabsf(h[i]));
 #pragma unroll
-    for (int g = 0; g < 4; g++) keepw[g] = nibble_mask8((keep >> (8 * g)) & 0xFFu);
+    for (int g = 0; g < 4; g++) keepw[g] = nibble_spread8((keep >> (8 * g)) & 0xFFu);
   }
   // the group maximum is always kept, so the backbone block amax is the window amax
   if constexpr (FMT == FMT_MX) bamax = fmaxf(bamax, __shfl_xor_sync(0xffffffffu, bamax, 1));
